@@ -1,0 +1,388 @@
+#!/usr/bin/env python
+"""Benchmark of the FlashLoop lazy loop-r attention sublayer on B200.
+
+One step = loops 2..R (gate, gathered QKV + RoPE, residual quantisation,
+column selection, selected-column reconstruction, sparse attention update,
+gathered output projection) of one synthetic 32K-token sequence per GPU,
+from the untouched loop-1 state.  The metric is tokens/s = S * (R - 1) per
+sequence per step, summed over ranks (weak scaling: each rank owns its own
+sequence; there is no exchange between ranks).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl cuda|reference]
+
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workload import CONFIGS, make_hidden_states, make_weights  # noqa: E402
+
+METRIC = "loop-step tokens/s at S=32K,R=4; HBM GB/s and tensor-pipe % of B200 peak"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: d_model {cfg.d_model}, {cfg.n_heads} heads x {cfg.head_dim}, S {cfg.seq}, "
+            f"R {cfg.n_loops}, tau {cfg.tau}, top-k {cfg.k}/head, active "
+            f"{'/'.join(f'{int(f * 100)}%' for f in cfg.active_fracs)}, bits "
+            f"{'/'.join(str(b) for b in cfg.bits)}")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu)], stdout=open(self.path, "w"),
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, smax, reasons, power = [], [], set(), []
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [t.strip() for t in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        os.unlink(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax), "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power)}
+
+
+# ----------------------------------------------------------------------------- CUDA arm
+def attention_pairs(active, cols):
+    """Causal-valid (i, j, h) pairs: i active, j selected for head h, j <= i."""
+    return int(sum(np.searchsorted(c, active, side="right").sum() for c in cols))
+
+
+def run_cuda(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from cross_loop_sparse_b200 import flashloop as F
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg, b=rank)
+    to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    xs = [to_dev(x) for x in X]
+    wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
+    p = F.Params.from_config(cfg)
+    st = F.FlashLoopState(p, device=dev)
+    S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
+    k_new = torch.empty((S, d), dtype=torch.float32, device=dev)
+    v_new = torch.empty_like(k_new)
+    F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
+    torch.cuda.synchronize()
+
+    launches_per_step = 0
+    attn_events = []
+
+    def step(record):
+        nonlocal launches_per_step
+        n = 0
+        for r in range(2, R + 1):
+            act, n_act = st[f"active{r}"], st["n_active"][r - 1:]
+            prev = None if r == 2 else st[f"active{r - 1}"]
+            n_prev = None if r == 2 else st["n_active"][r - 2:]
+            F.flashloop_gate(p, xs[r - 1], xs[r - 2], prev, n_prev, p.capacity[r - 2] if r > 2 else S,
+                             act, st[f"slot{r}"], n_act, p.capacity[r - 1], st["workspace"], st["err"])
+            F.flashloop_qkv_gathered(p, xs[r - 1], act, n_act, p.capacity[r - 1], wqkv, st["rope_cs"],
+                                     st[f"q{st.q_slot(r)}"], k_new, v_new)
+            F.flashloop_kv_quant_residual(p, r, k_new, v_new, act, n_act, st)
+            n += 3
+            if F.flashloop_selection_loop(p, r) == r:
+                src = st["colmass0"] if r == 2 else st["colmass1"]
+                F.flashloop_topk_columns(p, src, None, 0, p.topk[r - 1], st[f"cols{r}"])
+                n += 1
+            F.flashloop_selcol_dequant(p, r, st)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            F.flashloop_sparse_attn_update(p, r, st, 0)
+            if record:
+                e1.record(stream)
+                attn_events.append((r, e0, e1))
+            F.flashloop_out_proj(p, st["O"], act, n_act, p.capacity[r - 1], wo, st["Y"])
+            n += 3
+        launches_per_step = n
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step(False)
+    torch.cuda.synchronize()
+    barrier()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local_rank)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = t0.elapsed_time(t1)
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    err = st.error_code()
+    if err != 0:
+        raise RuntimeError(f"device error word {err}")
+
+    # Algorithmic work of the dominant kernel (attention update): 8*dh FLOP
+    # per causal-valid (active row, selected column, head) pair.
+    pairs = {}
+    for r in range(2, R + 1):
+        n = int(st["n_active"][r - 1].item())
+        act = st[f"active{r}"][:n].cpu().numpy()
+        cols = st.cols_for_loop(r).cpu().numpy()
+        pairs[r] = attention_pairs(act, cols)
+    attn_ms = sum(e0.elapsed_time(e1) for _, e0, e1 in attn_events)
+    attn_flop = sum(8 * cfg.head_dim * pairs[r] for r, _, _ in attn_events)
+    peaks, peak_kind = load_peaks()
+    achieved = attn_flop / (attn_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4), "traffic": None,
+                "kernel": "attn_update_kernel (sparse attention update, loops 2..R)",
+                "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
+                "attn_ms_per_step": round(attn_ms / args.steps, 4),
+                "attn_share_of_step": round(attn_ms / ms, 4)}
+
+    # End to end through the public API with host buffers: H2D of the step's
+    # hidden states X_2..X_R from pinned memory, loop_step for loops 2..R,
+    # D2H of Y.
+    host_x = [torch.from_numpy(X[r - 1].view(np.int16)).view(torch.bfloat16).pin_memory()
+              for r in range(2, R + 1)]
+    host_y = torch.empty((S, d), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 10))
+
+    def e2e_step():
+        for i, r in enumerate(range(2, R + 1)):
+            xs[r - 1].copy_(host_x[i], non_blocking=True)
+        for r in range(2, R + 1):
+            F.flashloop_loop_step(p, r, xs[r - 1], xs[r - 2], wqkv, wo, st)
+        host_y.copy_(st["Y"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    barrier()
+
+    tokens = S * (R - 1) * world
+    ms_step = ms / args.steps
+    out = {
+        "metric": METRIC, "value": round(tokens / (ms_step * 1e-3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded workload generator; random-init weights of the stated shape)",
+        "config": {"workload": workload_desc(cfg),
+                   "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
+                   "parallelism": f"one sequence per GPU, {world} GPU(s), no exchange",
+                   "active_tokens": {f"loop{r}": int(st['n_active'][r - 1].item()) for r in range(2, R + 1)},
+                   "attention_pairs": {f"loop{r}": pairs[r] for r in range(2, R + 1)}},
+        "roofline": roofline,
+        "e2e": {"value": round(tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": (R - 1) * S * d * 2, "d2h_bytes_per_step": S * d * 2,
+                "steps": e2e_steps},
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clk,
+    }
+    return out
+
+
+# ----------------------------------------------------------------------------- oracle timing
+class OracleSample:
+    """The CPU oracle on a bounded sample of the workload: loops 2..R for the
+    given heads of one sequence, from a loop-1 state computed once (untimed).
+    A full step is extrapolated as the gate once, the per-head work times
+    H / len(heads), and the output projection from a 1024-row sample."""
+
+    def __init__(self, cfg, heads=(0,)):
+        import oracle as O
+        self.O = O
+        self.cfg, self.heads = cfg, list(heads)
+        self.W = make_weights(cfg)
+        self.X, _ = make_hidden_states(cfg)
+        self.base = O.OracleSequence(cfg, self.W, self.X, heads=self.heads, keep_history=False)
+        self.base.run_loop1()
+
+    def step(self):
+        import copy
+        O, cfg, X = self.O, self.cfg, self.X
+        orc = copy.deepcopy(self.base)
+        t_gate = t_loops = t_wo = 0.0
+        for r in range(2, cfg.n_loops + 1):
+            t = time.perf_counter()
+            O.gate(X[r - 1], X[r - 2], orc.active[r - 1], cfg.tau)
+            t_gate += time.perf_counter() - t
+            t = time.perf_counter()
+            orc.run_loop(r)
+            t_loops += time.perf_counter() - t
+            n = orc.active[r].size
+            rows = min(1024, n)
+            t = time.perf_counter()
+            O.out_projection(np.zeros((rows, cfg.d_model), np.uint16), self.W["wo"])
+            t_wo += (time.perf_counter() - t) * n / rows
+        t_head = max(t_loops - t_gate, 0.0)
+        t_est = t_gate + t_head * cfg.n_heads / len(self.heads) + t_wo
+        sample = (f"oracle loops 2..{cfg.n_loops} on {len(self.heads)} of {cfg.n_heads} heads of one "
+                  f"{cfg.seq}-token sequence: gate {t_gate:.2f} s (counted once), per-head work "
+                  f"{t_head:.2f} s (scaled x{cfg.n_heads / len(self.heads):g}), W_o from a 1024-row sample "
+                  f"{t_wo:.2f} s (scaled to the active rows)")
+        return t_est, sample
+
+    @staticmethod
+    def cores():
+        try:
+            from threadpoolctl import threadpool_info
+            n = sum(i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas")
+            return n or os.cpu_count()
+        except Exception:
+            return os.cpu_count()
+
+
+def run_reference(args, cfg):
+    """The reference arm: the CPU oracle as it stands, on a bounded sample per step."""
+    smp = OracleSample(cfg)
+    times, sample = [], ""
+    for i in range(args.warmup + args.steps):
+        t_est, sample = smp.step()
+        if i >= args.warmup:
+            times.append(t_est)
+    ms = statistics.mean(times) * 1e3
+    tokens = cfg.seq * (cfg.n_loops - 1)
+    val = tokens / (ms * 1e-3)
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(val, 2), "unit": "tokens/s", "n_gpus": 1,
+        "steps": len(times), "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_desc(cfg), "parallelism": "CPU oracle, host cores"},
+        "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": OracleSample.cores(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
+    ap.add_argument("--config", default="prefill_32k", choices=[k for k, c in CONFIGS.items() if not c.decode])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    cfg = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        print(json.dumps(run_reference(args, cfg)), flush=True)
+        return 0
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    out = run_cuda(args, cfg, rank, world, local_rank)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        t_est, sample = OracleSample(cfg).step()
+        out["cpu_baseline"] = {"value": round(cfg.seq * (cfg.n_loops - 1) / t_est, 2), "unit": "tokens/s",
+                               "cores": OracleSample.cores(), "kind": "oracle", "sample": sample}
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,226 @@
+/*
+ * flashloop.h -- C ABI of the FlashLoop lazy loop-r attention sublayer on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is defined by "FlashLoop: Fast and Memory-Efficient Looped
+ * Transformers via Lazy Updates" (Yang & Liu): token-sparse updates (§4.1,
+ * App. D.1), loop-aware sparse attention (§4.2, App. D.2), cross-loop KV
+ * residual quantisation (§4.3, App. D.3) and the GPU engine of App. G
+ * (active-token execution, fused projections, packed low-bit KV streams read
+ * directly by the attention kernels, fused decode selection).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never allocates, never frees and never synchronises the host.  Every
+ *    call is asynchronous on the given stream (a cudaStream_t passed as
+ *    void*, NULL = legacy default stream).
+ *  - bf16 tensors are passed as uint16_t bit patterns, fp16 scales likewise.
+ *  - Layouts are row-major.  Hidden states X are [S, d_model]; linear weights
+ *    are [out, in] (y = x W^T); head h owns columns [h*dh, (h+1)*dh).
+ *  - A loop r (1-based) indexes per-loop arrays at position r-1.
+ *  - Counts of active tokens stay on the device: each kernel reads them there
+ *    and sizes its grid by the host-known upper bound (the capacity).
+ *  - Return value: FLASHLOOP_OK or a negative flashloop_status.  Arguments
+ *    are checked before any launch; a failed check launches nothing.
+ *    Device-side checks (capacity overflow, an index outside [0, S)) set
+ *    *err_word to a non-zero FLASHLOOP_DEVERR_* code; the caller reads it
+ *    after synchronising.  Kernels never trap and never spin without bound.
+ *  - Supported shapes: head_dim in {64, 128}, d_model = n_heads * head_dim,
+ *    d_model % 128 == 0, bits in {8, 4, 2} (bits[0] must be 8),
+ *    1 <= topk <= S.  Anything else returns FLASHLOOP_ERR_UNSUPPORTED.
+ */
+#ifndef FLASHLOOP_H
+#define FLASHLOOP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FLASHLOOP_MAX_LOOPS 16
+#define FLASHLOOP_GROUP 32
+
+typedef enum flashloop_status {
+  FLASHLOOP_OK = 0,
+  FLASHLOOP_ERR_INVALID_ARG = -1, /* null pointer, bad loop index, sizes out of range */
+  FLASHLOOP_ERR_UNSUPPORTED = -2, /* shape or bit width outside the supported set */
+  FLASHLOOP_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+  FLASHLOOP_ERR_DEVICE = -4,      /* reported by flashloop_check_error_word */
+  FLASHLOOP_ERR_ARCH = -5         /* the current device is not sm_100 */
+} flashloop_status;
+
+/* Codes a kernel may leave in *err_word. */
+#define FLASHLOOP_DEVERR_CAPACITY 1 /* more active tokens than the loop's capacity */
+#define FLASHLOOP_DEVERR_INDEX 2    /* a token or column index outside [0, S) */
+
+/* Problem description.  Plain values, read on the host only. */
+typedef struct flashloop_params {
+  int32_t seq;      /* S: tokens of the sequence (prefill) or of the context (decode) */
+  int32_t d_model;  /* = n_heads * head_dim */
+  int32_t n_heads;
+  int32_t head_dim; /* 64 or 128 */
+  int32_t n_loops;  /* R, 1..FLASHLOOP_MAX_LOOPS */
+  int32_t batch;    /* decode: number of sequences; prefill: 1 */
+  float tau;        /* gate threshold on the relative L2 change */
+  float rope_theta; /* RoPE base (1e4) */
+  int32_t topk[FLASHLOOP_MAX_LOOPS];     /* column budget k_r per loop (loop 1 unused), non-increasing */
+  int32_t bits[FLASHLOOP_MAX_LOOPS];     /* code width per loop: bits[0] = 8 (base); 8, 4 or 2 after */
+  int32_t capacity[FLASHLOOP_MAX_LOOPS]; /* rows allocated for loop r's active list and residual stream */
+} flashloop_params;
+
+/* One quantised cache (K or V) of a sequence: the loop-1 base over every
+ * token and, for loops r >= 2, a residual stream over the loop's active
+ * tokens only, stored at the token's position in the active list.
+ * Groups are 32 consecutive head_dim elements of one (token, head); a code is
+ * two's complement; INT4 packs element 2t in the low nibble of byte t, INT2
+ * element 4t+u in bits [2u, 2u+1] of byte t. */
+typedef struct flashloop_kv {
+  int8_t* base_codes;                          /* [S, H, dh] */
+  uint16_t* base_scales;                       /* [S, H, dh/32] fp16 */
+  uint8_t* res_codes[FLASHLOOP_MAX_LOOPS];     /* loop r: [capacity_r, H, dh*bits_r/8] */
+  uint16_t* res_scales[FLASHLOOP_MAX_LOOPS];   /* loop r: [capacity_r, H, dh/32] fp16 */
+} flashloop_kv;
+
+/* Whole per-sequence state of the sublayer (all device memory, caller-owned;
+ * a checkpoint is a copy of these buffers).
+ * Slots: q, m, Z and N have three slots.  Loop 1 writes slot 0; loop r >= 2
+ * reads slot sel(r-1) and writes slot sel(r), sel(r) = 1 + (r % 2), so the
+ * loop-1 state is never overwritten and loops 2..R can be re-run. */
+typedef struct flashloop_state {
+  flashloop_kv k;
+  flashloop_kv v;
+  int32_t* active[FLASHLOOP_MAX_LOOPS]; /* loop r: ascending active tokens, first n_r valid, [capacity_r] */
+  int32_t* slot[FLASHLOOP_MAX_LOOPS];   /* loop r: [S] position of the token in active[r-1], -1 if inactive */
+  int32_t* n_active;                    /* [FLASHLOOP_MAX_LOOPS] device counts n_r */
+  uint16_t* q[3];                       /* bf16 [S, H, dh] query slots */
+  float* m[3];                          /* [H, S] running max */
+  float* Z[3];                          /* [H, S] running denominator */
+  float* N[3];                          /* [H, S, dh] running numerator */
+  float* colmass[2];                    /* [H, S]: [0] dense loop-1 column mass, [1] latest sparse loop's */
+  int32_t* cols[FLASHLOOP_MAX_LOOPS];   /* loop r: [H, k_r] ascending selected columns (loops that select) */
+  uint16_t* O;                          /* bf16 [S, d_model] attention output (rows of inactive tokens kept) */
+  uint16_t* Y;                          /* bf16 [S, d_model] output projection (rows of inactive tokens kept) */
+  float* rope_cs;                       /* [S, dh/2] (cos, sin) pairs, see flashloop_rope_table */
+  int32_t* err_word;                    /* device error word, 0 = no error */
+  void* workspace;                      /* scratch, zero-filled once before first use */
+  size_t workspace_bytes;               /* >= flashloop_workspace_bytes(params) */
+} flashloop_state;
+
+/* ---------------------------------------------------------------- sizing */
+
+/* Scratch bytes the calls below need in state->workspace (host function). */
+size_t flashloop_workspace_bytes(const flashloop_params* p);
+
+/* Cache bytes of K and V for the given active counts n_r (n[0] = S):
+ * base 2*S*H*(dh + 2*dh/32) plus, per loop r >= 2, 2*n_r*H*(dh*bits_r/8 + 2*dh/32).
+ * Byte accounting of the cross-loop KV store ([FlashLoop §4.3, App. D.3]). */
+size_t flashloop_cache_bytes(const flashloop_params* p, const int32_t* n_per_loop);
+
+/* Fill the RoPE table: cs[2*(t*dh/2 + i)] = cos(t * theta^(-2i/dh)),
+ * cs[2*(...)+1] = sin(...), for t < n_pos, computed in double precision and
+ * rounded to float.  Rotate-half pairing (i, i + dh/2). */
+int flashloop_rope_table(const flashloop_params* p, int32_t n_pos, float* cs, void* stream);
+
+/* ---------------------------------------------------------------- the path */
+
+/* (a1) Token change gate and stream compaction [FlashLoop §3.1, §4.1, App. D.1].
+ * For the n_prev candidates prev_active[0..n_prev) (ascending), a token is
+ * active iff sum_c (x_cur - x_prev)^2 >= tau^2 * sum_c x_prev^2 (float32
+ * sums).  Writes the ascending active tokens to active_out, their positions
+ * to slot_out (every one of the S entries is written, -1 = inactive) and
+ * the count to *n_active_out.  prev_capacity bounds n_prev; out_capacity
+ * bounds the output (overflow sets FLASHLOOP_DEVERR_CAPACITY and truncates). */
+int flashloop_gate(const flashloop_params* p, const uint16_t* x_cur, const uint16_t* x_prev,
+                   const int32_t* prev_active, const int32_t* n_prev, int32_t prev_capacity,
+                   int32_t* active_out, int32_t* slot_out, int32_t* n_active_out, int32_t out_capacity,
+                   void* workspace, int32_t* err_word, void* stream);
+
+/* (a2) Gathered Q/K/V projection with RoPE [FlashLoop §4.3 (post-RoPE keys),
+ * App. E, App. G "fused projections"].  For a < *n_active, token t = active[a]:
+ * [q|k|v] = x[t] W_qkv^T (W_qkv = [W_q; W_k; W_v], [3d, d]), float32
+ * accumulation, RoPE at position t on q and k.  q is stored as bf16 at
+ * q_out[t] ([S, H, dh]); k and v as float32 at k_out[a], v_out[a]
+ * ([capacity, H, dh]).  active = NULL means the identity over S tokens. */
+int flashloop_qkv_gathered(const flashloop_params* p, const uint16_t* x, const int32_t* active,
+                           const int32_t* n_active, int32_t capacity, const uint16_t* w_qkv,
+                           const float* rope_cs, uint16_t* q_out, float* k_out, float* v_out,
+                           void* stream);
+
+/* (a3) Cross-loop KV residual quantisation [FlashLoop §3.3, §4.3, App. D.3].
+ * loop == 1: the INT8 base of k_new / v_new for every token (k_new[t]).
+ * loop >= 2: for a < *n_active, token t = active[a]: rho = x_new[a] - Xhat^(r-1)_t
+ * with Xhat^(r-1)_t = deq(base_t) + sum_{l=2}^{r-1} deq(res_l[slot_l[t]]) summed
+ * in float32 in that order; s = fp16_rn(max|rho| / qmax) per group of 32,
+ * code = clamp(rint(rho / s), -qmax, qmax) with IEEE float32 division
+ * (s == 0 gives code 0), qmax = 2^(bits_r - 1) - 1; stored at res_r[a]. */
+int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const float* k_new,
+                                const float* v_new, const int32_t* active, const int32_t* n_active,
+                                flashloop_state* st, void* stream);
+
+/* (a4) Column selection [FlashLoop §3.2, §4.2, App. D.2].  Per head h: the k
+ * candidates of largest float32 mass[h, j] (ties to the lower index, -0 == +0),
+ * written ascending to out[h*k ...].  candidates = NULL: all j in [0, S);
+ * otherwise candidates[h*n_cand ...] ascending.  n_cand <= 53248. */
+int flashloop_topk_columns(const flashloop_params* p, const float* mass, const int32_t* candidates,
+                           int32_t n_cand, int32_t k, int32_t* out, void* stream);
+
+/* (a5) Selected-column reconstruction [FlashLoop App. G: attention reads the
+ * packed anchor and residual streams, no full BF16 KV rebuild].  For loop
+ * r >= 2 and each head h, rebuilds Khat^(r-1)_j, Khat^(r)_j, Vhat^(r-1)_j and
+ * Vhat^(r)_j of the k selected columns j (cols of the latest selecting loop)
+ * from the base and residual streams (float32 sums in loop order, rounded to
+ * fp16) into state->workspace, where flashloop_sparse_attn_update reads them.
+ * loop == 1 rebuilds Khat^(1), Vhat^(1) of every token. */
+int flashloop_selcol_dequant(const flashloop_params* p, int32_t loop, flashloop_state* st,
+                             void* stream);
+
+/* (a6) Sparse attention update of loop r >= 2 [FlashLoop §3.2, §4.2,
+ * App. D.2, App. G].  For each head h, active row i (tokens of active[r-1])
+ * and selected column j <= i (cols of the latest selecting loop):
+ *   s_old = q_i^(r-1) . Khat_j^(r-1) / sqrt(dh),  s_new = q_i^(r) . Khat_j^(r) / sqrt(dh),
+ *   m' = max(m_i, max s_new), a = e^(m_i - m'),
+ *   Z' = a Z_i - sum e^(s_old - m') + sum e^(s_new - m'),
+ *   N' = a N_i - sum e^(s_old - m') Vhat_j^(r-1) + sum e^(s_new - m') Vhat_j^(r),
+ *   O_i = N' / Z' (bf16).
+ * Reads q slots sel(r-1), sel(r), the state slot sel(r-1) and the columns
+ * flashloop_selcol_dequant rebuilt (call it first, same loop); writes the
+ * state slot sel(r) and the rows of O.  With want_colmass != 0 also writes
+ * colmass[1][h, j] = sum_i e^(s_new - m') / Z' for the selected j.
+ * loop == 1 runs the dense loop-1 attention (every j <= i, no removal, the
+ * state starts empty) and always writes colmass[0]. */
+int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashloop_state* st,
+                                 int32_t want_colmass, void* stream);
+
+/* (a7) Gathered output projection: for a < *n_active, t = active[a]:
+ * y[t] = bf16(o[t] W_o^T) (float32 accumulation); other rows untouched. */
+int flashloop_out_proj(const flashloop_params* p, const uint16_t* o, const int32_t* active,
+                       const int32_t* n_active, int32_t capacity, const uint16_t* w_o, uint16_t* y,
+                       void* stream);
+
+/* One loop of the sublayer: a1..a7 at loop >= 2 (gate against x_prev), or the
+ * dense setup at loop == 1 (x_prev unused): every token active, INT8 base,
+ * dense causal attention on the reconstructed base, column mass, W_o.
+ * [FlashLoop §4, App. D]. */
+int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur,
+                        const uint16_t* x_prev, const uint16_t* w_qkv, const uint16_t* w_o,
+                        flashloop_state* st, void* stream);
+
+/* Host helper: the loop whose selection loop r uses (2 <= r): the latest
+ * loop l <= r with l == 2 or topk[l-1] < topk[l-2]. */
+int32_t flashloop_selection_loop(const flashloop_params* p, int32_t loop);
+
+/* Copy *err_word to the host (synchronising the stream) and map it to a
+ * status: FLASHLOOP_OK, or FLASHLOOP_ERR_DEVICE with the code in *code. */
+int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* stream);
+
+/* Static description of a status code. */
+const char* flashloop_status_string(int status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLASHLOOP_H */
