@@ -40,42 +40,102 @@ def run_gpu(cfg, W, X, stream=None):
 
 
 def check_selection(gpu_cols, orc_cols, mass):
-    """Equal sets, or different only between columns of (near-)equal mass."""
+    """Equal sets, or different only between columns of (near-)equal mass.
+    Returns the columns that are in one set only."""
     g, o = set(gpu_cols.tolist()), set(np.asarray(orc_cols).tolist())
     if g == o:
-        return 0
-    only_g, only_o = sorted(g - o), sorted(o - g)
+        return set()
+    only = (g - o) | (o - g)
     band = 1e-5 * float(np.max(mass))
     kth = min(mass[list(o)])
-    for j in only_g + only_o:
+    for j in only:
         assert abs(mass[j] - kth) <= band, (j, mass[j], kth)
-    return len(only_g)
+    return only
 
 
-def compare(cfg, orc, snaps, heads, check_y):
-    d, dh = cfg.d_model, cfg.head_dim
+def gpu_reconstruct(st, cfg, name, tokens, loop, slots):
+    """Khat/Vhat of the GPU cache (float64), rebuilt here from its bytes."""
+    base = st[f"{name}_base"].cpu().numpy()[tokens].astype(np.float64)
+    s = st[f"{name}_base_s"].cpu().numpy()[tokens].astype(np.float64)
+    acc = base * np.repeat(s, 32, axis=-1)
+    scale = np.repeat(s, 32, axis=-1)
+    for l in range(2, loop + 1):
+        sl = slots[l][tokens]
+        have = sl >= 0
+        if not have.any():
+            continue
+        c = O.unpack_codes(st[f"{name}_res{l}"].cpu().numpy()[sl[have]], cfg.bits[l - 1]).astype(np.float64)
+        sc = np.repeat(st[f"{name}_res{l}_s"].cpu().numpy()[sl[have]].astype(np.float64), 32, axis=-1)
+        acc[have] += c * sc
+        if l == loop:
+            scale[have] = sc
+    return acc, scale
+
+
+def check_caches(cfg, orc, st, heads):
+    """Both caches quantise (almost) the same keys and values: wherever they
+    differ the difference stays inside the two quantisers' rounding bounds.
+    Returns, per loop, the set of (held-head index, token) whose
+    reconstruction differs by more than float rounding."""
+    slots = {r: orc.Kc.slot[r] for r in range(2, cfg.n_loops + 1)}
+    hidx = np.array(heads)
+    flipped = {}
+    for r in range(1, cfg.n_loops + 1):
+        toks = orc.active[r]
+        flipped[r] = set()
+        for name, kv in (("k", orc.Kc), ("v", orc.Vc)):
+            g, sg = gpu_reconstruct(st, cfg, name, toks, r, slots)
+            g, sg = g[:, hidx], sg[:, hidx]
+            o = kv.reconstruct(toks, r).astype(np.float64)
+            so = np.repeat((kv.base[1] if r == 1 else kv.res[r][1]).astype(np.float64), 32, axis=-1)
+            diff = np.abs(g - o)
+            bound = (sg + so) / 2 * (1 + 1e-3) + 1e-4 * np.abs(o) + 1e-5
+            assert np.all(diff <= bound), (name, r, float((diff - bound).max()))
+            bad = np.argwhere(diff.max(axis=-1) > 1e-3 * np.maximum(np.abs(o).max(axis=-1), 1e-3))
+            flipped[r] |= {(int(a), int(toks[t])) for t, a in bad}
+        # a token's reconstruction persists into later loops while it is inactive
+        if r > 1:
+            flipped[r] |= flipped[r - 1]
+    return flipped
+
+
+def compare(cfg, orc, snaps, st, heads, check_y):
+    """Per loop: sets exact, selections exact up to near-ties, O (and Y)
+    within 1e-2 per row for at least 99.5% of the active rows and within
+    5e-2 for all, every row above 1e-2 explained by a quantiser rounding flip
+    or a near-tie selection in the columns it attends to."""
+    dh = cfg.head_dim
     cols = np.concatenate([np.arange(h * dh, (h + 1) * dh) for h in heads])
+    flipped = check_caches(cfg, orc, st, heads)
     worst = {}
+    sel_loop = {r: F.flashloop_selection_loop(F.Params.from_config(cfg), r) for r in range(2, cfg.n_loops + 1)}
     for r in range(1, cfg.n_loops + 1):
         s = snaps[r]
         act = orc.active[r]
         assert s["n"] == act.size
         assert np.array_equal(s["active"][: act.size], act)
+        swapped = {}
         if r >= 2:
             for a, h in enumerate(heads):
-                check_selection(s["cols"][h], orc.T[F.flashloop_selection_loop(F.Params.from_config(cfg), r)][a],
-                                orc.colmass[1][a])
-        og = bf16_rows(s["O"][act][:, cols])
-        oo = bf16_rows(orc.O_hist[r][act])
-        e = row_rel_l2(og, oo)
-        worst[f"O{r}"] = float(e.max())
-        assert e.max() < TOL, (r, e.max(), int(np.argmax(e)))
+                swapped[a] = check_selection(s["cols"][h], orc.T[sel_loop[r]][a], orc.colmass[1][a])
+        og = bf16_rows(s["O"][act][:, cols]).reshape(act.size, len(heads), dh)
+        oo = bf16_rows(orc.O_hist[r][act]).reshape(act.size, len(heads), dh)
+        e = row_rel_l2(og.reshape(act.size, -1), oo.reshape(act.size, -1))
+        worst[f"O{r}"] = (float(np.median(e)), float(e.max()))
+        assert e.max() < 5 * TOL, (r, e.max())
+        assert np.mean(e < TOL) >= 0.995, (r, np.mean(e < TOL))
+        for i in np.nonzero(e >= TOL)[0]:
+            tok = int(act[i])
+            a = int(np.argmax(np.linalg.norm(og[i] - oo[i], axis=-1)))
+            cause = (any(h2 == a and j <= tok for h2, j in flipped[r])
+                     or any(j <= tok for j in swapped.get(a, ())))
+            assert cause, (r, tok, float(e[i]))
         if check_y:
             yg = bf16_rows(s["Y"][act])
             yo = bf16_rows(orc.Y_hist[r][act])
             ey = row_rel_l2(yg, yo)
-            worst[f"Y{r}"] = float(ey.max())
-            assert ey.max() < TOL, (r, ey.max())
+            worst[f"Y{r}"] = (float(np.median(ey)), float(ey.max()))
+            assert ey.max() < 5 * TOL and np.mean(ey < TOL) >= 0.995, (r, ey.max())
     return worst
 
 
@@ -86,10 +146,10 @@ def test_loop_step_matches_oracle(name):
     X, _ = make_hidden_states(cfg)
     orc = O.OracleSequence(cfg, W, X).run()
     p, st, snaps = run_gpu(cfg, W, X)
-    worst = compare(cfg, orc, snaps, list(range(cfg.n_heads)), True)
+    worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True)
     print(name, worst)
-    # cache codes: identical except where rounding of the projection moved a
-    # value across a code boundary; reconstructions stay within the bound
+    # codes differ only where float rounding of the projection moved a value
+    # across a code boundary: rare, and one step for the base
     for name_, kv in (("k", orc.Kc), ("v", orc.Vc)):
         codes, s16 = kv.base
         got = st[f"{name_}_base"].cpu().numpy()
@@ -98,7 +158,7 @@ def test_loop_step_matches_oracle(name):
         for r in range(2, cfg.n_loops + 1):
             n = orc.active[r].size
             gc = O.unpack_codes(st[f"{name_}_res{r}"][:n].cpu().numpy(), cfg.bits[r - 1])
-            assert np.mean(gc != kv.res[r][0]) < 5e-3, (name_, r)
+            assert np.mean(gc != kv.res[r][0]) < 2e-3, (name_, r)
 
 
 @pytest.mark.parametrize("name,heads", [("depth_8k_r8", [0, 9]), ("prefill_32k", [5])])
@@ -108,7 +168,7 @@ def test_loop_step_matches_oracle_on_held_heads(name, heads):
     X, _ = make_hidden_states(cfg)
     orc = O.OracleSequence(cfg, W, X, heads=heads).run()
     p, st, snaps = run_gpu(cfg, W, X)
-    worst = compare(cfg, orc, snaps, heads, False)
+    worst = compare(cfg, orc, snaps, st, heads, False)
     print(name, worst)
     # Y at full size: every row of the final Y is its final O times W_o^T
     # (float64 check on a sample of rows)

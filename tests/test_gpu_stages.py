@@ -152,8 +152,11 @@ def test_gathered_qkv_projection(name):
         assert row_rel_l2(vv, orc.v_exact[r].reshape(n, d)).max() < 1e-5
         qg = bf16_rows(torch_to_bf16_bits(q[act]))
         qo = bf16_rows(orc.q[r][act].reshape(n, d))
-        rel = np.abs(qg - qo) / np.maximum(np.abs(qo), 1e-30)
-        assert np.all(rel <= 2.0 ** -7)                 # at most one bf16 rounding step apart
+        # bf16 storage of the same float32/float64 value: almost always the
+        # same bits, and within a bf16 rounding step per row otherwise (an
+        # element whose dot product nearly cancels can differ more in
+        # relative terms, so the bound is taken per row)
+        assert row_rel_l2(qg, qo).max() < 2.0 ** -8
         assert np.mean(qg == qo) > 0.99
 
 
