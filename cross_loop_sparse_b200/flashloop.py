@@ -82,6 +82,7 @@ _SIG = {
     "flashloop_cache_bytes": (c_size_t, [_P, _V]),
     "flashloop_rope_table": (_I, [_P, _I, _V, _V]),
     "flashloop_gate": (_I, [_P, _V, _V, _V, _V, _I, _V, _V, _V, _I, _V, _V, _V]),
+    "flashloop_gate_noalloc": (_I, [_P, _V, _V, _V, _V, _I, _V, _V, _V, _I, _V, _V]),
     "flashloop_qkv_gathered": (_I, [_P, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V]),
     "flashloop_kv_quant_residual": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
     "flashloop_topk_columns": (_I, [_P, _V, _V, _I, _I, _V, _V]),
@@ -161,6 +162,16 @@ def flashloop_gate(params, x_cur, x_prev, prev_active, n_prev, prev_capacity, ac
         ctypes.byref(params), _ptr(x_cur), _ptr(x_prev), _ptr(prev_active), _ptr(n_prev),
         prev_capacity, _ptr(active_out), _ptr(slot_out), _ptr(n_active_out), out_capacity,
         _ptr(workspace), _ptr(err_word), _stream(stream)))
+
+
+def flashloop_gate_noalloc(params, x_cur, x_prev, prev_active, n_prev, prev_capacity, active_out,
+                           slot_out, n_active_out, out_capacity, err_word, stream=None):
+    """flashloop_gate without a workspace: for callers that cannot allocate;
+    its scratch is a fixed device array inside the library (see the header)."""
+    return _check("flashloop_gate_noalloc", _lib.flashloop_gate_noalloc(
+        ctypes.byref(params), _ptr(x_cur), _ptr(x_prev), _ptr(prev_active), _ptr(n_prev),
+        prev_capacity, _ptr(active_out), _ptr(slot_out), _ptr(n_active_out), out_capacity,
+        _ptr(err_word), _stream(stream)))
 
 
 def flashloop_qkv_gathered(params, x, active, n_active, capacity, w_qkv, rope_cs, q_out, k_out,

@@ -138,6 +138,32 @@ int flashloop_gate(const flashloop_params* p, const uint16_t* x_cur, const uint1
                    int32_t* active_out, int32_t* slot_out, int32_t* n_active_out, int32_t out_capacity,
                    void* workspace, int32_t* err_word, void* stream);
 
+/* Variant of flashloop_gate for callers that cannot allocate device memory
+ * (the paper has no counterpart: this is an interface for deployment).  Such
+ * callers include a serving process that reserved all of HBM for its cache
+ * pools at start-up and runs with a frozen budget, a host framework that owns
+ * every device allocation, and latency-critical paths where cudaMalloc's
+ * implicit device synchronisation is not acceptable.  The result is the same
+ * as flashloop_gate's; there is no workspace argument.  Instead the
+ * scratch (one byte per candidate and a ticket) lives in a file-scope device
+ * array of the library: 64 KiB + 256 bytes that every GPU that loads the
+ * library holds until the process exits.
+ *  - Candidates (prev_capacity, or S when prev_active is NULL) above
+ *    FLASHLOOP_NOALLOC_MAX_CANDIDATES return FLASHLOOP_ERR_UNSUPPORTED.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) and caches it; make that first call before any
+ *    stream capture.
+ *  - Nothing is allocated or freed; each call zeroes the ticket with
+ *    cudaMemsetAsync on `stream`, then launches the gate kernel.
+ *  - Every call shares the one array, which keeps the previous call's
+ *    contents: calls that overlap on the GPU (other streams, other host
+ *    threads on the same device) race and must be serialised by the caller. */
+#define FLASHLOOP_NOALLOC_MAX_CANDIDATES 65536
+int flashloop_gate_noalloc(const flashloop_params* p, const uint16_t* x_cur, const uint16_t* x_prev,
+                           const int32_t* prev_active, const int32_t* n_prev, int32_t prev_capacity,
+                           int32_t* active_out, int32_t* slot_out, int32_t* n_active_out,
+                           int32_t out_capacity, int32_t* err_word, void* stream);
+
 /* (a2) Gathered Q/K/V projection with RoPE [FlashLoop §4.3 (post-RoPE keys),
  * App. E, App. G "fused projections"].  For a < *n_active, token t = active[a]:
  * [q|k|v] = x[t] W_qkv^T (W_qkv = [W_q; W_k; W_v], [3d, d]), float32
