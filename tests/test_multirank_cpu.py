@@ -1,0 +1,53 @@
+"""Host logic of the multi-GPU benchmark on CPU (gloo, world size 2): every
+rank owns a different seeded sequence and the timed region is reported as
+the maximum over ranks."""
+import os
+import socket
+
+import numpy as np
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _worker(rank, world, port, out):
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    from workload import CONFIGS, make_hidden_states
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        got = bench.max_over_ranks(1.5 + rank, "cpu")
+        X, planted = make_hidden_states(CONFIGS["tiny"], b=rank)
+        out[rank] = (got, int(X[0][:4, :4].astype(np.int64).sum()), planted[1][:8].tolist())
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_ranks_report_the_max_and_own_different_sequences():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as m:
+        out = m.dict()
+        mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True, start_method="spawn")
+        res = dict(out)
+    assert res[0][0] == res[1][0] == 2.5
+    assert res[0][1] != res[1][1] and res[0][2] != res[1][2]
+
+
+def test_single_process_max_is_identity():
+    import sys
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.max_over_ranks(3.25) == 3.25
