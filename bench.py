@@ -140,8 +140,6 @@ def run_cuda(args, cfg, rank, world, local_rank):
     p = F.Params.from_config(cfg)
     st = F.FlashLoopState(p, device=dev)
     S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
-    k_new = torch.empty((S, d), dtype=torch.float32, device=dev)
-    v_new = torch.empty_like(k_new)
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
     torch.cuda.synchronize()
 
@@ -157,10 +155,8 @@ def run_cuda(args, cfg, rank, world, local_rank):
             n_prev = None if r == 2 else st["n_active"][r - 2:]
             F.flashloop_gate(p, xs[r - 1], xs[r - 2], prev, n_prev, p.capacity[r - 2] if r > 2 else S,
                              act, st[f"slot{r}"], n_act, p.capacity[r - 1], st["workspace"], st["err"])
-            F.flashloop_qkv_gathered(p, xs[r - 1], act, n_act, p.capacity[r - 1], wqkv, st["rope_cs"],
-                                     st[f"q{st.q_slot(r)}"], k_new, v_new)
-            F.flashloop_kv_quant_residual(p, r, k_new, v_new, act, n_act, st)
-            n += 3
+            F.flashloop_qkv_quant(p, r, xs[r - 1], act, n_act, wqkv, st, st[f"q{st.q_slot(r)}"])
+            n += 2
             if F.flashloop_selection_loop(p, r) == r:
                 src = st["colmass0"] if r == 2 else st["colmass1"]
                 F.flashloop_topk_columns(p, src, None, 0, p.topk[r - 1], st[f"cols{r}"])

@@ -21,6 +21,8 @@ int launch_qkv_gemm(const flashloop_params*, const uint16_t*, const int32_t*, co
                     const uint16_t*, const float*, uint16_t*, float*, float*, int32_t*, cudaStream_t);
 int launch_out_gemm(const flashloop_params*, const uint16_t*, const int32_t*, const int32_t*, int,
                     const uint16_t*, uint16_t*, int32_t*, cudaStream_t);
+int launch_qkv_quant_gemm(const flashloop_params*, int, const uint16_t*, const int32_t*, const int32_t*, int,
+                          const uint16_t*, flashloop_state*, uint16_t*, cudaStream_t);
 }  // namespace fl
 
 #include "attn_args.cuh"
@@ -185,6 +187,28 @@ int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const f
   return launch_kv_quant(p, loop, k_new, v_new, active, n_active, st, as_stream(stream));
 }
 
+int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t* x, const int32_t* active,
+                        const int32_t* n_active, const uint16_t* w_qkv, flashloop_state* st,
+                        uint16_t* q_out, void* stream) {
+  int rc = check_common(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop < 1 || loop > p->n_loops || !x || !w_qkv || !st || !q_out || !st->rope_cs)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop >= 2) {
+    if (!active || !n_active) return FLASHLOOP_ERR_INVALID_ARG;
+    for (int l = 2; l <= loop; ++l) {
+      if (!st->k.res_codes[l - 1] || !st->k.res_scales[l - 1] || !st->v.res_codes[l - 1] ||
+          !st->v.res_scales[l - 1])
+        return FLASHLOOP_ERR_INVALID_ARG;
+      if (l < loop && !st->slot[l - 1]) return FLASHLOOP_ERR_INVALID_ARG;
+    }
+  }
+  return launch_qkv_quant_gemm(p, loop, x, loop == 1 ? nullptr : active, loop == 1 ? nullptr : n_active,
+                               capacity_of(p, loop), w_qkv, st, q_out, as_stream(stream));
+}
+
 int flashloop_topk_columns(const flashloop_params* p, const float* mass, const int32_t* candidates,
                            int32_t n_cand, int32_t k, int32_t* out, void* stream) {
   int rc = check_common(p);
@@ -311,16 +335,10 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   rc = check_state(p, st, loop);
   if (rc != FLASHLOOP_OK) return rc;
   cudaStream_t s = as_stream(stream);
-  const Workspace w = workspace_layout(p);
-  float* k_new = ws_ptr<float>(st->workspace, w.k_new);
-  float* v_new = ws_ptr<float>(st->workspace, w.v_new);
   const int cur = slot_of_loop(loop);
   const int cap = capacity_of(p, loop);
   if (loop == 1) {
-    rc = launch_qkv_gemm(p, x_cur, nullptr, nullptr, p->seq, w_qkv, st->rope_cs, st->q[0], k_new,
-                         v_new, st->err_word, s);
-    if (rc != FLASHLOOP_OK) return rc;
-    rc = launch_kv_quant(p, 1, k_new, v_new, nullptr, nullptr, st, s);
+    rc = launch_qkv_quant_gemm(p, 1, x_cur, nullptr, nullptr, p->seq, w_qkv, st, st->q[0], s);
     if (rc != FLASHLOOP_OK) return rc;
     rc = flashloop_selcol_dequant(p, 1, st, stream);
     if (rc != FLASHLOOP_OK) return rc;
@@ -335,10 +353,7 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   rc = launch_gate(p, x_cur, x_prev, prev_act, n_prev, capacity_of(p, loop - 1), act,
                    st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
   if (rc != FLASHLOOP_OK) return rc;
-  rc = launch_qkv_gemm(p, x_cur, act, n_act, cap, w_qkv, st->rope_cs, st->q[cur], k_new, v_new,
-                       st->err_word, s);
-  if (rc != FLASHLOOP_OK) return rc;
-  rc = launch_kv_quant(p, loop, k_new, v_new, act, n_act, st, s);
+  rc = launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, st->q[cur], s);
   if (rc != FLASHLOOP_OK) return rc;
   const int sel = flashloop_selection_loop(p, loop);
   if (sel == loop) {

@@ -85,6 +85,7 @@ _SIG = {
     "flashloop_gate_noalloc": (_I, [_P, _V, _V, _V, _V, _I, _V, _V, _V, _I, _V, _V]),
     "flashloop_qkv_gathered": (_I, [_P, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V]),
     "flashloop_kv_quant_residual": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
+    "flashloop_qkv_quant": (_I, [_P, _I, _V, _V, _V, _V, _S, _V, _V]),
     "flashloop_topk_columns": (_I, [_P, _V, _V, _I, _I, _V, _V]),
     "flashloop_selcol_dequant": (_I, [_P, _I, _S, _V]),
     "flashloop_sparse_attn_update": (_I, [_P, _I, _S, _I, _V]),
@@ -185,6 +186,12 @@ def flashloop_kv_quant_residual(params, loop, k_new, v_new, active, n_active, st
     return _check("flashloop_kv_quant_residual", _lib.flashloop_kv_quant_residual(
         ctypes.byref(params), loop, _ptr(k_new), _ptr(v_new), _ptr(active), _ptr(n_active),
         ctypes.byref(state.c), _stream(stream)))
+
+
+def flashloop_qkv_quant(params, loop, x, active, n_active, w_qkv, state, q_out, stream=None):
+    return _check("flashloop_qkv_quant", _lib.flashloop_qkv_quant(
+        ctypes.byref(params), loop, _ptr(x), _ptr(active), _ptr(n_active), _ptr(w_qkv),
+        ctypes.byref(state.c), _ptr(q_out), _stream(stream)))
 
 
 def flashloop_topk_columns(params, mass, candidates, n_cand, k, out, stream=None):

@@ -186,6 +186,17 @@ int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const f
                                 const float* v_new, const int32_t* active, const int32_t* n_active,
                                 flashloop_state* st, void* stream);
 
+/* (a2)+(a3) fused: the gathered projection of flashloop_qkv_gathered whose
+ * epilogue quantises k and v of loop `loop` straight into the state's
+ * streams (INT8 base at loop 1, the residual against Xhat^(loop-1) at loop
+ * >= 2, stored at the row's position in the active list), with the same
+ * arithmetic as flashloop_kv_quant_residual; q (RoPE'd, bf16) goes to
+ * q_out[t].  [FlashLoop §4.3, §4.4: KV update fused with quantisation.]
+ * loop == 1 projects every token (active ignored). */
+int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t* x, const int32_t* active,
+                        const int32_t* n_active, const uint16_t* w_qkv, flashloop_state* st,
+                        uint16_t* q_out, void* stream);
+
 /* (a4) Column selection [FlashLoop §3.2, §4.2, App. D.2].  Per head h: the k
  * candidates of largest float32 mass[h, j] (ties to the lower index, -0 == +0),
  * written ascending to out[h*k ...].  candidates = NULL: all j in [0, S);

@@ -220,3 +220,39 @@ def test_out_projection_staged(name):
     # rows outside the active set are untouched
     inactive = np.setdiff1d(np.arange(cfg.seq), act)
     assert torch.count_nonzero(y[inactive].float()).item() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
+def test_fused_projection_quantiser_matches_unfused(name):
+    """flashloop_qkv_quant (projection epilogue writes the codes) against
+    flashloop_qkv_gathered + flashloop_kv_quant_residual on the same device
+    inputs: identical q bits and identical cache bytes at every loop."""
+    cfg, W, X, planted, orc = oracle_run(name)
+    p, sa = new_state(cfg)
+    _, sb = new_state(cfg)
+    upload_sets(orc, sa, cfg.n_loops)
+    upload_sets(orc, sb, cfg.n_loops)
+    wqkv = bf16_to_torch(W["wqkv"])
+    d, S = cfg.d_model, cfg.seq
+    k = torch.zeros((S, d), dtype=torch.float32, device="cuda")
+    v = torch.zeros_like(k)
+    for r in range(1, cfg.n_loops + 1):
+        x = bf16_to_torch(X[r - 1])
+        qa = torch.zeros((S, d), dtype=torch.bfloat16, device="cuda")
+        qb = torch.zeros_like(qa)
+        if r == 1:
+            F.flashloop_qkv_gathered(p, x, None, None, S, wqkv, sa["rope_cs"], qa, k, v)
+            F.flashloop_kv_quant_residual(p, 1, k, v, None, None, sa)
+            F.flashloop_qkv_quant(p, 1, x, None, None, wqkv, sb, qb)
+        else:
+            act, n = sa[f"active{r}"], sa["n_active"][r - 1:]
+            F.flashloop_qkv_gathered(p, x, act, n, S, wqkv, sa["rope_cs"], qa, k, v)
+            F.flashloop_kv_quant_residual(p, r, k, v, act, n, sa)
+            F.flashloop_qkv_quant(p, r, x, sb[f"active{r}"], sb["n_active"][r - 1:], wqkv, sb, qb)
+        torch.cuda.synchronize()
+        assert torch.equal(qa.view(torch.int16), qb.view(torch.int16)), r
+        keys = ["k_base", "k_base_s", "v_base", "v_base_s"] if r == 1 else \
+            [f"k_res{r}", f"k_res{r}_s", f"v_res{r}", f"v_res{r}_s"]
+        for key in keys:
+            assert torch.equal(sa[key].view(torch.uint8), sb[key].view(torch.uint8)), (r, key)
+    assert sa.error_code() == 0 and sb.error_code() == 0
