@@ -13,7 +13,7 @@ int launch_gate(const flashloop_params*, const uint16_t*, const uint16_t*, const
                 const int32_t*, int, int32_t*, int32_t*, int32_t*, int, void*, int32_t*, cudaStream_t);
 int launch_kv_quant(const flashloop_params*, int, const float*, const float*, const int32_t*,
                     const int32_t*, flashloop_state*, cudaStream_t);
-int launch_selcol_dequant(const flashloop_params*, int, const int32_t*, int, flashloop_state*,
+int launch_selcol_dequant(const flashloop_params*, int, const int32_t*, int, int, flashloop_state*,
                           __half*, __half*, __half*, __half*, cudaStream_t);
 int launch_topk(const flashloop_params*, const float*, const int32_t*, int, int, int32_t*, int32_t*,
                 cudaStream_t);
@@ -28,7 +28,7 @@ int launch_qkv_quant_gemm(const flashloop_params*, int, const uint16_t*, const i
 #include "attn_args.cuh"
 
 namespace fl {
-int launch_attn_update(const flashloop_params*, const AttnArgs&, cudaStream_t);
+int launch_attn_tc(const flashloop_params*, const AttnArgs&, int, cudaStream_t);
 int launch_colmass(const flashloop_params*, const ColmassArgs&, cudaStream_t);
 
 // ---------------------------------------------------------------------------
@@ -240,9 +240,10 @@ static int check_state(const flashloop_params* p, const flashloop_state* st, int
   return FLASHLOOP_OK;
 }
 
-// Buffers of the rebuilt selected columns inside the workspace.
+// Buffers of the rebuilt selected columns inside the workspace: K as
+// [H, kcp, dh], V transposed as [H, dh, kcp] (kcp = kc rounded up to 8).
 struct ColBuffers {
-  int kc;
+  int kc, kcp;
   const int32_t* cols;
   __half *k_new, *v_new, *k_old, *v_old;
 };
@@ -253,9 +254,10 @@ static ColBuffers col_buffers(const flashloop_params* p, int loop, flashloop_sta
   const bool dense = loop == 1;
   const int sel = dense ? 1 : flashloop_selection_loop(p, loop);
   b.kc = dense ? p->seq : p->topk[sel - 1];
+  b.kcp = pad8(b.kc);
   b.cols = dense ? nullptr : st->cols[sel - 1];
   __half* base = ws_ptr<__half>(st->workspace, w.cols_kv);
-  const size_t one = (size_t)p->n_heads * b.kc * p->head_dim;
+  const size_t one = (size_t)p->n_heads * b.kcp * p->head_dim;
   b.k_new = base;
   b.v_new = base + one;
   b.k_old = dense ? nullptr : base + 2 * one;
@@ -271,7 +273,7 @@ int flashloop_selcol_dequant(const flashloop_params* p, int32_t loop, flashloop_
   rc = check_state(p, st, loop);
   if (rc != FLASHLOOP_OK) return rc;
   const ColBuffers b = col_buffers(p, loop, st);
-  return launch_selcol_dequant(p, loop, b.cols, b.kc, st, b.k_old, b.k_new, b.v_old, b.v_new,
+  return launch_selcol_dequant(p, loop, b.cols, b.kc, b.kcp, st, b.k_old, b.k_new, b.v_old, b.v_new,
                                as_stream(stream));
 }
 
@@ -299,11 +301,11 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
   a.o = st->O;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->head_dim);
   a.err = st->err_word;
-  rc = launch_attn_update(p, a, s);
+  rc = launch_attn_tc(p, a, b.kcp, s);
   if (rc != FLASHLOOP_OK) return rc;
   if (dense || want_colmass) {
     ColmassArgs c{};
-    c.S = p->seq; c.H = p->n_heads; c.kc = b.kc;
+    c.S = p->seq; c.H = p->n_heads; c.kc = b.kc; c.kcp = b.kcp;
     c.rows = a.rows; c.n_rows = a.n_rows; c.row_cap = a.row_cap; c.cols = b.cols;
     c.k_new = b.k_new; c.q = st->q[cur]; c.m = st->m[cur]; c.z = st->Z[cur];
     c.out = dense ? st->colmass[0] : st->colmass[1];

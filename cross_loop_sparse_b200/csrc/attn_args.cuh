@@ -30,12 +30,12 @@ struct AttnArgs {
 };
 
 struct ColmassArgs {
-  int S, H, kc;
+  int S, H, kc, kcp;          // kcp = row pitch of k_new
   const int32_t* rows;
   const int32_t* n_rows;
   int row_cap;
   const int32_t* cols;     // [H, kc] ascending (NULL: identity)
-  const __half* k_new;     // [H, kc, DH]
+  const __half* k_new;     // [H, kcp, DH]
   const uint16_t* q;       // bf16 [S, H*DH]
   const float* m;          // [H, S] final row max (natural units)
   const float* z;          // [H, S]

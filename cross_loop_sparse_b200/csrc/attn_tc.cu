@@ -1,0 +1,558 @@
+// (a6) Sparse attention update (and the dense loop-1 attention) on the
+// sm_100a tensor cores: tcgen05.mma with Q, P and the running numerator in
+// TMEM, K and V tiles streamed by TMA.
+//
+// [FlashLoop §3.2, §4.2, App. D.2]: for every active row i of loop r and
+// selected column j <= i, the loop r-1 contribution of (i, j) is removed from
+// the row's running state and the loop-r one added:
+//   S_old = Q^(r-1) Khat^(r-1)^T / sqrt(dh),  S_new = Q^(r) Khat^(r)^T / sqrt(dh)
+//   N' = a N + [e^(S_new - m') | -e^(S_old - m')] [Vhat^(r); Vhat^(r-1)]
+//   Z' = a Z + sum e^(S_new - m') - sum e^(S_old - m')
+// A block owns 128 active rows of one head at a time (persistent over
+// (head, row-tile) work items) and walks the head's ascending selected columns
+// in tiles of 64 up to its largest row token.
+//
+// TMEM (512 columns): Q_new | Q_old (fp16 pairs), N (f32, DH columns), two
+// score buffers {S_new 64 | S_old 64}; P = [e_new | -e_old] (fp16 pairs) is
+// written over the S_new half of its buffer and fed to the P.V MMA from TMEM.
+// Roles: warps 0-3 own one row each (TMEM lane) and do the masking,
+// exponentials, running max and sums, the Q / N set-up and the write-back;
+// warp 4 allocates TMEM and streams K (64 x DH) and V^T (DH x 64) tiles by TMA;
+// warp 5 issues S(t+1) while the rows process S(t), then P(t).V.
+// The running maximum is a per-row reference raised only when a tile's
+// maximum exceeds it by 8 (log2 units), which keeps every exponential
+// <= 2^8 and represents the same (m, N, Z) state (N and Z are defined up to
+// the common factor e^m).  All waits are bounded.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include "attn_args.cuh"
+#include "common.cuh"
+#include "tc_util.cuh"
+
+namespace fl {
+
+constexpr int kAtRows = 128, kAtCols = 64, kAtStages = 3, kAtThreads = 192;
+constexpr float kAtLog2e = 1.4426950408889634f;
+constexpr float kRescaleThreshold = 8.f;
+
+template <int DH>
+struct AtCfg {
+  static constexpr int kKBytes = kAtCols * DH * 2;  // K tile: 64 rows x DH (DH/64 swizzle chunks)
+  static constexpr int kVBytes = DH * kAtCols * 2;  // V^T tile: DH rows x 64
+  static constexpr int kStageBytes = 2 * kKBytes + 2 * kVBytes;
+  static constexpr int kSmem = 1024 + kAtStages * kStageBytes + 512;
+  static constexpr uint32_t kColQn = 0;
+  static constexpr uint32_t kColQo = DH / 2;
+  static constexpr uint32_t kColN = DH;
+  static constexpr uint32_t kColS = 2 * DH;  // buffer b: S_new at kColS + 128 b, S_old at +64
+  static constexpr uint32_t kIdescS = f16_idesc(128, kAtCols, 0);
+  static constexpr uint32_t kIdescPV = f16_idesc(128, DH, 0);
+};
+
+struct AtArgs {
+  int S, H, kc, dense;
+  const int32_t* rows;
+  const int32_t* n_rows;
+  int row_cap;
+  const int32_t* cols;   // [H, kc] ascending (NULL: identity)
+  const uint16_t* q_new; // bf16 [S, H*DH]
+  const uint16_t* q_old;
+  const float* m_in;
+  const float* z_in;
+  const float* n_in;
+  float* m_out;
+  float* z_out;
+  float* n_out;
+  uint16_t* o;
+  float scale_log2;
+  int32_t* err;
+};
+
+__device__ __forceinline__ int at_count_le(const int32_t* cols, int n, int tok) {
+  int lo = 0, hi = n;
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(cols + mid) <= tok) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+// Number of column tiles work item (h, rt) needs: columns up to its last row token.
+__device__ __forceinline__ int at_tiles(const AtArgs& g, int h, int rt, int n_rows) {
+  int last = min(n_rows, (rt + 1) * kAtRows) - 1;
+  int tok = g.rows ? __ldg(g.rows + last) : last;
+  if (tok < 0) return 0;
+  if (tok >= g.S) tok = g.S - 1;
+  const int nc = g.cols ? at_count_le(g.cols + (size_t)h * g.kc, g.kc, tok) : min(tok + 1, g.kc);
+  return (nc + kAtCols - 1) / kAtCols;
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kAtThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
+               const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_vo, AtArgs g) {
+  using C = AtCfg<DH>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAtStages * C::kStageBytes);
+  uint64_t* kv_full = bars;                    // [stages]
+  uint64_t* kv_empty = bars + kAtStages;       // [stages]
+  uint64_t* s_full = bars + 2 * kAtStages;     // [2]
+  uint64_t* p_full = s_full + 2;               // [2]
+  uint64_t* pv_done = p_full + 2;              // [2]
+  uint64_t* q_ready = pv_done + 2;             // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const bool has_old = !g.dense;
+  int n_rows = g.n_rows ? *g.n_rows : g.S;
+  if (n_rows > g.row_cap) n_rows = g.row_cap;
+  if (n_rows < 0) n_rows = 0;
+  const int row_tiles = (n_rows + kAtRows - 1) / kAtRows;
+  const int total = row_tiles * g.H;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAtStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 128);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(q_ready, 128);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------ TMA loads
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const uint32_t bytes = has_old ? C::kStageBytes : (C::kKBytes + C::kVBytes);
+      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
+        const int h = item / row_tiles, rt = item % row_tiles;
+        const int nt = at_tiles(g, h, rt, n_rows);
+        for (int t = 0; t < nt; ++t) {
+          if (!mbar_wait(&kv_empty[stage], phase ^ 1)) {
+            set_error(g.err, kDevErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          mbar_arrive_expect_tx(&kv_full[stage], bytes);
+#pragma unroll
+          for (int c = 0; c < DH / 64; ++c)
+            tma_load_3d(st + c * (kAtCols * 128), &tm_kn, c * 64, t * kAtCols, h, &kv_full[stage]);
+          tma_load_3d(st + 2 * C::kKBytes, &tm_vn, t * kAtCols, 0, h, &kv_full[stage]);
+          if (has_old) {
+#pragma unroll
+            for (int c = 0; c < DH / 64; ++c)
+              tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), &tm_ko, c * 64, t * kAtCols, h, &kv_full[stage]);
+            tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, &tm_vo, t * kAtCols, 0, h, &kv_full[stage]);
+          }
+          if (++stage == kAtStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t u = 0;        // global tile counter (S buffer = u & 1)
+      uint32_t item_no = 0;
+      bool ok = true;
+      for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x, ++item_no) {
+        const int h = item / row_tiles, rt = item % row_tiles;
+        const int nt = at_tiles(g, h, rt, n_rows);
+        if (!mbar_wait(q_ready, item_no & 1)) {
+          set_error(g.err, kDevErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        int prev_stage = -1;
+        for (int t = 0; t <= nt; ++t) {
+          if (t < nt) {
+            // S(t) into buffer u & 1
+            if (!mbar_wait(&kv_full[stage], phase)) {
+              set_error(g.err, kDevErrTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sb = tmem + C::kColS + (u & 1) * 128;
+            const uint32_t k_addr = smem_u32(smem + stage * C::kStageBytes);
+#pragma unroll
+            for (int ks = 0; ks < DH / 16; ++ks) {
+              const uint32_t kd = k_addr + (ks >> 2) * (kAtCols * 128) + (ks & 3) * 32;
+              umma_f16_ts(sb, tmem + C::kColQn + ks * 8, sw128_kmajor_desc(kd), C::kIdescS, ks > 0);
+              if (has_old)
+                umma_f16_ts(sb + 64, tmem + C::kColQo + ks * 8, sw128_kmajor_desc(kd + C::kKBytes), C::kIdescS,
+                            ks > 0);
+            }
+            umma_commit(&s_full[u & 1]);
+          }
+          if (t > 0) {
+            // P(t-1).V into N
+            const uint32_t up = u - 1;
+            if (!mbar_wait(&p_full[up & 1], (up >> 1) & 1)) {
+              set_error(g.err, kDevErrTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
+            const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKBytes);
+#pragma unroll
+            for (int ks = 0; ks < kAtCols / 16; ++ks)
+              umma_f16_ts(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
+            if (has_old) {
+#pragma unroll
+              for (int ks = 0; ks < kAtCols / 16; ++ks)
+                umma_f16_ts(tmem + C::kColN, pcol + 32 + ks * 8, sw128_kmajor_desc(v_addr + C::kVBytes + ks * 32),
+                            C::kIdescPV, 1u);
+            }
+            umma_commit(&kv_empty[prev_stage]);
+            umma_commit(&pv_done[up & 1]);
+          }
+          if (t < nt) {
+            prev_stage = stage;
+            if (++stage == kAtStages) {
+              stage = 0;
+              phase ^= 1;
+            }
+            ++u;
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ rows
+    const int row = warp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int HD = g.H * DH;
+    uint32_t u = 0;
+    uint32_t item_no = 0;
+    for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x, ++item_no) {
+      const int h = item / row_tiles, rt = item % row_tiles;
+      const int nt = at_tiles(g, h, rt, n_rows);
+      const int a = rt * kAtRows + row;
+      int tok = -1;
+      if (a < n_rows) {
+        tok = g.rows ? __ldg(g.rows + a) : a;
+        if (tok < 0 || tok >= g.S) {
+          set_error(g.err, FLASHLOOP_DEVERR_INDEX);
+          tok = -1;
+        }
+      }
+      // Q_new, Q_old (bf16 -> fp16 pairs) and N into TMEM; m, Z into registers.
+      {
+        uint32_t r[32];
+#pragma unroll
+        for (int which = 0; which < 2; ++which) {
+          const uint16_t* qsrc = which == 0 ? g.q_new : g.q_old;
+          const bool load = tok >= 0 && (which == 0 || has_old);
+#pragma unroll
+          for (int half = 0; half < DH / 64; ++half) {
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              uint4 w = make_uint4(0, 0, 0, 0);
+              if (load) w = *reinterpret_cast<const uint4*>(qsrc + (size_t)tok * HD + (size_t)h * DH + half * 64 + v * 8);
+              r[4 * v + 0] = bf16x2_to_half2_bits(w.x);
+              r[4 * v + 1] = bf16x2_to_half2_bits(w.y);
+              r[4 * v + 2] = bf16x2_to_half2_bits(w.z);
+              r[4 * v + 3] = bf16x2_to_half2_bits(w.w);
+            }
+            __syncwarp();
+            tmem_st32(tmem + lane_base + (which == 0 ? C::kColQn : C::kColQo) + half * 32, r);
+          }
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+#pragma unroll
+          for (int v = 0; v < 8; ++v) {
+            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (!g.dense && tok >= 0)
+              w = *reinterpret_cast<const float4*>(g.n_in + ((size_t)h * g.S + tok) * DH + c0 + 4 * v);
+            r[4 * v + 0] = __float_as_uint(w.x);
+            r[4 * v + 1] = __float_as_uint(w.y);
+            r[4 * v + 2] = __float_as_uint(w.z);
+            r[4 * v + 3] = __float_as_uint(w.w);
+          }
+          __syncwarp();
+          tmem_st32(tmem + lane_base + C::kColN + c0, r);
+        }
+        tmem_wait_st();
+      }
+      float m_ref = -INFINITY, z = 0.f;
+      if (!g.dense && tok >= 0) {
+        m_ref = g.m_in[(size_t)h * g.S + tok] * kAtLog2e;
+        z = g.z_in[(size_t)h * g.S + tok];
+      }
+      tc_fence_before();
+      mbar_arrive(q_ready);
+
+      const int32_t* hcols = g.cols ? g.cols + (size_t)h * g.kc : nullptr;
+      // smallest row token of this warp: tiles at or below it need no causal mask
+      int wmin = tok < 0 ? 0x7fffffff : tok;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) wmin = min(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+      bool failed = false;
+      for (int t = 0; t < nt; ++t, ++u) {
+        const uint32_t b = u & 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (u >> 1) & 1))) {
+          set_error(g.err, kDevErrTimeout);
+          *abort_flag = 1;
+          failed = true;
+          break;
+        }
+        tc_fence_after();
+        uint32_t rn[2][32], ro[2][32];
+        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
+        __syncwarp();
+        tmem_ld32(sbase, rn[0]);
+        tmem_ld32(sbase + 32, rn[1]);
+        if (has_old) {
+          tmem_ld32(sbase + 64, ro[0]);
+          tmem_ld32(sbase + 96, ro[1]);
+        }
+        tmem_wait_ld();
+        // column tokens of this tile
+        const int c0 = t * kAtCols;
+        const int last_c = min(c0 + kAtCols, g.kc) - 1;
+        const int last_tok = hcols ? __ldg(hcols + last_c) : last_c;
+        const bool need_mask = (c0 + kAtCols > g.kc) || (last_tok > wmin);
+        // scores in the log2 domain, masked columns -> -inf (kept as float bits in place)
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          float vn = __uint_as_float(rn[e >> 5][e & 31]) * g.scale_log2;
+          float vo = has_old ? __uint_as_float(ro[e >> 5][e & 31]) * g.scale_log2 : -INFINITY;
+          if (need_mask || tok < 0) {
+            const int cj = c0 + e;
+            const int ct = cj < g.kc ? (hcols ? __ldg(hcols + cj) : cj) : 0x7fffffff;
+            if (tok < 0 || ct > tok) {
+              vn = -INFINITY;
+              vo = -INFINITY;
+            }
+          }
+          rn[e >> 5][e & 31] = __float_as_uint(vn);
+          ro[e >> 5][e & 31] = __float_as_uint(vo);
+        }
+        float mx = -INFINITY;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(rn[e >> 5][e & 31]));
+        const bool need = mx > m_ref + kRescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          // raise the reference of this warp's rows: N and Z scale by 2^(m_ref - mx)
+          const float new_ref = need ? mx : m_ref;
+          const float f = need ? ex2(m_ref - new_ref) : 1.f;
+          if (t > 0) {
+            const uint32_t up = u - 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[up & 1], (up >> 1) & 1))) {
+              set_error(g.err, kDevErrTimeout);
+              *abort_flag = 1;
+              failed = true;
+              break;
+            }
+            tc_fence_after();
+          }
+          uint32_t r[32];
+#pragma unroll
+          for (int cc = 0; cc < DH; cc += 32) {
+            __syncwarp();
+            tmem_ld32(tmem + lane_base + C::kColN + cc, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+            __syncwarp();
+            tmem_st32(tmem + lane_base + C::kColN + cc, r);
+          }
+          tmem_wait_st();
+          z *= f;
+          m_ref = new_ref;
+        }
+        uint32_t pk[32];
+        float zs = 0.f;
+#pragma unroll
+        for (int e2 = 0; e2 < 32; ++e2) {
+          const float x0 = __uint_as_float(rn[(2 * e2) >> 5][(2 * e2) & 31]);
+          const float x1 = __uint_as_float(rn[(2 * e2 + 1) >> 5][(2 * e2 + 1) & 31]);
+          const float p0 = x0 == -INFINITY ? 0.f : ex2(x0 - m_ref);
+          const float p1 = x1 == -INFINITY ? 0.f : ex2(x1 - m_ref);
+          zs += p0 + p1;
+          pk[e2] = pack_half2(p0, p1);
+        }
+        __syncwarp();
+        tmem_st32(sbase, pk);
+        if (has_old) {
+#pragma unroll
+          for (int e2 = 0; e2 < 32; ++e2) {
+            const float x0 = __uint_as_float(ro[(2 * e2) >> 5][(2 * e2) & 31]);
+            const float x1 = __uint_as_float(ro[(2 * e2 + 1) >> 5][(2 * e2 + 1) & 31]);
+            const float p0 = x0 == -INFINITY ? 0.f : ex2(x0 - m_ref);
+            const float p1 = x1 == -INFINITY ? 0.f : ex2(x1 - m_ref);
+            zs -= p0 + p1;
+            pk[e2] = pack_half2(-p0, -p1);
+          }
+          __syncwarp();
+          tmem_st32(sbase + 32, pk);
+        }
+        z += zs;
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
+      }
+      if (failed) break;
+      // write back: wait for the last P.V of this item
+      if (nt > 0) {
+        const uint32_t up = u - 1;
+        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[up & 1], (up >> 1) & 1))) {
+          set_error(g.err, kDevErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+      }
+      const float inv = 1.f / z;
+#pragma unroll
+      for (int cc = 0; cc < DH; cc += 32) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + C::kColN + cc, r);
+        tmem_wait_ld();
+        if (tok >= 0) {
+          float4* nd = reinterpret_cast<float4*>(g.n_out + ((size_t)h * g.S + tok) * DH + cc);
+#pragma unroll
+          for (int v = 0; v < 8; ++v)
+            nd[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          uint4* od = reinterpret_cast<uint4*>(g.o + (size_t)tok * HD + (size_t)h * DH + cc);
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint32_t w[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int e = 8 * v + 2 * q;
+              w[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(r[e]) * inv) |
+                     ((uint32_t)float_to_bf16_bits(__uint_as_float(r[e + 1]) * inv) << 16);
+            }
+            od[v] = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        }
+      }
+      if (tok >= 0) {
+        g.m_out[(size_t)h * g.S + tok] = m_ref / kAtLog2e;
+        g.z_out[(size_t)h * g.S + tok] = z;
+      }
+      tc_fence_before();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 at_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 3-D fp16 tensor map: dims (innermost first) d0 x d1 x d2, row pitch p1 and
+// plane pitch p2 in elements, box b0 x b1 x 1, 128-byte swizzle.  Coordinates
+// past d1 read as zero.
+static int make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                            uint64_t p1, uint64_t p2, uint32_t b0, uint32_t b1) {
+  auto fn = at_encode_fn();
+  if (fn == nullptr) return FLASHLOOP_ERR_CUDA;
+  if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (p1 * 2) % 16 != 0 || (p2 * 2) % 16 != 0)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {p1 * 2, p2 * 2};
+  cuuint32_t box[3] = {b0, b1, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FLASHLOOP_OK : FLASHLOOP_ERR_CUDA;
+}
+
+static int at_sm_count() {
+  static int cached[128];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+// K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.
+int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
+  const int dh = p->head_dim, H = p->n_heads;
+  CUtensorMap tkn, tko, tvn, tvo;
+  int rc = make_tmap_f16_3d(&tkn, a.k_new, dh, a.kc, H, dh, (uint64_t)kcp * dh, 64, kAtCols);
+  if (rc == FLASHLOOP_OK) rc = make_tmap_f16_3d(&tvn, a.v_new, a.kc, dh, H, kcp, (uint64_t)kcp * dh, kAtCols, dh);
+  if (rc == FLASHLOOP_OK && !a.dense) {
+    rc = make_tmap_f16_3d(&tko, a.k_old, dh, a.kc, H, dh, (uint64_t)kcp * dh, 64, kAtCols);
+    if (rc == FLASHLOOP_OK) rc = make_tmap_f16_3d(&tvo, a.v_old, a.kc, dh, H, kcp, (uint64_t)kcp * dh, kAtCols, dh);
+  } else {
+    tko = tkn;
+    tvo = tvn;
+  }
+  if (rc != FLASHLOOP_OK) return rc;
+  AtArgs g{};
+  g.S = a.S; g.H = a.H; g.kc = a.kc; g.dense = a.dense; g.rows = a.rows; g.n_rows = a.n_rows;
+  g.row_cap = a.row_cap; g.cols = a.cols; g.q_new = a.q_new; g.q_old = a.q_old; g.m_in = a.m_in;
+  g.z_in = a.z_in; g.n_in = a.n_in; g.m_out = a.m_out; g.z_out = a.z_out; g.n_out = a.n_out; g.o = a.o;
+  g.scale_log2 = a.scale_log2; g.err = a.err;
+  const int max_items = ((a.row_cap + kAtRows - 1) / kAtRows) * H;
+  int grid = at_sm_count();
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  if (dh == 128) {
+    FL_TRY(cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtCfg<128>::kSmem));
+    attn_tc_kernel<128><<<grid, kAtThreads, AtCfg<128>::kSmem, stream>>>(tkn, tko, tvn, tvo, g);
+  } else {
+    FL_TRY(cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtCfg<64>::kSmem));
+    attn_tc_kernel<64><<<grid, kAtThreads, AtCfg<64>::kSmem, stream>>>(tkn, tko, tvn, tvo, g);
+  }
+  return launch_status();
+}
+
+}  // namespace fl

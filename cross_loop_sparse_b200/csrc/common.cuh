@@ -62,6 +62,7 @@ struct Workspace {
 };
 
 inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+inline int pad8(int x) { return (x + 7) & ~7; }
 
 inline int max_topk(const flashloop_params* p) {
   int k = 0;
@@ -77,8 +78,8 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   w.flags = off; off = align256(off + S);
   w.k_new = off; off = align256(off + S * H * dh * sizeof(float));
   w.v_new = off; off = align256(off + S * H * dh * sizeof(float));
-  size_t sel = 4 * H * (size_t)max_topk(p) * dh;
-  size_t dense = 2 * H * S * dh;
+  size_t sel = 4 * H * (size_t)pad8(max_topk(p)) * dh;
+  size_t dense = 2 * H * (size_t)pad8(p->seq) * dh;
   w.cols_kv = off; off = align256(off + (sel > dense ? sel : dense) * sizeof(__half));
   w.total = off;
   return w;

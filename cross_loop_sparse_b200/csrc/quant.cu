@@ -176,71 +176,99 @@ int launch_kv_quant(const flashloop_params* p, int loop, const float* k_new, con
 }
 
 // (a5) Rebuild Khat^(r-1), Khat^(r), Vhat^(r-1), Vhat^(r) of the selected
-// columns as fp16 [H, kc, dh] (loop 1 / dense: Khat^(1), Vhat^(1) of every
-// token).  [FlashLoop App. G]: only the selected columns are rebuilt, never
-// the full cache.
+// columns (loop 1 / dense: Khat^(1), Vhat^(1) of every token) as fp16:
+// K as [H, kcp, dh] rows, V transposed as [H, dh, kcp] so that both feed the
+// attention MMAs as K-major tiles.  [FlashLoop App. G]: only the selected
+// columns are rebuilt, never the full cache.  One block = 64 columns of one
+// head; V rows are staged in shared memory and written transposed.
 template <int DH>
 __global__ void __launch_bounds__(kQuantThreads)
-selcol_dequant_kernel(const int32_t* __restrict__ cols, int kc, int S, int H, int loop,
+selcol_dequant_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, int H, int loop,
                       KVStreams Ks, KVStreams Vs, LoopTables lt, __half* k_old, __half* k_new,
-                      __half* v_old, __half* v_new, int32_t* err) {
+                      __half* vt_old, __half* vt_new, int32_t* err) {
   constexpr int E = DH / 32;
-  const int lane = threadIdx.x & 31;
-  const long long total = (long long)kc * H * 2;
-  const long long warps = (long long)gridDim.x * (blockDim.x >> 5);
-  for (long long w = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < total;
-       w += warps) {
-    const int which = static_cast<int>(w & 1);
-    const int c = static_cast<int>((w >> 1) % kc);
-    const int h = static_cast<int>((w >> 1) / kc);
-    const int j = cols ? cols[(size_t)h * kc + c] : c;
-    if (j < 0 || j >= S) {
-      if (lane == 0) set_error(err, FLASHLOOP_DEVERR_INDEX);
-      continue;
-    }
-    const KVStreams& kv = which == 0 ? Ks : Vs;
-    float acc[E];
-    reconstruct_lane<E, DH>(kv, lt, j, h, H, loop > 1 ? loop - 1 : 1, lane, acc);
-    const size_t off = ((size_t)h * kc + c) * DH + lane * E;
-    if (loop > 1) {
-      __half* dst_old = (which == 0 ? k_old : v_old) + off;
-#pragma unroll
-      for (int e = 0; e < E; ++e) dst_old[e] = __float2half_rn(acc[e]);
-      const int sl = lt.slot[loop - 1][j];
-      if (sl >= 0) {
-        const int b = lt.bits[loop - 1];
-        const int g = (lane * E) / FLASHLOOP_GROUP;
-        const uint8_t* row = kv.res_codes[loop - 1] + ((size_t)sl * H + h) * (DH * b / 8);
-        const float s =
-            half_bits_to_float(kv.res_scales[loop - 1][((size_t)sl * H + h) * (DH / 32) + g]);
-        int cc[E];
-        unpack_codes<E>(row, lane * E, b, cc);
-#pragma unroll
-        for (int e = 0; e < E; ++e) acc[e] = acc[e] + static_cast<float>(cc[e]) * s;
+  __shared__ __align__(16) __half sv[2][64][DH + 8];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int h = blockIdx.y, j0 = blockIdx.x * 64;
+  const bool has_old = loop > 1;
+  for (int c = warp; c < 64; c += kQuantThreads / 32) {
+    const int col = j0 + c;
+    int j = -1;
+    if (col < kc) {
+      j = cols ? cols[(size_t)h * kc + col] : col;
+      if (j < 0 || j >= S) {
+        if (lane == 0) set_error(err, FLASHLOOP_DEVERR_INDEX);
+        j = -1;
       }
     }
-    __half* dst = (which == 0 ? k_new : v_new) + off;
+    for (int which = 0; which < 2; ++which) {
+      const KVStreams& kv = which == 0 ? Ks : Vs;
+      float acc[E], oldv[E];
+      if (j >= 0) {
+        reconstruct_lane<E, DH>(kv, lt, j, h, H, has_old ? loop - 1 : 1, lane, acc);
 #pragma unroll
-    for (int e = 0; e < E; ++e) dst[e] = __float2half_rn(acc[e]);
+        for (int e = 0; e < E; ++e) oldv[e] = acc[e];
+        if (has_old) {
+          const int sl = lt.slot[loop - 1][j];
+          if (sl >= 0) {
+            const int b = lt.bits[loop - 1];
+            const int g = (lane * E) / FLASHLOOP_GROUP;
+            const uint8_t* row = kv.res_codes[loop - 1] + ((size_t)sl * H + h) * (DH * b / 8);
+            const float sc = half_bits_to_float(kv.res_scales[loop - 1][((size_t)sl * H + h) * (DH / 32) + g]);
+            int cc[E];
+            unpack_codes<E>(row, lane * E, b, cc);
+#pragma unroll
+            for (int e = 0; e < E; ++e) acc[e] = acc[e] + static_cast<float>(cc[e]) * sc;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) acc[e] = oldv[e] = 0.f;
+      }
+      if (which == 0) {
+        if (col < kcp) {
+          const size_t off = ((size_t)h * kcp + col) * DH + lane * E;
+#pragma unroll
+          for (int e = 0; e < E; ++e) k_new[off + e] = __float2half_rn(acc[e]);
+          if (has_old) {
+#pragma unroll
+            for (int e = 0; e < E; ++e) k_old[off + e] = __float2half_rn(oldv[e]);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          sv[1][c][lane * E + e] = __float2half_rn(acc[e]);
+          sv[0][c][lane * E + e] = __float2half_rn(oldv[e]);
+        }
+      }
+    }
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < 2 * DH * 32; idx += kQuantThreads) {
+    const int which = idx / (DH * 32);
+    if (which == 0 && !has_old) continue;
+    const int rem = idx % (DH * 32);
+    const int d = rem / 32, jp = (rem % 32) * 2;
+    if (j0 + jp >= kcp) continue;
+    __half* dst = (which == 0 ? vt_old : vt_new) + ((size_t)h * DH + d) * kcp + j0 + jp;
+    *reinterpret_cast<__half2*>(dst) = __halves2half2(sv[which][jp][d], sv[which][jp + 1][d]);
   }
 }
 
-int launch_selcol_dequant(const flashloop_params* p, int loop, const int32_t* cols, int kc,
-                          flashloop_state* st, __half* k_old, __half* k_new, __half* v_old,
-                          __half* v_new, cudaStream_t stream) {
+int launch_selcol_dequant(const flashloop_params* p, int loop, const int32_t* cols, int kc, int kcp,
+                          flashloop_state* st, __half* k_old, __half* k_new, __half* vt_old,
+                          __half* vt_new, cudaStream_t stream) {
   const int H = p->n_heads;
-  const long long items = (long long)kc * H * 2;
-  long long grid = (items + (kQuantThreads / 32) - 1) / (kQuantThreads / 32);
-  if (grid > 148 * 16) grid = 148 * 16;
-  if (grid < 1) grid = 1;
+  dim3 grid((kcp + 63) / 64, H);
   const KVStreams Ks = kv_streams(st->k), Vs = kv_streams(st->v);
   const LoopTables lt = loop_tables(p, st);
   if (p->head_dim == 128) {
-    selcol_dequant_kernel<128><<<(int)grid, kQuantThreads, 0, stream>>>(
-        cols, kc, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, v_old, v_new, st->err_word);
+    selcol_dequant_kernel<128><<<grid, kQuantThreads, 0, stream>>>(
+        cols, kc, kcp, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
   } else {
-    selcol_dequant_kernel<64><<<(int)grid, kQuantThreads, 0, stream>>>(
-        cols, kc, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, v_old, v_new, st->err_word);
+    selcol_dequant_kernel<64><<<grid, kQuantThreads, 0, stream>>>(
+        cols, kc, kcp, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
   }
   return launch_status();
 }
