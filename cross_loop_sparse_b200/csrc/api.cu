@@ -309,7 +309,8 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
     c.rows = a.rows; c.n_rows = a.n_rows; c.row_cap = a.row_cap; c.cols = b.cols;
     c.k_new = b.k_new; c.q = st->q[cur]; c.m = st->m[cur]; c.z = st->Z[cur];
     c.out = dense ? st->colmass[0] : st->colmass[1];
-    c.scale_log2 = a.scale_log2; c.err = st->err_word;
+    c.scale_log2 = 1.0f;  // the rebuilt keys already carry log2(e)/sqrt(dh)
+    c.err = st->err_word;
     rc = launch_colmass(p, c, s);
   }
   return rc;

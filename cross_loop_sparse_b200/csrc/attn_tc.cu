@@ -33,7 +33,8 @@
 
 namespace fl {
 
-constexpr int kAtRows = 128, kAtCols = 64, kAtStages = 3, kAtThreads = 192;
+constexpr int kAtRows = 128, kAtCols = 64, kAtStages = 3, kAtThreads = 320;
+constexpr int kAtRowThreads = 256;  // warps 0-7: two threads per row, one per half of a tile
 constexpr float kAtLog2e = 1.4426950408889634f;
 constexpr float kRescaleThreshold = 8.f;
 
@@ -42,7 +43,7 @@ struct AtCfg {
   static constexpr int kKBytes = kAtCols * DH * 2;  // K tile: 64 rows x DH (DH/64 swizzle chunks)
   static constexpr int kVBytes = DH * kAtCols * 2;  // V^T tile: DH rows x 64
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kVBytes;
-  static constexpr int kSmem = 1024 + kAtStages * kStageBytes + 512;
+  static constexpr int kSmem = 1024 + kAtStages * kStageBytes + 512 + 6 * 128 * 4;
   static constexpr uint32_t kColQn = 0;
   static constexpr uint32_t kColQo = DH / 2;
   static constexpr uint32_t kColN = DH;
@@ -122,14 +123,14 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], 128);
+      mbar_init(&p_full[b], kAtRowThreads);
       mbar_init(&pv_done[b], 1);
     }
-    mbar_init(q_ready, 128);
+    mbar_init(q_ready, kAtRowThreads);
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 8) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -138,16 +139,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA loads
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
       const uint32_t bytes = has_old ? C::kStageBytes : (C::kKBytes + C::kVBytes);
+      int issued[kAtStages];
+      for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
       for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
         const int h = item / row_tiles, rt = item % row_tiles;
         const int nt = at_tiles(g, h, rt, n_rows);
-        for (int t = 0; t < nt; ++t) {
+        for (int t = 0; t < nt && !*abort_flag; ++t) {
           if (!mbar_wait(&kv_empty[stage], phase ^ 1)) {
             set_error(g.err, kDevErrTimeout);
             *abort_flag = 1;
@@ -165,14 +168,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
               tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), &tm_ko, c * 64, t * kAtCols, h, &kv_full[stage]);
             tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, &tm_vo, t * kAtCols, 0, h, &kv_full[stage]);
           }
+          issued[stage] = phase;
           if (++stage == kAtStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      // never leave with a copy in flight: wait (bounded) for the last load of every stage
+      for (int s2 = 0; s2 < kAtStages; ++s2)
+        if (issued[s2] >= 0) (void)mbar_wait(&kv_full[s2], (uint32_t)issued[s2]);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       int stage = 0;
@@ -249,12 +256,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
     }
   } else {
     // ------------------------------------------------------------ rows
-    const int row = warp * 32 + lane;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // Two threads per row: half 0 takes columns [0, 32) of each tile (and
+    // Q_new / the first half of N), half 1 columns [32, 64) (and Q_old / the
+    // second half of N).  The two warps of a row pair exchange tile maxima and
+    // sums through shared memory at a named barrier.  A named barrier cannot
+    // time out, so both warps always execute the same barrier sequence: after
+    // a failed wait (or an abort raised elsewhere) a warp turns "dead" - it
+    // skips waits, tensor-memory work and writes but keeps the control flow.
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int pair_bar = 1 + quarter;
+    float* xchg = reinterpret_cast<float*>(tmem_slot + 4);  // [2 parities][2 halves][128] maxima, then [2][128] sums
     const int HD = g.H * DH;
+    constexpr int kHalfCols = DH / 2;
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity) {
+      if (!dead && __any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+      if (dead) return;
+      if (!__all_sync(0xffffffffu, mbar_wait(bar, parity))) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        dead = true;
+        return;
+      }
+      tc_fence_after();
+    };
     uint32_t u = 0;
-    uint32_t item_no = 0;
-    for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x, ++item_no) {
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
       const int h = item / row_tiles, rt = item % row_tiles;
       const int nt = at_tiles(g, h, rt, n_rows);
       const int a = rt * kAtRows + row;
@@ -262,106 +291,111 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       if (a < n_rows) {
         tok = g.rows ? __ldg(g.rows + a) : a;
         if (tok < 0 || tok >= g.S) {
-          set_error(g.err, FLASHLOOP_DEVERR_INDEX);
+          if (half == 0) set_error(g.err, FLASHLOOP_DEVERR_INDEX);
           tok = -1;
         }
       }
-      // Q_new, Q_old (bf16 -> fp16 pairs) and N into TMEM; m, Z into registers.
-      {
-        uint32_t r[32];
-#pragma unroll
-        for (int which = 0; which < 2; ++which) {
-          const uint16_t* qsrc = which == 0 ? g.q_new : g.q_old;
-          const bool load = tok >= 0 && (which == 0 || has_old);
-#pragma unroll
-          for (int half = 0; half < DH / 64; ++half) {
-#pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint4 w = make_uint4(0, 0, 0, 0);
-              if (load) w = *reinterpret_cast<const uint4*>(qsrc + (size_t)tok * HD + (size_t)h * DH + half * 64 + v * 8);
-              r[4 * v + 0] = bf16x2_to_half2_bits(w.x);
-              r[4 * v + 1] = bf16x2_to_half2_bits(w.y);
-              r[4 * v + 2] = bf16x2_to_half2_bits(w.z);
-              r[4 * v + 3] = bf16x2_to_half2_bits(w.w);
-            }
-            __syncwarp();
-            tmem_st32(tmem + lane_base + (which == 0 ? C::kColQn : C::kColQo) + half * 32, r);
-          }
-        }
-#pragma unroll
+      // Q (fp16 pairs, exact from bf16) and this half of N into TMEM.  The
+      // rebuilt keys carry the factor log2(e)/sqrt(dh), so S is in log2 units.
+      if (!dead) {
+        const uint16_t* qsrc = half == 0 ? g.q_new : g.q_old;
+        const bool load_q = tok >= 0 && (half == 0 || has_old);
+        const uint32_t qcol = half == 0 ? C::kColQn : C::kColQo;
+#pragma unroll 1
         for (int c0 = 0; c0 < DH; c0 += 32) {
+          uint32_t r[16];
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
+          for (int v = 0; v < 4; ++v) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (load_q) w = *reinterpret_cast<const uint4*>(qsrc + (size_t)tok * HD + (size_t)h * DH + c0 + v * 8);
+            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+            for (int q = 0; q < 4; ++q) r[4 * v + q] = bf16x2_to_half2_bits(ws[q]);
+          }
+          __syncwarp();
+          tmem_st16(tmem + lane_base + qcol + c0 / 2, r);
+        }
+#pragma unroll 1
+        for (int c0 = 0; c0 < kHalfCols; c0 += 16) {
+          uint32_t r[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
             float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
             if (!g.dense && tok >= 0)
-              w = *reinterpret_cast<const float4*>(g.n_in + ((size_t)h * g.S + tok) * DH + c0 + 4 * v);
+              w = *reinterpret_cast<const float4*>(g.n_in + ((size_t)h * g.S + tok) * DH + half * kHalfCols + c0 + 4 * v);
             r[4 * v + 0] = __float_as_uint(w.x);
             r[4 * v + 1] = __float_as_uint(w.y);
             r[4 * v + 2] = __float_as_uint(w.z);
             r[4 * v + 3] = __float_as_uint(w.w);
           }
           __syncwarp();
-          tmem_st32(tmem + lane_base + C::kColN + c0, r);
+          tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + c0, r);
         }
         tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_ready);
       }
-      float m_ref = -INFINITY, z = 0.f;
-      if (!g.dense && tok >= 0) {
-        m_ref = g.m_in[(size_t)h * g.S + tok] * kAtLog2e;
-        z = g.z_in[(size_t)h * g.S + tok];
+      float m_ref = 0.f, z = 0.f;
+      if (tok >= 0) {
+        m_ref = g.dense ? -INFINITY : g.m_in[(size_t)h * g.S + tok] * kAtLog2e;
+        if (!g.dense && half == 0) z = g.z_in[(size_t)h * g.S + tok];
       }
-      tc_fence_before();
-      mbar_arrive(q_ready);
 
       const int32_t* hcols = g.cols ? g.cols + (size_t)h * g.kc : nullptr;
-      // smallest row token of this warp: tiles at or below it need no causal mask
       int wmin = tok < 0 ? 0x7fffffff : tok;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) wmin = min(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
-      bool failed = false;
       for (int t = 0; t < nt; ++t, ++u) {
         const uint32_t b = u & 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&s_full[b], (u >> 1) & 1))) {
-          set_error(g.err, kDevErrTimeout);
-          *abort_flag = 1;
-          failed = true;
-          break;
-        }
-        tc_fence_after();
-        uint32_t rn[2][32], ro[2][32];
-        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
-        __syncwarp();
-        tmem_ld32(sbase, rn[0]);
-        tmem_ld32(sbase + 32, rn[1]);
-        if (has_old) {
-          tmem_ld32(sbase + 64, ro[0]);
-          tmem_ld32(sbase + 96, ro[1]);
-        }
-        tmem_wait_ld();
-        // column tokens of this tile
         const int c0 = t * kAtCols;
-        const int last_c = min(c0 + kAtCols, g.kc) - 1;
-        const int last_tok = hcols ? __ldg(hcols + last_c) : last_c;
+        const int c_end = min(c0 + kAtCols, g.kc);
+        const int last_tok = hcols ? __ldg(hcols + c_end - 1) : c_end - 1;
         const bool need_mask = (c0 + kAtCols > g.kc) || (last_tok > wmin);
-        // scores in the log2 domain, masked columns -> -inf (kept as float bits in place)
+        // the valid columns of this tile for this row form a prefix (columns ascend)
+        int nvalid = kAtCols;
+        if (need_mask) {
+          if (tok < 0) {
+            nvalid = 0;
+          } else {
+            int lo = c0, hi = c_end;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              const int ct = hcols ? __ldg(hcols + mid) : mid;
+              if (ct <= tok) lo = mid + 1;
+              else hi = mid;
+            }
+            nvalid = lo - c0;
+          }
+        }
+        const int first = half * 32;  // this thread's first column in the tile
+        wait_or_die(&s_full[b], (u >> 1) & 1);
+        uint32_t rn[32], ro[32];
+        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
+        float mx = -INFINITY;
+        if (!dead) {
+          __syncwarp();
+          tmem_ld32(sbase + first, rn);
+          if (has_old) tmem_ld32(sbase + 64 + first, ro);
+          tmem_wait_ld();
+          if (nvalid >= first + 32) {
 #pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          float vn = __uint_as_float(rn[e >> 5][e & 31]) * g.scale_log2;
-          float vo = has_old ? __uint_as_float(ro[e >> 5][e & 31]) * g.scale_log2 : -INFINITY;
-          if (need_mask || tok < 0) {
-            const int cj = c0 + e;
-            const int ct = cj < g.kc ? (hcols ? __ldg(hcols + cj) : cj) : 0x7fffffff;
-            if (tok < 0 || ct > tok) {
-              vn = -INFINITY;
-              vo = -INFINITY;
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(rn[e]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (first + e >= nvalid) {
+                rn[e] = 0xff800000u;  // -inf
+                ro[e] = 0xff800000u;
+              }
+              mx = fmaxf(mx, __uint_as_float(rn[e]));
             }
           }
-          rn[e >> 5][e & 31] = __float_as_uint(vn);
-          ro[e >> 5][e & 31] = __float_as_uint(vo);
         }
-        float mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 64; ++e) mx = fmaxf(mx, __uint_as_float(rn[e >> 5][e & 31]));
+        float* xm = xchg + (b * 2) * 128;  // [half][128] of this parity
+        xm[half * 128 + row] = mx;
+        named_bar_sync(pair_bar, 64);
+        mx = fmaxf(mx, xm[(1 - half) * 128 + row]);
+        if (dead) continue;
         const bool need = mx > m_ref + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           // raise the reference of this warp's rows: N and Z scale by 2^(m_ref - mx)
@@ -369,87 +403,79 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           const float f = need ? ex2(m_ref - new_ref) : 1.f;
           if (t > 0) {
             const uint32_t up = u - 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[up & 1], (up >> 1) & 1))) {
-              set_error(g.err, kDevErrTimeout);
-              *abort_flag = 1;
-              failed = true;
-              break;
-            }
-            tc_fence_after();
+            wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+            if (dead) continue;
           }
-          uint32_t r[32];
-#pragma unroll
-          for (int cc = 0; cc < DH; cc += 32) {
+#pragma unroll 1
+          for (int cc = 0; cc < kHalfCols; cc += 16) {
+            uint32_t r[16];
             __syncwarp();
-            tmem_ld32(tmem + lane_base + C::kColN + cc, r);
+            tmem_ld16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
             __syncwarp();
-            tmem_st32(tmem + lane_base + C::kColN + cc, r);
+            tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
           }
           tmem_wait_st();
           z *= f;
           m_ref = new_ref;
         }
-        uint32_t pk[32];
+        uint32_t pk[16];
         float zs = 0.f;
 #pragma unroll
-        for (int e2 = 0; e2 < 32; ++e2) {
-          const float x0 = __uint_as_float(rn[(2 * e2) >> 5][(2 * e2) & 31]);
-          const float x1 = __uint_as_float(rn[(2 * e2 + 1) >> 5][(2 * e2 + 1) & 31]);
-          const float p0 = x0 == -INFINITY ? 0.f : ex2(x0 - m_ref);
-          const float p1 = x1 == -INFINITY ? 0.f : ex2(x1 - m_ref);
+        for (int e2 = 0; e2 < 16; ++e2) {
+          const float p0 = ex2(__uint_as_float(rn[2 * e2]) - m_ref);
+          const float p1 = ex2(__uint_as_float(rn[2 * e2 + 1]) - m_ref);
           zs += p0 + p1;
           pk[e2] = pack_half2(p0, p1);
         }
         __syncwarp();
-        tmem_st32(sbase, pk);
+        tmem_st16(sbase + half * 16, pk);
         if (has_old) {
 #pragma unroll
-          for (int e2 = 0; e2 < 32; ++e2) {
-            const float x0 = __uint_as_float(ro[(2 * e2) >> 5][(2 * e2) & 31]);
-            const float x1 = __uint_as_float(ro[(2 * e2 + 1) >> 5][(2 * e2 + 1) & 31]);
-            const float p0 = x0 == -INFINITY ? 0.f : ex2(x0 - m_ref);
-            const float p1 = x1 == -INFINITY ? 0.f : ex2(x1 - m_ref);
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float p0 = ex2(__uint_as_float(ro[2 * e2]) - m_ref);
+            const float p1 = ex2(__uint_as_float(ro[2 * e2 + 1]) - m_ref);
             zs -= p0 + p1;
             pk[e2] = pack_half2(-p0, -p1);
           }
           __syncwarp();
-          tmem_st32(sbase + 32, pk);
+          tmem_st16(sbase + 32 + half * 16, pk);
         }
         z += zs;
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
       }
-      if (failed) break;
-      // write back: wait for the last P.V of this item
       if (nt > 0) {
         const uint32_t up = u - 1;
-        if (!__all_sync(0xffffffffu, mbar_wait(&pv_done[up & 1], (up >> 1) & 1))) {
-          set_error(g.err, kDevErrTimeout);
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
+        wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
       }
-      const float inv = 1.f / z;
-#pragma unroll
-      for (int cc = 0; cc < DH; cc += 32) {
-        uint32_t r[32];
+      // combine the two halves' sums
+      float* xz = xchg + 4 * 128;
+      xz[half * 128 + row] = z;
+      named_bar_sync(pair_bar, 64);
+      const float z_row = xz[row] + xz[128 + row];
+      named_bar_sync(pair_bar, 64);
+      if (dead) continue;
+      const float inv = 1.f / z_row;
+#pragma unroll 1
+      for (int cc = 0; cc < kHalfCols; cc += 16) {
+        uint32_t r[16];
         __syncwarp();
-        tmem_ld32(tmem + lane_base + C::kColN + cc, r);
+        tmem_ld16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
         tmem_wait_ld();
         if (tok >= 0) {
-          float4* nd = reinterpret_cast<float4*>(g.n_out + ((size_t)h * g.S + tok) * DH + cc);
+          const int col = half * kHalfCols + cc;
+          float4* nd = reinterpret_cast<float4*>(g.n_out + ((size_t)h * g.S + tok) * DH + col);
 #pragma unroll
-          for (int v = 0; v < 8; ++v)
+          for (int v = 0; v < 4; ++v)
             nd[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
                                 __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          uint4* od = reinterpret_cast<uint4*>(g.o + (size_t)tok * HD + (size_t)h * DH + cc);
+          uint4* od = reinterpret_cast<uint4*>(g.o + (size_t)tok * HD + (size_t)h * DH + col);
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
+          for (int v = 0; v < 2; ++v) {
             uint32_t w[4];
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
@@ -461,16 +487,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           }
         }
       }
-      if (tok >= 0) {
+      if (tok >= 0 && half == 0) {
         g.m_out[(size_t)h * g.S + tok] = m_ref / kAtLog2e;
-        g.z_out[(size_t)h * g.S + tok] = z;
+        g.z_out[(size_t)h * g.S + tok] = z_row;
       }
       tc_fence_before();
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 8) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }

@@ -349,6 +349,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
+      int issued[kTcStages];
+      for (int s2 = 0; s2 < kTcStages; ++s2) issued[s2] = -1;
       for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
         const int n0 = (tile % n_tiles) * kTcBN;
         for (int kt = 0; kt < KT; ++kt) {
@@ -359,12 +361,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
           }
           mbar_arrive_expect_tx(&full[stage], kTcBBytes);
           tma_load_2d(sB + stage * kTcBBytes, &tmap_b, kt * kTcBK, n0, &full[stage]);
+          issued[stage] = phase;
           if (++stage == kTcStages) {
             stage = 0;
             phase ^= 1;
           }
         }
       }
+      // never leave with a copy in flight: the full barrier of each stage's last
+      // load completes once its bytes (and the A rows) have landed (bounded wait)
+      for (int s2 = 0; s2 < kTcStages; ++s2)
+        if (issued[s2] >= 0) (void)mbar_wait(&full[s2], (uint32_t)issued[s2]);
     }
   } else if (warp == 5) {
     // ---- MMA issue

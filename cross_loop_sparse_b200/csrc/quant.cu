@@ -177,14 +177,15 @@ int launch_kv_quant(const flashloop_params* p, int loop, const float* k_new, con
 
 // (a5) Rebuild Khat^(r-1), Khat^(r), Vhat^(r-1), Vhat^(r) of the selected
 // columns (loop 1 / dense: Khat^(1), Vhat^(1) of every token) as fp16:
-// K as [H, kcp, dh] rows, V transposed as [H, dh, kcp] so that both feed the
-// attention MMAs as K-major tiles.  [FlashLoop App. G]: only the selected
+// K as [H, kcp, dh] rows scaled by `kscale` (log2(e)/sqrt(dh), so that q.k
+// comes out in log2 units; one fp16 rounding either way), V transposed as
+// [H, dh, kcp], so that both feed the attention MMAs as K-major tiles.  [FlashLoop App. G]: only the selected
 // columns are rebuilt, never the full cache.  One block = 64 columns of one
 // head; V rows are staged in shared memory and written transposed.
 template <int DH>
 __global__ void __launch_bounds__(kQuantThreads)
 selcol_dequant_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, int H, int loop,
-                      KVStreams Ks, KVStreams Vs, LoopTables lt, __half* k_old, __half* k_new,
+                      float kscale, KVStreams Ks, KVStreams Vs, LoopTables lt, __half* k_old, __half* k_new,
                       __half* vt_old, __half* vt_new, int32_t* err) {
   constexpr int E = DH / 32;
   __shared__ __align__(16) __half sv[2][64][DH + 8];
@@ -229,10 +230,10 @@ selcol_dequant_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, 
         if (col < kcp) {
           const size_t off = ((size_t)h * kcp + col) * DH + lane * E;
 #pragma unroll
-          for (int e = 0; e < E; ++e) k_new[off + e] = __float2half_rn(acc[e]);
+          for (int e = 0; e < E; ++e) k_new[off + e] = __float2half_rn(acc[e] * kscale);
           if (has_old) {
 #pragma unroll
-            for (int e = 0; e < E; ++e) k_old[off + e] = __float2half_rn(oldv[e]);
+            for (int e = 0; e < E; ++e) k_old[off + e] = __float2half_rn(oldv[e] * kscale);
           }
         }
       } else {
@@ -263,12 +264,13 @@ int launch_selcol_dequant(const flashloop_params* p, int loop, const int32_t* co
   dim3 grid((kcp + 63) / 64, H);
   const KVStreams Ks = kv_streams(st->k), Vs = kv_streams(st->v);
   const LoopTables lt = loop_tables(p, st);
+  const float kscale = 1.4426950408889634f / sqrtf(static_cast<float>(p->head_dim));
   if (p->head_dim == 128) {
     selcol_dequant_kernel<128><<<grid, kQuantThreads, 0, stream>>>(
-        cols, kc, kcp, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
+        cols, kc, kcp, p->seq, H, loop, kscale, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
   } else {
     selcol_dequant_kernel<64><<<grid, kQuantThreads, 0, stream>>>(
-        cols, kc, kcp, p->seq, H, loop, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
+        cols, kc, kcp, p->seq, H, loop, kscale, Ks, Vs, lt, k_old, k_new, vt_old, vt_new, st->err_word);
   }
   return launch_status();
 }
