@@ -183,4 +183,23 @@ __device__ __forceinline__ void unpack_codes(const uint8_t* row, int e0, int bit
   }
 }
 
+// Quantiser code of x with stored scale s > 0: clamp(rint(fl(x / s)), -qmax, qmax)
+// where fl is the IEEE round-to-nearest float32 quotient.  The quotient is
+// taken from an approximate reciprocal (a few ulps off, i.e. < 2^-16 for
+// |x/s| <= 128); only when it falls within 2^-12 of a half-integer, where the
+// two could round differently, is the exact IEEE quotient computed.  The
+// result is therefore identical to the definition for every input.
+__device__ __forceinline__ float quant_code(float x, float s, float rs, int qmax) {
+  const float q = x * rs;
+  float c = rintf(q);
+  if (fabsf(q - c) > 0.5f - 2.44140625e-4f) c = rintf(__fdiv_rn(x, s));
+  return fminf(fmaxf(c, static_cast<float>(-qmax)), static_cast<float>(qmax));
+}
+
+__device__ __forceinline__ float approx_rcp(float s) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;\n" : "=f"(r) : "f"(s));
+  return r;
+}
+
 }  // namespace fl

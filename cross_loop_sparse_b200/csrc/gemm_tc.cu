@@ -10,16 +10,19 @@
 // Persistent, warp-specialised kernel: tile 128 rows x 256 columns, K step 64,
 // 4-stage shared-memory ring, two TMEM accumulators (512 columns) so the
 // epilogue of one tile overlaps the main loop of the next.
-//   warps 0-3  gather the A rows (active tokens) with 16-byte cp.async into
-//              the 128-byte-swizzled layout, arrive when their copies land;
-//   warp 4     allocates TMEM; lane 0 streams the weight tiles by TMA;
-//   warp 5     lane 0 issues tcgen05.mma (M128 N256 K16, bf16 -> f32);
-//   warps 6-9  epilogue, one TMEM lane (= tile row) per thread:
-//              OUT  -> bf16 Y at the token's row;
-//              QKV  -> RoPE (table computed in double) on q and k, bf16 q at
-//                      the token's row, and either float32 k/v at the row's
-//                      compact position or, fused, the loop's INT8 base /
-//                      INT4 / INT2 residual codes and fp16 scales.
+//   warps 0-1   gather the A rows (active tokens) with 16-byte cp.async into
+//               the 128-byte-swizzled layout and arrive when their copies land
+//               (a TMA tile::gather4 of four 128-byte rows per request was
+//               measured 2.8x slower on this shape);
+//   warp 2      allocates TMEM; lane 0 streams the weight tiles by TMA;
+//   warp 3      lane 0 issues tcgen05.mma (M128 N256 K16, bf16 -> f32);
+//   warps 4-11  epilogue, two warps per TMEM lane quarter (one per 128-column
+//               half of the tile), one row per thread:
+//               OUT  -> bf16 Y at the token's row;
+//               QKV  -> RoPE (table computed in double) on q and k, bf16 q at
+//                       the token's row, and either float32 k/v at the row's
+//                       compact position or, fused, the loop's INT8 base /
+//                       INT4 / INT2 residual codes and fp16 scales.
 // Every wait is bounded; a wait that gives up records FLASHLOOP error 3 and
 // the block unwinds, releasing its TMEM.
 #include <cuda.h>
@@ -30,7 +33,8 @@
 
 namespace fl {
 
-constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4, kTcThreads = 320;
+constexpr int kTcBM = 128, kTcBN = 256, kTcBK = 64, kTcStages = 4, kTcThreads = 384;
+constexpr int kTcEpiThreads = 256, kTcProdThreads = 64;
 constexpr int kTcABytes = kTcBM * kTcBK * 2;  // 16 KiB
 constexpr int kTcBBytes = kTcBN * kTcBK * 2;  // 32 KiB
 constexpr int kTcSmem = 1024 + kTcStages * (kTcABytes + kTcBBytes) + 256;
@@ -122,15 +126,11 @@ __device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits
   uint16_t sbits = __half_as_ushort(hs);
   if ((sbits & 0x7FFFu) == 0x7C00u) sbits = (sbits & 0x8000u) | 0x7BFFu;
   const float s = __half2float(__ushort_as_half(sbits));
+  const float rs = s > 0.f ? approx_rcp(s) : 0.f;
   uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
-    int c = 0;
-    if (s > 0.f) {
-      float q = rintf(__fdiv_rn(x[e], s));
-      q = fminf(fmaxf(q, static_cast<float>(-qmax)), static_cast<float>(qmax));
-      c = static_cast<int>(q);
-    }
+    const int c = s > 0.f ? static_cast<int>(quant_code(x[e], s, rs, qmax)) : 0;
     const int bit = e * bits;
     w[bit >> 5] |= (static_cast<uint32_t>(c) & ((1u << bits) - 1u)) << (bit & 31);
   }
@@ -147,7 +147,7 @@ __device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits
 
 template <int DH>
 __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int m0, int n0, int row,
-                                              int n_rows, uint32_t tbase) {
+                                              int n_rows, uint32_t tbase, int half) {
   const int a = m0 + row;
   int t = -1;
   if (a < n_rows) {
@@ -156,7 +156,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int
   }
   if (mode == kTcOut) {
 #pragma unroll 1
-    for (int c0 = 0; c0 < kTcBN; c0 += 32) {
+    for (int c0 = half * 128; c0 < half * 128 + 128; c0 += 32) {
       uint32_t r[32];
       __syncwarp();
       tmem_ld32(tbase + c0, r);
@@ -180,11 +180,12 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int
   const int section = n0 / d;  // 0 = q, 1 = k, 2 = v
   const int c_base = n0 - section * d;
 #pragma unroll 1
-  for (int hl = 0; hl < kTcBN / DH; ++hl) {
-    const int h = (c_base + hl * DH) / DH;
+  for (int hl = 0; hl < 128 / DH; ++hl) {
+    const int hcol = half * 128 + hl * DH;  // first tile column of this head
+    const int h = (c_base + hcol) / DH;
 #pragma unroll 1
     for (int j = 0; j < kChunksPerHalf; ++j) {
-      const int lo = hl * DH + j * 32, hi = lo + kHalf;
+      const int lo = hcol + j * 32, hi = lo + kHalf;
       uint32_t rl[32], rh[32];
       __syncwarp();
       tmem_ld32(tbase + lo, rl);
@@ -280,17 +281,17 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kTcStages; ++s) {
-      mbar_init(&full[s], 128 + 1);
+      mbar_init(&full[s], kTcProdThreads + 1);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 128);
+      mbar_init(&acc_empty[b], kTcEpiThreads);
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 4) {
+  if (warp == 2) {
     tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
@@ -299,19 +300,19 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  if (warp < 4) {
-    // ---- A producers: gather the active rows
+  if (warp < 2) {
+    // ---- A producers: gather the active rows (16 rows x 8 chunks per pass)
     const int tid = threadIdx.x;
     const int chunk = tid & 7;
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x) {
       const int m0 = (tile / n_tiles) * kTcBM;
-      const uint16_t* src[8];
-      int ok[8];
+      const uint16_t* src[16];
+      int ok[16];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const int r = (tid >> 3) + 16 * i;
+      for (int i = 0; i < 16; ++i) {
+        const int r = (tid >> 3) + 8 * i;
         const int a = m0 + r;
         int t = -1;
         if (a < n_rows) {
@@ -332,8 +333,8 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
         }
         uint8_t* dst = sA + stage * kTcABytes;
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const int r = (tid >> 3) + 16 * i;
+        for (int i = 0; i < 16; ++i) {
+          const int r = (tid >> 3) + 8 * i;
           cp_async16(dst + sw128_offset(r, chunk), src[i] + kt * kTcBK, ok[i] ? 16 : 0);
         }
         cp_async_mbar_arrive_noinc(&full[stage]);
@@ -344,7 +345,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
       }
     }
     cp_async_wait_all();
-  } else if (warp == 4) {
+  } else if (warp == 2) {
     // ---- weight tiles by TMA
     if (lane == 0) {
       int stage = 0;
@@ -373,7 +374,7 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
       for (int s2 = 0; s2 < kTcStages; ++s2)
         if (issued[s2] >= 0) (void)mbar_wait(&full[s2], (uint32_t)issued[s2]);
     }
-  } else if (warp == 5) {
+  } else if (warp == 3) {
     // ---- MMA issue
     if (lane == 0) {
       int stage = 0;
@@ -417,14 +418,15 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
       }
     }
   } else {
-    // ---- epilogue: one TMEM lane (tile row) per thread
+    // ---- epilogue: warps 4-11, two per TMEM lane quarter, one row per thread
     const int lane_grp = warp & 3;
+    const int half = (warp - 4) >> 2;
     const int row = lane_grp * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
-      if (!mbar_wait(&acc_full[buf], acc_phase)) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], acc_phase))) {
         set_error(g.err, kDevErrTimeout);
         *abort_flag = 1;
         break;
@@ -433,14 +435,14 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
       const int m0 = (tile / n_tiles) * kTcBM;
       const int n0 = (tile % n_tiles) * kTcBN;
       const uint32_t tbase = tmem_base + ((uint32_t)(lane_grp * 32) << 16) + buf * kTcBN;
-      epilogue_tile<DH>(g, mode, m0, n0, row, n_rows, tbase);
+      epilogue_tile<DH>(g, mode, m0, n0, row, n_rows, tbase, half);
       tc_fence_before();
       mbar_arrive(&acc_empty[buf]);
     }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 2) {
     tc_fence_after();
     tmem_dealloc(tmem_base, 512);
   }

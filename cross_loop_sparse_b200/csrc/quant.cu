@@ -70,14 +70,10 @@ __device__ __forceinline__ void quantize_store(const float (&x)[E], int bits, in
   const float s = half_bits_to_float(sbits);
   uint32_t packed = 0;
   const uint32_t mask = (1u << bits) - 1u;
+  const float rs = s > 0.f ? approx_rcp(s) : 0.f;
 #pragma unroll
   for (int e = 0; e < E; ++e) {
-    int c = 0;
-    if (s > 0.f) {
-      float q = rintf(__fdiv_rn(x[e], s));
-      q = fminf(fmaxf(q, static_cast<float>(-qmax)), static_cast<float>(qmax));
-      c = static_cast<int>(q);
-    }
+    const int c = s > 0.f ? static_cast<int>(quant_code(x[e], s, rs, qmax)) : 0;
     packed |= (static_cast<uint32_t>(c) & mask) << (e * bits);
   }
   const int lane_bits = E * bits;

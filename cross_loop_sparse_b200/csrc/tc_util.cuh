@@ -214,3 +214,19 @@ __device__ __forceinline__ void named_bar_arrive(int id, int count) {
 }
 
 }  // namespace fl
+
+namespace fl {
+
+// TMA gather of four rows (r0..r3) x one 64-element box starting at column x
+// into 4 consecutive 128-byte rows of shared memory (2-D map, box one row
+// high).  No multicast.
+__device__ __forceinline__ void tma_gather4(void* dst, const void* tmap, int x, int r0, int r1, int r2, int r3,
+                                            uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];\n"
+      ::"r"(smem_u32(dst)), "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+}  // namespace fl
