@@ -29,6 +29,10 @@ int launch_qkv_quant_gemm(const flashloop_params*, int, const uint16_t*, const i
 
 namespace fl {
 int launch_attn_tc(const flashloop_params*, const AttnArgs&, int, cudaStream_t);
+DecodeLayout decode_layout(const flashloop_params*);
+int launch_decode_attn(const flashloop_params*, int, const flashloop_state*, flashloop_decode_state*, cudaStream_t);
+int launch_decode_step(const flashloop_params*, int, const uint16_t*, const uint16_t*, const uint16_t*,
+                       const flashloop_state*, flashloop_decode_state*, cudaStream_t);
 int launch_colmass(const flashloop_params*, const ColmassArgs&, cudaStream_t);
 
 // ---------------------------------------------------------------------------
@@ -192,21 +196,21 @@ int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t*
                         uint16_t* q_out, void* stream) {
   int rc = check_common(p);
   if (rc != FLASHLOOP_OK) return rc;
-  if (loop < 1 || loop > p->n_loops || !x || !w_qkv || !st || !q_out || !st->rope_cs)
+  if (loop < 1 || loop > p->n_loops || !x || !w_qkv || !st || !st->rope_cs)
     return FLASHLOOP_ERR_INVALID_ARG;
   if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
     return FLASHLOOP_ERR_INVALID_ARG;
+  if (active != nullptr && n_active == nullptr) return FLASHLOOP_ERR_INVALID_ARG;
   if (loop >= 2) {
-    if (!active || !n_active) return FLASHLOOP_ERR_INVALID_ARG;
+    if (!active) return FLASHLOOP_ERR_INVALID_ARG;
     for (int l = 2; l <= loop; ++l) {
       if (!st->k.res_codes[l - 1] || !st->k.res_scales[l - 1] || !st->v.res_codes[l - 1] ||
-          !st->v.res_scales[l - 1])
+          !st->v.res_scales[l - 1] || !st->slot[l - 1])
         return FLASHLOOP_ERR_INVALID_ARG;
-      if (l < loop && !st->slot[l - 1]) return FLASHLOOP_ERR_INVALID_ARG;
     }
   }
-  return launch_qkv_quant_gemm(p, loop, x, loop == 1 ? nullptr : active, loop == 1 ? nullptr : n_active,
-                               capacity_of(p, loop), w_qkv, st, q_out, as_stream(stream));
+  return launch_qkv_quant_gemm(p, loop, x, active, active ? n_active : nullptr,
+                               active ? capacity_of(p, loop) : p->seq, w_qkv, st, q_out, as_stream(stream));
 }
 
 int flashloop_topk_columns(const flashloop_params* p, const float* mass, const int32_t* candidates,
@@ -376,6 +380,104 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   rc = flashloop_sparse_attn_update(p, loop, st, want_cm, stream);
   if (rc != FLASHLOOP_OK) return rc;
   return launch_out_gemm(p, st->O, act, n_act, cap, w_o, st->Y, st->err_word, s);
+}
+
+size_t flashloop_kv_workspace_bytes(const flashloop_params* p) {
+  if (check_params(p) != FLASHLOOP_OK) return 0;
+  return workspace_layout(p).flags + (size_t)p->seq;
+}
+
+int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur, const uint16_t* x_prev,
+                      const uint16_t* w_qkv, flashloop_state* st, void* stream) {
+  int rc = check_common(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop < 1 || loop > p->n_loops || !x_cur || !w_qkv || !st || !st->rope_cs || !st->err_word)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  cudaStream_t s = as_stream(stream);
+  if (loop == 1) return launch_qkv_quant_gemm(p, 1, x_cur, nullptr, nullptr, p->seq, w_qkv, st, nullptr, s);
+  if (!x_prev || !st->n_active || !st->workspace || st->workspace_bytes < flashloop_kv_workspace_bytes(p))
+    return FLASHLOOP_ERR_INVALID_ARG;
+  for (int l = 2; l <= loop; ++l)
+    if (!st->active[l - 1] || !st->slot[l - 1] || !st->k.res_codes[l - 1] || !st->k.res_scales[l - 1] ||
+        !st->v.res_codes[l - 1] || !st->v.res_scales[l - 1])
+      return FLASHLOOP_ERR_INVALID_ARG;
+  int32_t* act = st->active[loop - 1];
+  int32_t* n_act = st->n_active + (loop - 1);
+  const int cap = capacity_of(p, loop);
+  rc = launch_gate(p, x_cur, x_prev, loop == 2 ? nullptr : st->active[loop - 2],
+                   loop == 2 ? nullptr : st->n_active + (loop - 2), capacity_of(p, loop - 1), act,
+                   st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
+  if (rc != FLASHLOOP_OK) return rc;
+  return launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, nullptr, s);
+}
+
+// ---------------------------------------------------------------------------
+// decode
+// ---------------------------------------------------------------------------
+static int check_decode_params(const flashloop_params* p) {
+  int rc = check_params(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (p->batch < 1 || p->batch > 64) return FLASHLOOP_ERR_INVALID_ARG;
+  const int hd = p->n_heads * p->head_dim, hg = hd / 32;
+  if (hd % 256 != 0 || 256 % hg != 0 || hg % 8 != 0) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (p->n_loops >= 2 && p->topk[1] > p->seq + 1) return FLASHLOOP_ERR_INVALID_ARG;
+  return FLASHLOOP_OK;
+}
+
+static int check_decode_state(const flashloop_params* p, int loop, const flashloop_state* ctx,
+                              const flashloop_decode_state* ds) {
+  if (!ctx || !ds || !ds->err_word || !ds->workspace || !ds->O) return FLASHLOOP_ERR_INVALID_ARG;
+  if (ds->workspace_bytes < decode_layout(p).total) return FLASHLOOP_ERR_INVALID_ARG;
+  if (!ctx->k.base_codes || !ctx->k.base_scales || !ctx->v.base_codes || !ctx->v.base_scales ||
+      !ds->k.base_codes || !ds->k.base_scales || !ds->v.base_codes || !ds->v.base_scales)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  for (int l = 2; l <= loop; ++l)
+    if (!ctx->slot[l - 1] || !ctx->k.res_codes[l - 1] || !ctx->k.res_scales[l - 1] || !ctx->v.res_codes[l - 1] ||
+        !ctx->v.res_scales[l - 1] || !ds->k.res_codes[l - 1] || !ds->k.res_scales[l - 1] ||
+        !ds->v.res_codes[l - 1] || !ds->v.res_scales[l - 1])
+      return FLASHLOOP_ERR_INVALID_ARG;
+  const int cur = slot_of_loop(loop);
+  if (!ds->q[cur] || !ds->m[cur] || !ds->Z[cur] || !ds->N[cur]) return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop >= 2) {
+    const int prev = slot_of_loop(loop - 1);
+    if (!ds->q[prev] || !ds->m[prev] || !ds->Z[prev] || !ds->N[prev]) return FLASHLOOP_ERR_INVALID_ARG;
+  }
+  if (p->n_loops >= 2 && !ds->cols) return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop == 1 && !ds->probs) return FLASHLOOP_ERR_INVALID_ARG;
+  return FLASHLOOP_OK;
+}
+
+size_t flashloop_decode_workspace_bytes(const flashloop_params* p) {
+  if (check_decode_params(p) != FLASHLOOP_OK) return 0;
+  return decode_layout(p).total;
+}
+
+int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
+                          flashloop_decode_state* ds, void* stream) {
+  int rc = check_decode_params(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  rc = check_arch();
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop < 1 || loop > p->n_loops) return FLASHLOOP_ERR_INVALID_ARG;
+  rc = check_decode_state(p, loop, ctx, ds);
+  if (rc != FLASHLOOP_OK) return rc;
+  return launch_decode_attn(p, loop, ctx, ds, as_stream(stream));
+}
+
+int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_t* x_tok,
+                          const uint16_t* w_qkv, const uint16_t* w_o, const flashloop_state* ctx,
+                          flashloop_decode_state* ds, void* stream) {
+  int rc = check_decode_params(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  rc = check_arch();
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop < 1 || loop > p->n_loops || !x_tok || !w_qkv || !w_o) return FLASHLOOP_ERR_INVALID_ARG;
+  rc = check_decode_state(p, loop, ctx, ds);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (!ds->rope_cs || !ds->Y) return FLASHLOOP_ERR_INVALID_ARG;
+  return launch_decode_step(p, loop, x_tok, w_qkv, w_o, ctx, ds, as_stream(stream));
 }
 
 int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* stream) {

@@ -85,6 +85,14 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   return w;
 }
 
+// Decode scratch layout (offsets into flashloop_decode_state::workspace) and
+// the split of the dense loop-1 pass (nsplit column ranges of `range`
+// columns per sequence) and of the sparse loops (nblk ranges per head).
+struct DecodeLayout {
+  size_t k_new, v_new, scores, part_m, part_mu, part_Z, part_N, total;
+  int nsplit, range, nblk;
+};
+
 template <typename T>
 inline T* ws_ptr(void* base, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(base) + off);

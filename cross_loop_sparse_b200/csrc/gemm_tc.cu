@@ -209,6 +209,7 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int
       }
       const int col_lo = c_base + lo, col_hi = c_base + hi;
       if (section == 0) {
+        if (g.q_out == nullptr) continue;  // a decode context stores only its K/V
         uint16_t* dst_l = g.q_out + (size_t)t * d + col_lo;
         uint16_t* dst_h = g.q_out + (size_t)t * d + col_hi;
 #pragma unroll
@@ -246,8 +247,10 @@ __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int
 #pragma unroll
           for (int e = 0; e < 32; ++e) xh[e] = xh[e] - prev[e];
         }
-        uint8_t* crow = codes + ((size_t)a * H + h) * row_bytes;
-        uint16_t* srow = scales + ((size_t)a * H + h) * (DH / 32);
+        // the base is indexed by token, a residual by the token's slot in this loop's active list
+        const int dst_row = g.loop == 1 ? t : g.lt.slot[g.loop - 1][t];
+        uint8_t* crow = codes + ((size_t)dst_row * H + h) * row_bytes;
+        uint16_t* srow = scales + ((size_t)dst_row * H + h) * (DH / 32);
         quant_store_group(xl, bits, crow + g_lo * 4 * bits, srow + g_lo);
         quant_store_group(xh, bits, crow + g_hi * 4 * bits, srow + g_hi);
       }

@@ -42,7 +42,7 @@ __device__ __forceinline__ void reconstruct_lane(const KVStreams& kv, const Loop
     for (int e = 0; e < E; ++e) acc[e] = static_cast<float>(row[e0 + e]) * s;
   }
   for (int l = 2; l <= upto; ++l) {
-    const int sl = lt.slot[l - 1][t];
+    const int sl = lt.slot[l - 1] ? lt.slot[l - 1][t] : t;  // no slot map: every row present at its own index
     if (sl < 0) continue;
     const int b = lt.bits[l - 1];
     const uint8_t* row = kv.res_codes[l - 1] + ((size_t)sl * H + h) * (DH * b / 8);
@@ -168,6 +168,34 @@ int launch_kv_quant(const flashloop_params* p, int loop, const float* k_new, con
     kv_quant_kernel<64><<<(int)grid, kQuantThreads, 0, stream>>>(
         k_new, v_new, active, n_active, cap, p->seq, H, loop, Ks, Vs, lt, kc, ks, vc, vs, st->err_word);
   }
+  return launch_status();
+}
+
+// The same quantisation for n_rows rows that are present at every loop (the
+// decode tokens): row a of k_new / v_new goes to row a of the base (loop 1)
+// or of the loop's residual stream, and reconstruction reads row a of every
+// earlier stream.
+int launch_kv_quant_rows(int dh, int loop, int n_rows, int H, const int* bits, const float* k_new,
+                         const float* v_new, const flashloop_kv& k, const flashloop_kv& v, int32_t* err,
+                         cudaStream_t stream) {
+  const long long items = (long long)n_rows * H * 2;
+  const int grid = (int)((items + (kQuantThreads / 32) - 1) / (kQuantThreads / 32));
+  const KVStreams Ks = kv_streams(k), Vs = kv_streams(v);
+  LoopTables lt{};
+  for (int i = 0; i < FLASHLOOP_MAX_LOOPS; ++i) {
+    lt.slot[i] = nullptr;
+    lt.bits[i] = bits[i];
+  }
+  uint8_t* kc = loop == 1 ? reinterpret_cast<uint8_t*>(k.base_codes) : k.res_codes[loop - 1];
+  uint8_t* vc = loop == 1 ? reinterpret_cast<uint8_t*>(v.base_codes) : v.res_codes[loop - 1];
+  uint16_t* ks = loop == 1 ? k.base_scales : k.res_scales[loop - 1];
+  uint16_t* vs = loop == 1 ? v.base_scales : v.res_scales[loop - 1];
+  if (dh == 128)
+    kv_quant_kernel<128><<<grid, kQuantThreads, 0, stream>>>(k_new, v_new, nullptr, nullptr, n_rows, n_rows, H,
+                                                              loop, Ks, Vs, lt, kc, ks, vc, vs, err);
+  else
+    kv_quant_kernel<64><<<grid, kQuantThreads, 0, stream>>>(k_new, v_new, nullptr, nullptr, n_rows, n_rows, H,
+                                                             loop, Ks, Vs, lt, kc, ks, vc, vs, err);
   return launch_status();
 }
 

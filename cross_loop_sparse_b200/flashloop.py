@@ -48,7 +48,7 @@ class Params(ctypes.Structure):
         p = cls()
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
-        p.n_loops, p.batch = cfg.n_loops, 1
+        p.n_loops, p.batch = cfg.n_loops, (cfg.batch if cfg.decode else 1)
         p.tau = cfg.tau if tau is None else tau
         p.rope_theta = cfg.rope_theta
         ks = cfg.k_per_loop() if topk is None else list(topk)
@@ -72,9 +72,17 @@ class StateC(ctypes.Structure):
                 ("workspace", c_void_p), ("workspace_bytes", c_size_t)]
 
 
+class DecodeStateC(ctypes.Structure):
+    _fields_ = [("k", KV), ("v", KV), ("rope_cs", c_void_p), ("q", c_void_p * 3), ("m", c_void_p * 3),
+                ("Z", c_void_p * 3), ("N", c_void_p * 3), ("probs", c_void_p), ("cols", c_void_p),
+                ("O", c_void_p), ("Y", c_void_p), ("err_word", c_void_p), ("workspace", c_void_p),
+                ("workspace_bytes", c_size_t)]
+
+
 # ----------------------------------------------------------------------------- prototypes
 _P = POINTER(Params)
 _S = POINTER(StateC)
+_D = POINTER(DecodeStateC)
 _V = c_void_p
 _I = c_int32
 _SIG = {
@@ -91,6 +99,11 @@ _SIG = {
     "flashloop_sparse_attn_update": (_I, [_P, _I, _S, _I, _V]),
     "flashloop_out_proj": (_I, [_P, _V, _V, _V, _I, _V, _V, _V]),
     "flashloop_loop_step": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
+    "flashloop_kv_step": (_I, [_P, _I, _V, _V, _V, _S, _V]),
+    "flashloop_kv_workspace_bytes": (c_size_t, [_P]),
+    "flashloop_decode_workspace_bytes": (c_size_t, [_P]),
+    "flashloop_decode_attn": (_I, [_P, _I, _S, _D, _V]),
+    "flashloop_decode_step": (_I, [_P, _I, _V, _V, _V, _S, _D, _V]),
     "flashloop_selection_loop": (_I, [_P, _I]),
     "flashloop_check_error_word": (_I, [_V, POINTER(c_int32), _V]),
     "flashloop_status_string": (ctypes.c_char_p, [_I]),
@@ -221,6 +234,31 @@ def flashloop_loop_step(params, loop, x_cur, x_prev, w_qkv, w_o, state, stream=N
         ctypes.byref(state.c), _stream(stream)))
 
 
+def flashloop_kv_step(params, loop, x_cur, x_prev, w_qkv, state, stream=None):
+    return _check("flashloop_kv_step", _lib.flashloop_kv_step(
+        ctypes.byref(params), loop, _ptr(x_cur), _ptr(x_prev), _ptr(w_qkv), ctypes.byref(state.c),
+        _stream(stream)))
+
+
+def flashloop_kv_workspace_bytes(params: Params) -> int:
+    return int(_lib.flashloop_kv_workspace_bytes(ctypes.byref(params)))
+
+
+def flashloop_decode_workspace_bytes(params: Params) -> int:
+    return int(_lib.flashloop_decode_workspace_bytes(ctypes.byref(params)))
+
+
+def flashloop_decode_attn(params, loop, ctx, dstate, stream=None):
+    return _check("flashloop_decode_attn", _lib.flashloop_decode_attn(
+        ctypes.byref(params), loop, ctypes.byref(ctx.c), ctypes.byref(dstate.c), _stream(stream)))
+
+
+def flashloop_decode_step(params, loop, x_tok, w_qkv, w_o, ctx, dstate, stream=None):
+    return _check("flashloop_decode_step", _lib.flashloop_decode_step(
+        ctypes.byref(params), loop, _ptr(x_tok), _ptr(w_qkv), _ptr(w_o), ctypes.byref(ctx.c),
+        ctypes.byref(dstate.c), _stream(stream)))
+
+
 def flashloop_check_error_word(err_word, stream=None):
     """Returns the device error code (0 = none); synchronises the stream."""
     code = c_int32(0)
@@ -235,7 +273,11 @@ class FlashLoopState:
     """Caller-owned device buffers of one sequence (torch tensors) and the
     C struct that points at them.  Allocation is the only work done here."""
 
-    def __init__(self, params: Params, device="cuda"):
+    def __init__(self, params: Params, device="cuda", kv_only=False, rope_period=None):
+        """kv_only: only what flashloop_kv_step touches (caches, active lists,
+        slot maps, counts, the gate's scratch, RoPE table, error word).
+        rope_period: positions restart every rope_period rows (sequences laid
+        end to end, as a decode context is)."""
         self.params = params
         S, H, dh, d, R = params.seq, params.n_heads, params.head_dim, params.d_model, params.n_loops
         self.device = device
@@ -261,6 +303,22 @@ class FlashLoopState:
             c.active[r - 1], c.slot[r - 1] = act.data_ptr(), slot.data_ptr()
         self.t["n_active"] = z((MAX_LOOPS,), torch.int32)
         c.n_active = self.t["n_active"].data_ptr()
+        self.t["rope_cs"] = z((S, dh // 2, 2), torch.float32)
+        self.t["err"] = z((1,), torch.int32)
+        c.rope_cs, c.err_word = self.t["rope_cs"].data_ptr(), self.t["err"].data_ptr()
+        self.c = c
+        if rope_period is None:
+            flashloop_rope_table(params, S, self.t["rope_cs"])
+        else:
+            assert S % rope_period == 0
+            one = z((rope_period, dh // 2, 2), torch.float32)
+            flashloop_rope_table(params, rope_period, one)
+            self.t["rope_cs"].copy_(one.repeat(S // rope_period, 1, 1))
+        if kv_only:
+            ws = flashloop_kv_workspace_bytes(params)
+            self.t["workspace"] = z((max(ws, 256),), torch.uint8)
+            c.workspace, c.workspace_bytes = self.t["workspace"].data_ptr(), ws
+            return
         for i in range(3):
             self.t[f"q{i}"] = z((S, d), torch.bfloat16)
             self.t[f"m{i}"] = z((H, S), torch.float32)
@@ -277,21 +335,104 @@ class FlashLoopState:
                 c.cols[r - 1] = self.t[f"cols{r}"].data_ptr()
         self.t["O"] = z((S, d), torch.bfloat16)
         self.t["Y"] = z((S, d), torch.bfloat16)
-        self.t["rope_cs"] = z((S, dh // 2, 2), torch.float32)
-        self.t["err"] = z((1,), torch.int32)
         ws = flashloop_workspace_bytes(params)
         self.t["workspace"] = z((max(ws, 256),), torch.uint8)
         c.O, c.Y = self.t["O"].data_ptr(), self.t["Y"].data_ptr()
-        c.rope_cs, c.err_word = self.t["rope_cs"].data_ptr(), self.t["err"].data_ptr()
         c.workspace, c.workspace_bytes = self.t["workspace"].data_ptr(), ws
-        self.c = c
-        flashloop_rope_table(params, S, self.t["rope_cs"])
 
     def __getitem__(self, key):
         return self.t[key]
 
     def cols_for_loop(self, r):
         return self.t[f"cols{flashloop_selection_loop(self.params, r)}"]
+
+    def q_slot(self, r):
+        return 0 if r == 1 else 1 + (r % 2)
+
+    def error_code(self, stream=None):
+        return flashloop_check_error_word(self.t["err"], stream)
+
+
+# ----------------------------------------------------------------------------- decode
+def decode_context_params(params: Params, capacity=None) -> Params:
+    """Params of the B contexts of a decode laid end to end (seq = B*S), the
+    layout flashloop_decode_attn reads; capacities default to B*S."""
+    p = Params()
+    ctypes.pointer(p)[0] = params
+    p.seq = params.batch * params.seq
+    p.batch = 1
+    for r in range(params.n_loops):
+        p.capacity[r] = p.seq if capacity is None else capacity[r]
+    return p
+
+
+class DecodeContext(FlashLoopState):
+    """Caches of the B contexts of a decode (kv-only state of B*S rows, RoPE
+    positions restarting at every sequence)."""
+
+    def __init__(self, params: Params, device="cuda", capacity=None):
+        self.dec_params = params
+        super().__init__(decode_context_params(params, capacity), device, kv_only=True,
+                         rope_period=params.seq)
+
+    def prepare(self, xs, w_qkv, stream=None):
+        """KV path of loops 1..R: xs[r-1] is bf16 [B*S, d] (the contexts of loop r)."""
+        p = self.params
+        for r in range(1, p.n_loops + 1):
+            flashloop_kv_step(p, r, xs[r - 1], xs[r - 2] if r > 1 else None, w_qkv, self, stream)
+
+
+class DecodeState:
+    """Caller-owned device buffers of a decode step (B sequences, one token
+    each at position S) and the C struct that points at them."""
+
+    def __init__(self, params: Params, device="cuda"):
+        self.params = params
+        S, H, dh, d, R, B = (params.seq, params.n_heads, params.head_dim, params.d_model, params.n_loops,
+                             params.batch)
+        dev = torch.device(device)
+        z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)  # noqa: E731
+        self.t = {}
+        c = DecodeStateC()
+        for name, kv in (("k", c.k), ("v", c.v)):
+            base = z((B, H, dh), torch.int8)
+            bs = z((B, H, dh // GROUP), torch.float16)
+            self.t[f"{name}_base"], self.t[f"{name}_base_s"] = base, bs
+            kv.base_codes, kv.base_scales = base.data_ptr(), bs.data_ptr()
+            for r in range(2, R + 1):
+                b = params.bits[r - 1]
+                codes = z((B, H, dh * b // 8), torch.uint8)
+                sc = z((B, H, dh // GROUP), torch.float16)
+                self.t[f"{name}_res{r}"], self.t[f"{name}_res{r}_s"] = codes, sc
+                kv.res_codes[r - 1], kv.res_scales[r - 1] = codes.data_ptr(), sc.data_ptr()
+        for i in range(3):
+            self.t[f"q{i}"] = z((B, d), torch.bfloat16)
+            self.t[f"m{i}"] = z((B, H), torch.float32)
+            self.t[f"Z{i}"] = z((B, H), torch.float32)
+            self.t[f"N{i}"] = z((B, H, dh), torch.float32)
+            c.q[i], c.m[i] = self.t[f"q{i}"].data_ptr(), self.t[f"m{i}"].data_ptr()
+            c.Z[i], c.N[i] = self.t[f"Z{i}"].data_ptr(), self.t[f"N{i}"].data_ptr()
+        self.t["probs"] = z((B, H, S + 1), torch.float32)
+        k = params.topk[1] if R >= 2 else 1
+        self.t["cols"] = z((B, H, k), torch.int32)
+        self.t["O"] = z((B, d), torch.bfloat16)
+        self.t["Y"] = z((B, d), torch.bfloat16)
+        self.t["err"] = z((1,), torch.int32)
+        table = z((S + 1, dh // 2, 2), torch.float32)
+        flashloop_rope_table(params, S + 1, table)
+        self.t["rope_cs"] = table[S].clone()
+        ws = flashloop_decode_workspace_bytes(params)
+        if ws == 0:
+            raise FlashLoopError("flashloop_decode_workspace_bytes", -2)
+        self.t["workspace"] = z((ws,), torch.uint8)
+        c.rope_cs, c.probs, c.cols = (self.t["rope_cs"].data_ptr(), self.t["probs"].data_ptr(),
+                                      self.t["cols"].data_ptr())
+        c.O, c.Y, c.err_word = self.t["O"].data_ptr(), self.t["Y"].data_ptr(), self.t["err"].data_ptr()
+        c.workspace, c.workspace_bytes = self.t["workspace"].data_ptr(), ws
+        self.c = c
+
+    def __getitem__(self, key):
+        return self.t[key]
 
     def q_slot(self, r):
         return 0 if r == 1 else 1 + (r % 2)

@@ -189,10 +189,13 @@ int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const f
 /* (a2)+(a3) fused: the gathered projection of flashloop_qkv_gathered whose
  * epilogue quantises k and v of loop `loop` straight into the state's
  * streams (INT8 base at loop 1, the residual against Xhat^(loop-1) at loop
- * >= 2, stored at the row's position in the active list), with the same
+ * >= 2), with the same
  * arithmetic as flashloop_kv_quant_residual; q (RoPE'd, bf16) goes to
  * q_out[t].  [FlashLoop §4.3, §4.4: KV update fused with quantisation.]
- * loop == 1 projects every token (active ignored). */
+ * The base row of token t is t; a residual row is slot[loop-1][t] (the
+ * token's position in this loop's active list, written by the gate).
+ * loop == 1 with active == NULL projects every token.  q_out may be NULL
+ * (q is then not stored: a decode context needs only its K/V). */
 int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t* x, const int32_t* active,
                         const int32_t* n_active, const uint16_t* w_qkv, flashloop_state* st,
                         uint16_t* q_out, void* stream);
@@ -244,6 +247,85 @@ int flashloop_out_proj(const flashloop_params* p, const uint16_t* o, const int32
 int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur,
                         const uint16_t* x_prev, const uint16_t* w_qkv, const uint16_t* w_o,
                         flashloop_state* st, void* stream);
+
+/* The KV path of one loop, without attention: at loop 1 the INT8 base of
+ * every token; at loop r >= 2 the gate of x_cur against x_prev over loop
+ * r-1's active list (flashloop_gate) and the residual of the active tokens
+ * (flashloop_qkv_quant with q_out = NULL).  Reads/writes st->k, st->v,
+ * st->active, st->slot, st->n_active, st->workspace (the gate's part, see
+ * flashloop_kv_workspace_bytes), st->rope_cs and st->err_word only.
+ * [FlashLoop §4.3: the cross-loop KV store of the converged and active
+ * tokens]; this is what a decode context keeps from its prefill. */
+int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur, const uint16_t* x_prev,
+                      const uint16_t* w_qkv, flashloop_state* st, void* stream);
+
+/* Scratch bytes flashloop_kv_step needs in st->workspace (zero-filled once). */
+size_t flashloop_kv_workspace_bytes(const flashloop_params* p);
+
+/* ---------------------------------------------------------------- decode */
+
+/* (a8) Decode state of B sequences, one new token each at position S =
+ * p->seq (the context length), all device memory, caller-owned.
+ * The token of sequence b has its own K/V streams: base row b, and for every
+ * loop l >= 2 residual row b (the token is active at every loop).
+ * q, m, Z and N use the slots of flashloop_state: loop 1 writes slot 0, loop
+ * r >= 2 reads slot sel(r-1) and writes slot sel(r) = 1 + (r % 2).
+ * m is kept in log2 units: m = max_j q.k_j * log2(e) / sqrt(dh), and
+ * Z = sum_j 2^(s_j - m), so that e^(natural max) * Z is the softmax sum. */
+typedef struct flashloop_decode_state {
+  flashloop_kv k;            /* token streams: base [B, H, dh], residual of loop l [B, H, dh*bits_l/8] */
+  flashloop_kv v;
+  const float* rope_cs;      /* (cos, sin) pairs of position S: [dh/2][2] (row S of flashloop_rope_table) */
+  uint16_t* q[3];            /* bf16 [B, H, dh] query slots */
+  float* m[3];               /* [B, H] */
+  float* Z[3];               /* [B, H] */
+  float* N[3];               /* [B, H, dh] */
+  float* probs;              /* [B, H, S+1] float32 loop-1 attention probabilities of the token */
+  int32_t* cols;             /* [B, H, topk[1]] ascending selected columns in [0, S] (S = the token) */
+  uint16_t* O;               /* bf16 [B, d_model] */
+  uint16_t* Y;               /* bf16 [B, d_model] */
+  int32_t* err_word;         /* device error word, 0 = no error */
+  void* workspace;           /* scratch (need not be cleared) */
+  size_t workspace_bytes;    /* >= flashloop_decode_workspace_bytes(params) */
+} flashloop_decode_state;
+
+/* Scratch bytes of flashloop_decode_step / flashloop_decode_attn (host function).
+ * p->batch = B in [1, 64]; additionally n_heads*head_dim must be a multiple of
+ * 256 and n_heads*head_dim/32 a divisor of 256 that is a multiple of 8
+ * (e.g. 16 x 128, 4 x 64); returns 0 for any other shape. */
+size_t flashloop_decode_workspace_bytes(const flashloop_params* p);
+
+/* (a8) Decode attention of loop `loop` [FlashLoop App. G: custom attention
+ * kernels read the packed anchor and residual streams directly; fused sparse
+ * decode selection].  ctx holds the B contexts' caches as one sequence of B*S
+ * rows (token j of sequence b at row b*S + j; its loop-l residual at row
+ * ctx->slot[l-1][b*S + j], -1 = none), written by the KV path of loops
+ * 1..R (flashloop_gate, flashloop_qkv_quant with p->seq = B*S); only ctx->k,
+ * ctx->v and ctx->slot are read.  Columns 0..S-1 are the context, column S is
+ * the token itself (its streams in ds).
+ * loop 1: dense attention of q (slot 0) over Khat^(1), Vhat^(1) of columns
+ *   0..S (base codes dequantised in the loads): state slot 0, O, probs; then
+ *   cols = per (sequence, head) the topk[1] columns of largest float32
+ *   probability (ties to the lower index), ascending.
+ * loop r >= 2: for the selected columns j,
+ *   s_old = q^(r-1).Khat_j^(r-1)/sqrt(dh), s_new = q^(r).Khat_j^(r)/sqrt(dh),
+ *   m' = max(m, max s_new), Z' = e^(m-m') Z - sum e^(s_old-m') + sum e^(s_new-m'),
+ *   N' likewise with Vhat^(r-1), Vhat^(r); O = N'/Z' (bf16).  Khat/Vhat are
+ *   rebuilt from the packed streams in the loads (float32 sums in loop order).
+ * Argument errors are returned before any launch; a column index outside
+ * [0, S] sets FLASHLOOP_DEVERR_INDEX. */
+int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
+                          flashloop_decode_state* ds, void* stream);
+
+/* (a8) One loop of the decode token, B sequences: q, k, v = x_tok W_qkv^T
+ * (x_tok bf16 [B, d_model], float32 accumulation, RoPE at position S on q and
+ * k, q -> ds->q slot); k and v quantised into the token streams (INT8 base at
+ * loop 1, the residual against the reconstructed previous loop after it,
+ * the arithmetic of flashloop_kv_quant_residual); flashloop_decode_attn; then
+ * Y = bf16(O W_o^T).  The token is active at every loop (no gate). */
+int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_t* x_tok,
+                          const uint16_t* w_qkv, const uint16_t* w_o, const flashloop_state* ctx,
+                          flashloop_decode_state* ds, void* stream);
 
 /* Host helper: the loop whose selection loop r uses (2 <= r): the latest
  * loop l <= r with l == 2 or topk[l-1] < topk[l-2]. */

@@ -533,6 +533,7 @@ class OracleDecode:
         self.O = {}
         self.Y = {}
         self.state = {}
+        self.q = {}
         self.probs = None
 
     def _context_kv(self, r):
@@ -592,6 +593,7 @@ class OracleDecode:
                         m[a:a + 1], Z[a:a + 1], N[a:a + 1])
                     m[a], Z[a], N[a] = m2[0], Z2[0], N2[0]
             q_prev = qt
+            self.q[r] = qt[0]
             O = to_bf16_bits((N / Z[:, None]).reshape(1, Hs * dh))
             self.O[r] = O[0]
             self.state[r] = (m.copy(), Z.copy(), N.copy())
