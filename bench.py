@@ -27,13 +27,15 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workload import CONFIGS, make_hidden_states, make_weights  # noqa: E402
+from workload import CONFIGS, make_decode_tokens, make_hidden_states, make_weights  # noqa: E402
 
 METRIC = "loop-step tokens/s at S=32K,R=4; HBM GB/s and tensor-pipe % of B200 peak"
+DECODE_METRIC = "decode tokens/s (B sequences x 1 token x R loops) at S_ctx=32K,R=4; HBM GB/s of B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) of one loop-2 attention launch at 32K, from the ncu capture summarised in
-# profiles/attn_update_mma_prefill_32k_loop2.md; None once the kernel changes until it is re-captured.
-ATTN_LOOP2_TRAFFIC = {"attn_update_kernel<128>": 736.1e6}
+# DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures summarised
+# under profiles/; None once the kernel changes until it is re-captured.
+ATTN_LOOP2_TRAFFIC = {"attn_tc_kernel<128>": 731.3e6}
+DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": None}
 
 
 def max_over_ranks(value, device=None):
@@ -87,6 +89,12 @@ class ClockSampler:
                 stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.proc = None
+            return
+        # the sampler takes a moment to start: wait for its first line so
+        # that the samples fall inside the timed region that follows
+        t_end = time.time() + 3.0
+        while time.time() < t_end and os.path.getsize(self.path) == 0:
+            time.sleep(0.02)
 
     def stop(self):
         if self.proc is None:
@@ -222,8 +230,8 @@ def run_cuda(args, cfg, rank, world, local_rank):
     achieved = flop2 / (ms2 * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": ATTN_LOOP2_TRAFFIC.get("attn_update_kernel<128>"),
-                "kernel": "attn_update_kernel<128>, loop-2 launch (sparse attention update)",
+                "traffic": ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
+                "kernel": "attn_tc_kernel<128>, loop-2 launch (sparse attention update, tcgen05)",
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
                 "per_loop": {f"loop{r}": {"ms": round(statistics.mean(v), 4),
@@ -281,6 +289,202 @@ def run_cuda(args, cfg, rank, world, local_rank):
     return out
 
 
+# ----------------------------------------------------------------------------- decode (CUDA arm)
+def decode_stream_bytes(cfg, n_cols, loop, per_col_present=None):
+    """Bytes of K and V codes + fp16 scales of n_cols (column, head) entries:
+    the base and, for every loop 2..loop, the residual where present
+    (per_col_present[l] = fraction of the columns present at loop l)."""
+    dh = cfg.head_dim
+    per = dh + 2 * (dh // 32)
+    for l in range(2, loop + 1):
+        frac = 1.0 if per_col_present is None else per_col_present[l]
+        per += frac * (dh * cfg.bits[l - 1] // 8 + 2 * (dh // 32))
+    return 2 * n_cols * per
+
+
+def run_decode_cuda(args, cfg, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+    from cross_loop_sparse_b200 import flashloop as F
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    stream = torch.cuda.current_stream()
+    B, S, d, R, H, dh = cfg.batch, cfg.seq, cfg.d_model, cfg.n_loops, cfg.n_heads, cfg.head_dim
+    W = make_weights(cfg)
+    to_dev = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
+    wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
+    p = F.Params.from_config(cfg)
+    ctx = F.DecodeContext(p, device=dev)
+    ds = F.DecodeState(p, device=dev)
+    seqs = [rank * B + i for i in range(B)]
+    # the contexts' caches (what their prefill leaves), built loop by loop on the GPU; untimed
+    ctx_x = [make_hidden_states(cfg, b)[0] for b in seqs]
+    xs = [to_dev(np.concatenate([c[r] for c in ctx_x], axis=0)) for r in range(R)]
+    del ctx_x
+    ctx.prepare(xs, wqkv)
+    del xs
+    toks = [make_decode_tokens(cfg, b) for b in seqs]
+    host_tok = [np.stack([t[r] for t in toks]) for r in range(R)]
+    xt = [to_dev(x) for x in host_tok]
+    torch.cuda.synchronize()
+
+    events = []
+
+    def step(record):
+        for r in range(1, R + 1):
+            F.flashloop_decode_qkv(p, r, xt[r - 1], wqkv, ds)
+            if record:
+                e0 = torch.cuda.Event(enable_timing=True)
+                e1 = torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+            F.flashloop_decode_attn(p, r, ctx, ds)
+            if record:
+                e1.record(stream)
+                events.append((r, e0, e1))
+            if r == 1:
+                F.flashloop_decode_select(p, ds)
+            F.flashloop_decode_out(p, wo, ds)
+        # per loop: GEMV + token quantisation, attention + merge, out GEMV; top-k at loop 1
+        return 5 * R + 1
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        launches = step(False)
+    torch.cuda.synchronize()
+    barrier()
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        gpu_id = str(local_rank)
+    clocks = ClockSampler(gpu_id)
+    clocks.start()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(args.steps):
+        launches = step(True)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier()
+    ms = max_over_ranks(t0.elapsed_time(t1), dev)
+    for name, err in (("context", ctx.error_code()), ("decode", ds.error_code())):
+        if err != 0:
+            raise RuntimeError(f"{name} device error word {err}")
+
+    per_loop = {}
+    for r, e0, e1 in events:
+        per_loop.setdefault(r, []).append(e0.elapsed_time(e1))
+    peaks, peak_kind = load_peaks()
+    # loop 1 (the dominant pass): the INT8 base codes + scales of K and V of
+    # every column 0..S of every (sequence, head), and the probabilities written
+    P1 = S + 1
+    bytes1 = decode_stream_bytes(cfg, B * H * P1, 1) + B * H * P1 * 4
+    ms1 = statistics.mean(per_loop[1])
+    achieved = bytes1 / (ms1 * 1e-3) / 1e9
+    n_ctx = ctx["n_active"].cpu().numpy()
+    cols = ds["cols"].cpu().numpy()
+    # fraction of the selected (sequence, head, column) entries with a loop-l residual
+    is_tok = cols == S
+    rows = np.arange(B)[:, None, None] * S + np.minimum(cols, S - 1)
+    present = {l: float(((ctx[f"slot{l}"].cpu().numpy()[rows] >= 0) | is_tok).mean()) for l in range(2, R + 1)}
+    sparse = {}
+    for r in range(2, R + 1):
+        b_r = decode_stream_bytes(cfg, cols.size, r, present)
+        m_r = statistics.mean(per_loop[r])
+        sparse[f"loop{r}"] = {"ms": round(m_r, 4), "gbs": round(b_r / (m_r * 1e-3) / 1e9, 1),
+                              "bytes": int(b_r)}
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": DECODE_DENSE_TRAFFIC.get(f"decode_dense_kernel<{dh},{H * dh // 256}>"),
+                "kernel": f"decode_dense_kernel<{dh},{H * dh // 256}> + decode_dense_merge_kernel "
+                          "(loop-1 pass, timed together)",
+                "algorithmic": f"K and V INT8 base codes + fp16 scales of {B}x{H}x{P1} (sequence, head, column) "
+                               f"entries + float32 probabilities = {bytes1:.4g} B",
+                "peak_source": f"{peak_kind} HBM copy bandwidth",
+                "per_loop": {"loop1": {"ms": round(ms1, 4), "gbs": round(achieved, 1)}, **sparse},
+                "attn_share_of_step": round(sum(sum(v) for v in per_loop.values()) / ms, 4)}
+
+    # End to end through the public API with host buffers: H2D of the B tokens'
+    # hidden states of loops 1..R from pinned memory, decode_step per loop,
+    # D2H of Y.
+    host_x = [torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).pin_memory() for x in host_tok]
+    host_y = torch.empty((B, d), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, min(args.steps, 20))
+
+    def e2e_step():
+        for r in range(R):
+            xt[r].copy_(host_x[r], non_blocking=True)
+        for r in range(1, R + 1):
+            F.flashloop_decode_step(p, r, xt[r - 1], wqkv, wo, ctx, ds)
+        host_y.copy_(ds["Y"], non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    barrier()
+
+    tokens = B * world
+    ms_step = ms / args.steps
+    return {
+        "metric": DECODE_METRIC, "value": round(tokens / (ms_step * 1e-3), 1), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded workload generator; random-init weights of the stated shape)",
+        "config": {"workload": f"{cfg.name}: {B} sequences x 1 token at position {S} against {S}-token "
+                               f"contexts, d_model {d}, {H} heads x {dh}, R {R}, top-k {cfg.k}/head, bits "
+                               f"{'/'.join(str(b) for b in cfg.bits)}",
+                   "l2": "inputs larger than L2: the loop-1 pass reads 1.14 GB of cache per step",
+                   "parallelism": f"{B} sequences per GPU, {world} GPU(s), no exchange",
+                   "context_active_rows": {f"loop{r}": int(n_ctx[r - 1]) for r in range(2, R + 1)}},
+        "roofline": roofline,
+        "e2e": {"value": round(tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
+                "h2d_bytes_per_step": R * B * d * 2, "d2h_bytes_per_step": B * d * 2, "steps": e2e_steps},
+        "gpu_launches": launches * args.steps,
+        "clocks": clk,
+    }
+
+
+class DecodeOracleSample:
+    """The CPU oracle's decode on a bounded sample: one sequence, one head,
+    its context part (what the prefill leaves) computed once untimed; each
+    step re-runs the token's loops 1..R.  A full step is that time x B x H."""
+
+    def __init__(self, cfg, heads=(0,)):
+        import oracle as O
+        self.O, self.cfg, self.heads = O, cfg, list(heads)
+        self.W = make_weights(cfg)
+        self.ctx = make_hidden_states(cfg, 0)[0]
+        self.tok = make_decode_tokens(cfg, 0)
+        self.base = O.OracleDecode(cfg, self.W, self.ctx, self.tok, heads=self.heads).prepare_context()
+
+    def step(self):
+        import copy
+        orc = copy.deepcopy(self.base)
+        t = time.perf_counter()
+        orc.run()
+        dt = time.perf_counter() - t
+        scale = self.cfg.batch * self.cfg.n_heads / len(self.heads)
+        sample = (f"oracle decode loops 1..{self.cfg.n_loops} of one token against a {self.cfg.seq}-token "
+                  f"context on {len(self.heads)} of {self.cfg.n_heads} heads ({dt:.2f} s, includes the "
+                  f"cache writes of the context rows), scaled x{scale:g} to {self.cfg.batch} sequences x "
+                  f"{self.cfg.n_heads} heads")
+        return dt * scale, sample
+
+
 # ----------------------------------------------------------------------------- oracle timing
 class OracleSample:
     """The CPU oracle on a bounded sample of the workload: loops 2..R for the
@@ -334,6 +538,24 @@ class OracleSample:
 
 def run_reference(args, cfg):
     """The reference arm: the CPU oracle as it stands, on a bounded sample per step."""
+    if cfg.decode:
+        smp = DecodeOracleSample(cfg)
+        times, sample = [], ""
+        for i in range(args.warmup + args.steps):
+            t_est, sample = smp.step()
+            if i >= args.warmup:
+                times.append(t_est)
+        ms = statistics.mean(times) * 1e3
+        val = cfg.batch / (ms * 1e-3)
+        return {
+            "impl": "reference", "metric": DECODE_METRIC, "value": round(val, 4), "unit": "tokens/s",
+            "n_gpus": 1, "steps": len(times), "warmup": args.warmup, "ms_per_step": round(ms, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.description, "parallelism": "CPU oracle, host cores"},
+            "cpu_baseline": {"value": round(val, 4), "unit": "tokens/s", "cores": OracleSample.cores(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        }
     smp = OracleSample(cfg)
     times, sample = [], ""
     for i in range(args.warmup + args.steps):
@@ -360,7 +582,7 @@ def main():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
-    ap.add_argument("--config", default="prefill_32k", choices=[k for k, c in CONFIGS.items() if not c.decode])
+    ap.add_argument("--config", default="prefill_32k", choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
@@ -381,11 +603,16 @@ def main():
         import torch.distributed as dist
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    out = run_cuda(args, cfg, rank, world, local_rank)
+    out = (run_decode_cuda if cfg.decode else run_cuda)(args, cfg, rank, world, local_rank)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        t_est, sample = OracleSample(cfg).step()
-        out["cpu_baseline"] = {"value": round(cfg.seq * (cfg.n_loops - 1) / t_est, 2), "unit": "tokens/s",
-                               "cores": OracleSample.cores(), "kind": "oracle", "sample": sample}
+        if cfg.decode:
+            t_est, sample = DecodeOracleSample(cfg).step()
+            value = round(cfg.batch / t_est, 4)
+        else:
+            t_est, sample = OracleSample(cfg).step()
+            value = round(cfg.seq * (cfg.n_loops - 1) / t_est, 2)
+        out["cpu_baseline"] = {"value": value, "unit": "tokens/s", "cores": OracleSample.cores(),
+                               "kind": "oracle", "sample": sample}
     if world > 1:
         import torch.distributed as dist
         dist.barrier()

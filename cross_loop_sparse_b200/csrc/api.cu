@@ -16,7 +16,8 @@ int launch_kv_quant(const flashloop_params*, int, const float*, const float*, co
 int launch_selcol_dequant(const flashloop_params*, int, const int32_t*, int, int, flashloop_state*,
                           __half*, __half*, __half*, __half*, cudaStream_t);
 int launch_topk(const flashloop_params*, const float*, const int32_t*, int, int, int32_t*, int32_t*,
-                cudaStream_t);
+                cudaStream_t, const float* row_m = nullptr, const float* row_z = nullptr,
+                float* probs_out = nullptr);
 int launch_qkv_gemm(const flashloop_params*, const uint16_t*, const int32_t*, const int32_t*, int,
                     const uint16_t*, const float*, uint16_t*, float*, float*, int32_t*, cudaStream_t);
 int launch_out_gemm(const flashloop_params*, const uint16_t*, const int32_t*, const int32_t*, int,
@@ -31,8 +32,10 @@ namespace fl {
 int launch_attn_tc(const flashloop_params*, const AttnArgs&, int, cudaStream_t);
 DecodeLayout decode_layout(const flashloop_params*);
 int launch_decode_attn(const flashloop_params*, int, const flashloop_state*, flashloop_decode_state*, cudaStream_t);
-int launch_decode_step(const flashloop_params*, int, const uint16_t*, const uint16_t*, const uint16_t*,
-                       const flashloop_state*, flashloop_decode_state*, cudaStream_t);
+int launch_decode_select(const flashloop_params*, flashloop_decode_state*, cudaStream_t);
+int launch_decode_qkv(const flashloop_params*, int, const uint16_t*, const uint16_t*, flashloop_decode_state*,
+                      cudaStream_t);
+int launch_decode_out(const flashloop_params*, const uint16_t*, flashloop_decode_state*, cudaStream_t);
 int launch_colmass(const flashloop_params*, const ColmassArgs&, cudaStream_t);
 
 // ---------------------------------------------------------------------------
@@ -220,7 +223,7 @@ int flashloop_topk_columns(const flashloop_params* p, const float* mass, const i
   if (!mass || !out) return FLASHLOOP_ERR_INVALID_ARG;
   const int n = candidates ? n_cand : p->seq;
   if (n < 1 || n > p->seq) return FLASHLOOP_ERR_INVALID_ARG;
-  if (n > 53248) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (n > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
   if (k < 1 || k > n) return FLASHLOOP_ERR_INVALID_ARG;
   return launch_topk(p, mass, candidates, n_cand, k, out, nullptr, as_stream(stream));
 }
@@ -363,6 +366,7 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   rc = launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, st->q[cur], s);
   if (rc != FLASHLOOP_OK) return rc;
   const int sel = flashloop_selection_loop(p, loop);
+  if (sel == loop && loop == 2 && p->seq > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
   if (sel == loop) {
     const int k = p->topk[loop - 1];
     if (loop == 2) {
@@ -426,10 +430,19 @@ static int check_decode_params(const flashloop_params* p) {
   return FLASHLOOP_OK;
 }
 
+static int check_decode_common(const flashloop_params* p, const flashloop_decode_state* ds) {
+  int rc = check_decode_params(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  rc = check_arch();
+  if (rc != FLASHLOOP_OK) return rc;
+  if (!ds || !ds->err_word || !ds->workspace || !ds->O) return FLASHLOOP_ERR_INVALID_ARG;
+  if (ds->workspace_bytes < decode_layout(p).total) return FLASHLOOP_ERR_INVALID_ARG;
+  return FLASHLOOP_OK;
+}
+
 static int check_decode_state(const flashloop_params* p, int loop, const flashloop_state* ctx,
                               const flashloop_decode_state* ds) {
-  if (!ctx || !ds || !ds->err_word || !ds->workspace || !ds->O) return FLASHLOOP_ERR_INVALID_ARG;
-  if (ds->workspace_bytes < decode_layout(p).total) return FLASHLOOP_ERR_INVALID_ARG;
+  if (!ctx || !ds) return FLASHLOOP_ERR_INVALID_ARG;
   if (!ctx->k.base_codes || !ctx->k.base_scales || !ctx->v.base_codes || !ctx->v.base_scales ||
       !ds->k.base_codes || !ds->k.base_scales || !ds->v.base_codes || !ds->v.base_scales)
     return FLASHLOOP_ERR_INVALID_ARG;
@@ -454,11 +467,23 @@ size_t flashloop_decode_workspace_bytes(const flashloop_params* p) {
   return decode_layout(p).total;
 }
 
+int flashloop_decode_qkv(const flashloop_params* p, int32_t loop, const uint16_t* x_tok, const uint16_t* w_qkv,
+                         flashloop_decode_state* ds, void* stream) {
+  int rc = check_decode_common(p, ds);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop < 1 || loop > p->n_loops || !x_tok || !w_qkv || !ds->rope_cs || !ds->q[slot_of_loop(loop)])
+    return FLASHLOOP_ERR_INVALID_ARG;
+  if (!ds->k.base_codes || !ds->k.base_scales || !ds->v.base_codes || !ds->v.base_scales)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  for (int l = 2; l <= loop; ++l)
+    if (!ds->k.res_codes[l - 1] || !ds->k.res_scales[l - 1] || !ds->v.res_codes[l - 1] || !ds->v.res_scales[l - 1])
+      return FLASHLOOP_ERR_INVALID_ARG;
+  return launch_decode_qkv(p, loop, x_tok, w_qkv, ds, as_stream(stream));
+}
+
 int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
                           flashloop_decode_state* ds, void* stream) {
-  int rc = check_decode_params(p);
-  if (rc != FLASHLOOP_OK) return rc;
-  rc = check_arch();
+  int rc = check_decode_common(p, ds);
   if (rc != FLASHLOOP_OK) return rc;
   if (loop < 1 || loop > p->n_loops) return FLASHLOOP_ERR_INVALID_ARG;
   rc = check_decode_state(p, loop, ctx, ds);
@@ -466,18 +491,42 @@ int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashlo
   return launch_decode_attn(p, loop, ctx, ds, as_stream(stream));
 }
 
+int flashloop_decode_select(const flashloop_params* p, flashloop_decode_state* ds, void* stream) {
+  int rc = check_decode_common(p, ds);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (p->n_loops < 2 || !ds->probs || !ds->cols) return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->seq + 1 > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
+  return launch_decode_select(p, ds, as_stream(stream));
+}
+
+int flashloop_decode_out(const flashloop_params* p, const uint16_t* w_o, flashloop_decode_state* ds,
+                         void* stream) {
+  int rc = check_decode_common(p, ds);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (!w_o || !ds->Y) return FLASHLOOP_ERR_INVALID_ARG;
+  return launch_decode_out(p, w_o, ds, as_stream(stream));
+}
+
 int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_t* x_tok,
                           const uint16_t* w_qkv, const uint16_t* w_o, const flashloop_state* ctx,
                           flashloop_decode_state* ds, void* stream) {
-  int rc = check_decode_params(p);
+  int rc = check_decode_common(p, ds);
   if (rc != FLASHLOOP_OK) return rc;
-  rc = check_arch();
-  if (rc != FLASHLOOP_OK) return rc;
-  if (loop < 1 || loop > p->n_loops || !x_tok || !w_qkv || !w_o) return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop < 1 || loop > p->n_loops || !x_tok || !w_qkv || !w_o || !ds->rope_cs || !ds->Y)
+    return FLASHLOOP_ERR_INVALID_ARG;
   rc = check_decode_state(p, loop, ctx, ds);
   if (rc != FLASHLOOP_OK) return rc;
-  if (!ds->rope_cs || !ds->Y) return FLASHLOOP_ERR_INVALID_ARG;
-  return launch_decode_step(p, loop, x_tok, w_qkv, w_o, ctx, ds, as_stream(stream));
+  if (loop == 1 && p->n_loops >= 2 && p->seq + 1 > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  rc = launch_decode_qkv(p, loop, x_tok, w_qkv, ds, s);
+  if (rc != FLASHLOOP_OK) return rc;
+  rc = launch_decode_attn(p, loop, ctx, ds, s);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (loop == 1 && p->n_loops >= 2) {
+    rc = launch_decode_select(p, ds, s);
+    if (rc != FLASHLOOP_OK) return rc;
+  }
+  return launch_decode_out(p, w_o, ds, s);
 }
 
 int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* stream) {

@@ -35,17 +35,22 @@ int launch_kv_quant_rows(int dh, int loop, int n_rows, int H, const int* bits, c
                          const float* v_new, const flashloop_kv& k, const flashloop_kv& v, int32_t* err,
                          cudaStream_t stream);
 int launch_topk(const flashloop_params* p, const float* mass, const int32_t* cand, int n_cand, int k,
-                int32_t* out, int32_t* err, cudaStream_t stream);
+                int32_t* out, int32_t* err, cudaStream_t stream, const float* row_m = nullptr,
+                const float* row_z = nullptr, float* probs_out = nullptr);
 
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kGemvRows = 8;      // x rows staged per pass of the GEMV
+constexpr int kGemvWarps = 8;     // warps of a GEMV block (they split K)
+constexpr int kGemvBatch = 4;     // 32-wide k steps of weight loads a lane has in flight
 constexpr int kStageCols = 8;     // columns per bulk-copy stage (all heads)
 constexpr int kStages = 4;        // ring depth
 constexpr int kChunkCols = 128;   // columns per online-softmax chunk
+constexpr int kScRow = kChunkCols + 4;  // row pitch of the per-head scores (bank spread)
 constexpr int kSparseThreads = 128;
 constexpr int kSparseCols = 256;  // selected columns per sparse block
+constexpr int kSparseStageCols = 16;  // columns per gather stage (8 threads each)
+constexpr int kSparseStages = 4;      // gather ring depth
 
 struct DecodeArgs {
   int S, H, B, P1, k, loop;
@@ -94,109 +99,118 @@ __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t b
 }
 
 // ---------------------------------------------------------------------------
-// y[b, n] = sum_k x[b, k] W[n, k] for the B token rows.  One warp owns the
-// output pair (n, n + dh/2) of one head block, so that the rotate-half RoPE
-// partners meet in one warp.  mode 0: N = 3d (q | k | v): RoPE on q and k at
-// the token position, q -> bf16 q_out [B, d], k, v -> f32 k_out, v_out
-// [B, d].  mode 1: N = d, y -> bf16 y_out [B, d].
+// y[b, n] = sum_k x[b, k] W[n, k] for the decode token rows, on the tensor
+// cores (mma.sync m16n8k16, bf16 operands, f32 accumulators): a weight tile
+// is the A operand (16 output rows x 16 k), eight token rows the B operand
+// (16 k x 8 tokens; blockIdx.y picks the group of eight).  A block owns two
+// 16-row tiles: rows n0.. and n0 + dh/2.. in the QKV projection (the
+// rotate-half RoPE partners) or two consecutive tiles of W_o; its
+// kGemvWarps warps split K and add their partial sums in shared memory.
+// Within a 32-wide k step a lane reads 16 consecutive bytes (8 k) of a
+// weight row: the step's two MMAs take k 8t..8t+3 and 8t+4..8t+7 of lane
+// quad t, a fixed permutation of k that the token operand follows, so the
+// sum over k is unchanged.
+// mode 0: N = 3d (q | k | v): RoPE on q and k at the token position,
+// q -> bf16 q_out [B, d], k, v -> f32 k_out, v_out [B, d].
+// mode 1: N = d, y -> bf16 y_out [B, d].
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kGemvWarps * 32)
 decode_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ w, int B, int K, int N,
                    int dh, int H, int mode, const float* __restrict__ rope_cs, uint16_t* q_out,
                    float* k_out, float* v_out, uint16_t* y_out) {
-  extern __shared__ __align__(16) float xs[];  // [kGemvRows][K]
+  __shared__ float red[kGemvWarps][2][16][8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int half = dh >> 1;
-  const int pair = blockIdx.x * (kThreads / 32) + warp;
-  const bool live = pair < (N >> 1);
-  const int hb = pair / half, i = pair % half;
-  const int n0 = hb * dh + i, n1 = n0 + half;
-  const int kc = K >> 3;  // 16-byte chunks per row
-  for (int b0 = 0; b0 < B; b0 += kGemvRows) {
-    const int nb = min(kGemvRows, B - b0);
-    __syncthreads();
-    for (int idx = threadIdx.x; idx < nb * kc; idx += kThreads) {
-      const int b = idx / kc, c = idx - b * kc;
-      const uint4 v = *reinterpret_cast<const uint4*>(x + (size_t)(b0 + b) * K + c * 8);
-      const float2 f0 = bf16x2_to_float2(v.x), f1 = bf16x2_to_float2(v.y);
-      const float2 f2 = bf16x2_to_float2(v.z), f3 = bf16x2_to_float2(v.w);
-      float4* d = reinterpret_cast<float4*>(xs + (size_t)b * K + c * 8);
-      d[0] = make_float4(f0.x, f0.y, f1.x, f1.y);
-      d[1] = make_float4(f2.x, f2.y, f3.x, f3.y);
-    }
-    __syncthreads();
-    if (!live) continue;
-    float a0[kGemvRows], a1[kGemvRows];
+  const int g = lane >> 2, t = lane & 3;
+  int n0, n1;
+  if (mode == 0) {
+    const int half = dh >> 1, tph = half / 16;  // tile pairs per head block
+    const int hb = blockIdx.x / tph, it = blockIdx.x - hb * tph;
+    n0 = hb * dh + it * 16;
+    n1 = n0 + half;
+  } else {
+    n0 = blockIdx.x * 32;
+    n1 = n0 + 16;
+  }
+  const int tok0 = blockIdx.y * 8;
+  const bool xrow = tok0 + g < B;
+  const uint16_t* xr = x + (size_t)(xrow ? tok0 + g : 0) * K;
+  const uint16_t* w0g = w + (size_t)(n0 + g) * K;
+  const uint16_t* w0h = w + (size_t)(n0 + g + 8) * K;
+  const uint16_t* w1g = w + (size_t)(n1 + g) * K;
+  const uint16_t* w1h = w + (size_t)(n1 + g + 8) * K;
+  const int kw = K / kGemvWarps;  // K slice of this warp (a multiple of 32)
+  const int k_begin = warp * kw, k_end = k_begin + kw;
+  float d0[4] = {0.f, 0.f, 0.f, 0.f}, d1[4] = {0.f, 0.f, 0.f, 0.f};
+  for (int kb = k_begin; kb < k_end; kb += 32 * kGemvBatch) {
+    uint4 a0g[kGemvBatch], a0h[kGemvBatch], a1g[kGemvBatch], a1h[kGemvBatch], xb[kGemvBatch];
 #pragma unroll
-    for (int b = 0; b < kGemvRows; ++b) a0[b] = a1[b] = 0.f;
-    const uint16_t* w0 = w + (size_t)n0 * K;
-    const uint16_t* w1 = w + (size_t)n1 * K;
-#pragma unroll 2
-    for (int c = lane; c < kc; c += 32) {
-      const uint4 u0 = ld_stream(w0 + c * 8), u1 = ld_stream(w1 + c * 8);
-      float wa[8], wb[8];
-      {
-        const uint32_t ua[4] = {u0.x, u0.y, u0.z, u0.w}, ub[4] = {u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 fa = bf16x2_to_float2(ua[e]), fb = bf16x2_to_float2(ub[e]);
-          wa[2 * e] = fa.x; wa[2 * e + 1] = fa.y;
-          wb[2 * e] = fb.x; wb[2 * e + 1] = fb.y;
-        }
-      }
-#pragma unroll
-      for (int b = 0; b < kGemvRows; ++b) {
-        if (b < nb) {
-          const float4* xp = reinterpret_cast<const float4*>(xs + (size_t)b * K + c * 8);
-          const float4 x0 = xp[0], x1 = xp[1];
-          const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            a0[b] = fmaf(wa[e], xv[e], a0[b]);
-            a1[b] = fmaf(wb[e], xv[e], a1[b]);
-          }
-        }
-      }
+    for (int i = 0; i < kGemvBatch; ++i) {
+      const int k = kb + 32 * i + 8 * t;
+      const bool in = kb + 32 * i < k_end;
+      const uint4 z = make_uint4(0u, 0u, 0u, 0u);
+      a0g[i] = in ? ld_stream(w0g + k) : z;
+      a0h[i] = in ? ld_stream(w0h + k) : z;
+      a1g[i] = in ? ld_stream(w1g + k) : z;
+      a1h[i] = in ? ld_stream(w1h + k) : z;
+      xb[i] = in && xrow ? *reinterpret_cast<const uint4*>(xr + k) : z;
     }
 #pragma unroll
-    for (int b = 0; b < kGemvRows; ++b) {
+    for (int i = 0; i < kGemvBatch; ++i) {
+      const uint32_t a00[4] = {a0g[i].x, a0h[i].x, a0g[i].y, a0h[i].y};
+      const uint32_t a01[4] = {a0g[i].z, a0h[i].z, a0g[i].w, a0h[i].w};
+      const uint32_t a10[4] = {a1g[i].x, a1h[i].x, a1g[i].y, a1h[i].y};
+      const uint32_t a11[4] = {a1g[i].z, a1h[i].z, a1g[i].w, a1h[i].w};
+      mma_bf16(d0, a00, xb[i].x, xb[i].y);
+      mma_bf16(d1, a10, xb[i].x, xb[i].y);
+      mma_bf16(d0, a01, xb[i].z, xb[i].w);
+      mma_bf16(d1, a11, xb[i].z, xb[i].w);
+    }
+  }
+  // D fragment: d[0] = (row g, token 2t), d[1] = (g, 2t+1), d[2] = (g+8, 2t), d[3] = (g+8, 2t+1)
+  red[warp][0][g][2 * t] = d0[0];
+  red[warp][0][g][2 * t + 1] = d0[1];
+  red[warp][0][g + 8][2 * t] = d0[2];
+  red[warp][0][g + 8][2 * t + 1] = d0[3];
+  red[warp][1][g][2 * t] = d1[0];
+  red[warp][1][g][2 * t + 1] = d1[1];
+  red[warp][1][g + 8][2 * t] = d1[2];
+  red[warp][1][g + 8][2 * t + 1] = d1[3];
+  __syncthreads();
+  const int tid = threadIdx.x;
+  if (tid >= 128) return;
+  const int r = tid >> 3, tb = tid & 7, row = tok0 + tb;  // (row of both tiles, token)
+  float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        a0[b] += __shfl_xor_sync(0xffffffffu, a0[b], o);
-        a1[b] += __shfl_xor_sync(0xffffffffu, a1[b], o);
-      }
-    }
-    float s0 = 0.f, s1 = 0.f;
-#pragma unroll
-    for (int b = 0; b < kGemvRows; ++b)
-      if (b == lane) { s0 = a0[b]; s1 = a1[b]; }
-    if (lane >= nb) continue;
-    const int row = b0 + lane;
-    if (mode == 1) {
-      y_out[(size_t)row * N + n0] = float_to_bf16_bits(s0);
-      y_out[(size_t)row * N + n1] = float_to_bf16_bits(s1);
-      continue;
-    }
-    const int d = H * dh;
-    const int section = hb / H, h = hb - section * H;
-    const size_t o0 = (size_t)row * d + h * dh + i, o1 = o0 + half;
-    if (section < 2) {
-      // rotate-half RoPE with explicit roundings (the same float32 result as
-      // the prefill projection's epilogue)
-      const float c = rope_cs[2 * i], sn = rope_cs[2 * i + 1];
-      const float y1 = __fsub_rn(__fmul_rn(s0, c), __fmul_rn(s1, sn));
-      const float y2 = __fadd_rn(__fmul_rn(s1, c), __fmul_rn(s0, sn));
-      s0 = y1;
-      s1 = y2;
-    }
-    if (section == 0) {
-      q_out[o0] = float_to_bf16_bits(s0);
-      q_out[o1] = float_to_bf16_bits(s1);
-    } else {
-      float* dst = section == 1 ? k_out : v_out;
-      dst[o0] = s0;
-      dst[o1] = s1;
-    }
+  for (int v = 0; v < kGemvWarps; ++v) {
+    s0 += red[v][0][r][tb];
+    s1 += red[v][1][r][tb];
+  }
+  if (row >= B) return;
+  if (mode == 1) {
+    y_out[(size_t)row * N + n0 + r] = float_to_bf16_bits(s0);
+    y_out[(size_t)row * N + n1 + r] = float_to_bf16_bits(s1);
+    return;
+  }
+  const int d = H * dh, half = dh >> 1;
+  const int hb = n0 / dh, i = n0 - hb * dh + r;  // element i of the first half of head block hb
+  const int section = hb / H, h = hb - section * H;
+  const size_t o0 = (size_t)row * d + h * dh + i, o1 = o0 + half;
+  if (section < 2) {
+    // rotate-half RoPE with explicit roundings (the same float32 result as
+    // the prefill projection's epilogue)
+    const float c = rope_cs[2 * i], sn = rope_cs[2 * i + 1];
+    const float y1 = __fsub_rn(__fmul_rn(s0, c), __fmul_rn(s1, sn));
+    const float y2 = __fadd_rn(__fmul_rn(s1, c), __fmul_rn(s0, sn));
+    s0 = y1;
+    s1 = y2;
+  }
+  if (section == 0) {
+    q_out[o0] = float_to_bf16_bits(s0);
+    q_out[o1] = float_to_bf16_bits(s1);
+  } else {
+    float* dst = section == 1 ? k_out : v_out;
+    dst[o0] = s0;
+    dst[o1] = s1;
   }
 }
 
@@ -207,22 +221,32 @@ decode_gemv_kernel(const uint16_t* __restrict__ x, const uint16_t* __restrict__ 
 // chunk streams its K stages (scores), then its V stages (weighted sums);
 // stages are [kStageCols, H*dh] code rows plus [kStageCols, H*dh/32] scales,
 // brought in by bulk copies into a kStages-deep ring.
-// Thread roles: scores — thread (column, head, group of 32) with the group's
-// 32 q values in registers; weighted sums — thread owns EPT consecutive
-// outputs of N (EPT = H*dh/256).
+// Warp roles: warp kDenseConsumers issues the copies (one lane), waiting on
+// a stage's `empty` barrier (one arrival per consumer warp) before reusing
+// it; the consumer warps wait on its `full` barrier (one lane polls).
+// Scores: thread (column, head, group of 32) with the group's 32 q values in
+// registers.  Weighted sums: thread owns EPT consecutive outputs of N
+// (EPT = H*dh/256).  The consumers meet at a named barrier twice per chunk
+// (around the softmax step between its K and V stages).
 // ---------------------------------------------------------------------------
+constexpr int kDenseConsumers = 8;
+constexpr int kDenseThreads = 32 * (kDenseConsumers + 1);
+constexpr int kConsumerBar = 1;  // named barrier of the consumer warps
+
 template <int DH, int EPT>
-__global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a) {
+__global__ void __launch_bounds__(kDenseThreads, 2) decode_dense_kernel(DecodeArgs a) {
   constexpr int G = DH / 32;
+  constexpr int kConsumerThreads = 32 * kDenseConsumers;
   const int H = a.H, HG = H * G;
   const int RB = H * DH;      // code bytes per column
   const int SB = HG * 2;      // scale bytes per column
   const int stage_bytes = kStageCols * (RB + SB);
   extern __shared__ __align__(128) uint8_t smem[];
   uint64_t* full = reinterpret_cast<uint64_t*>(smem);  // [kStages]
+  uint64_t* empty = full + kStages;                    // [kStages]
   uint8_t* ring = smem + 128;
-  float* sc = reinterpret_cast<float*>(ring + (size_t)kStages * stage_bytes);  // [H][kChunkCols]
-  float* run_m = sc + H * kChunkCols;   // [H]
+  float* sc = reinterpret_cast<float*>(ring + (size_t)kStages * stage_bytes);  // [H][kScRow]
+  float* run_m = sc + H * kScRow;       // [H]
   float* run_z = run_m + H;             // [H]
   float* alpha = run_z + H;             // [H]
   __shared__ volatile int s_abort;
@@ -233,8 +257,6 @@ __global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a)
   const int c_end = min(a.P1, c_begin + a.range);
   const int ncols = max(0, c_end - c_begin);
   const int nchunks = (ncols + kChunkCols - 1) / kChunkCols;
-  // stage s: chunk s / (2*spc), K if (s % (2*spc)) < spc, else V
-  const int spc = kChunkCols / kStageCols;
   int total = 0;
   for (int ch = 0; ch < nchunks; ++ch) {
     const int n = min(kChunkCols, ncols - ch * kChunkCols);
@@ -243,63 +265,78 @@ __global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a)
 
   if (tid == 0) {
     s_abort = 0;
-    for (int s = 0; s < kStages; ++s) mbar_init(&full[s], 1);
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kDenseConsumers);
+    }
     fence_mbar_init();
   }
-  for (int h = tid; h < H; h += kThreads) {
+  for (int h = tid; h < H; h += kDenseThreads) {
     run_m[h] = -INFINITY;
     run_z[h] = 0.f;
   }
   __syncthreads();
 
-  // map stage sequence number -> (chunk, is_v, stage-in-chunk)
-  auto stage_of = [&](int s, int& ch, int& isv, int& st) {
-    int rem = s;
-    for (ch = 0; ch < nchunks; ++ch) {
+  if (warp == kDenseConsumers) {
+    // ---------------- producer: one lane issues every stage's copies
+    if (lane != 0) return;
+    int s = 0;
+    for (int ch = 0; ch < nchunks && !s_abort; ++ch) {
+      const int chunk0 = c_begin + ch * kChunkCols;
       const int n = min(kChunkCols, ncols - ch * kChunkCols);
       const int ns = (n + kStageCols - 1) / kStageCols;
-      if (rem < 2 * ns) break;
-      rem -= 2 * ns;
+      for (int isv = 0; isv < 2 && !s_abort; ++isv) {
+        for (int st = 0; st < ns; ++st, ++s) {
+          const int buf = s % kStages;
+          if (s >= kStages && !mbar_wait_sleep(&empty[buf], ((s / kStages) - 1) & 1)) {
+            set_error(a.err, kDevErrTimeout);
+            s_abort = 1;
+            break;
+          }
+          const int col0 = chunk0 + st * kStageCols;
+          const int nc = min(kStageCols, chunk0 + n - col0);
+          const int n_ctx = max(0, min(nc, a.S - col0));
+          const bool has_tok = col0 + nc > a.S;
+          uint8_t* dst = ring + (size_t)buf * stage_bytes;
+          const KVStreams& cs = isv ? a.cv : a.ck;
+          const KVStreams& ts = isv ? a.tv : a.tk;
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&full[buf], (uint32_t)(n_ctx + (has_tok ? 1 : 0)) * (RB + SB));
+          if (n_ctx > 0) {
+            const size_t row = (size_t)b * a.S + col0;
+            bulk_load(dst, cs.base_codes + row * RB, (uint32_t)(n_ctx * RB), &full[buf]);
+            bulk_load(dst + kStageCols * RB, reinterpret_cast<const uint8_t*>(cs.base_scales) + row * SB,
+                      (uint32_t)(n_ctx * SB), &full[buf]);
+          }
+          if (has_tok) {
+            const int jt = a.S - col0;
+            bulk_load(dst + (size_t)jt * RB, ts.base_codes + (size_t)b * RB, (uint32_t)RB, &full[buf]);
+            bulk_load(dst + kStageCols * RB + (size_t)jt * SB,
+                      reinterpret_cast<const uint8_t*>(ts.base_scales) + (size_t)b * SB, (uint32_t)SB, &full[buf]);
+          }
+        }
+      }
     }
-    const int n = min(kChunkCols, ncols - ch * kChunkCols);
-    const int ns = (n + kStageCols - 1) / kStageCols;
-    isv = rem >= ns;
-    st = isv ? rem - ns : rem;
-  };
-  auto issue = [&](int s) {
-    int ch, isv, st;
-    stage_of(s, ch, isv, st);
-    const int col0 = c_begin + ch * kChunkCols + st * kStageCols;
-    const int n = min(kStageCols, min(c_begin + (ch + 1) * kChunkCols, c_end) - col0);
-    const int n_ctx = max(0, min(n, a.S - col0));
-    const bool has_tok = col0 + n > a.S;
-    uint8_t* buf = ring + (size_t)(s % kStages) * stage_bytes;
-    uint64_t* bar = &full[s % kStages];
-    const KVStreams& cs = isv ? a.cv : a.ck;
-    const KVStreams& ts = isv ? a.tv : a.tk;
-    const uint32_t bytes = (uint32_t)(n_ctx + (has_tok ? 1 : 0)) * (RB + SB);
-    fence_proxy_async_smem();
-    mbar_arrive_expect_tx(bar, bytes);
-    if (n_ctx > 0) {
-      const size_t row = (size_t)b * a.S + col0;
-      bulk_load(buf, cs.base_codes + row * RB, (uint32_t)(n_ctx * RB), bar);
-      bulk_load(buf + kStageCols * RB, reinterpret_cast<const uint8_t*>(cs.base_scales) + row * SB,
-                (uint32_t)(n_ctx * SB), bar);
-    }
-    if (has_tok) {
-      const int jt = a.S - col0;
-      bulk_load(buf + (size_t)jt * RB, ts.base_codes + (size_t)b * RB, (uint32_t)RB, bar);
-      bulk_load(buf + kStageCols * RB + (size_t)jt * SB,
-                reinterpret_cast<const uint8_t*>(ts.base_scales) + (size_t)b * SB, (uint32_t)SB, bar);
-    }
-  };
+    // copies still in flight land before the block can exit: the consumers
+    // wait for every stage, or, after an abort, this lane waits here
+    if (s_abort)
+      for (int t = max(0, s - kStages); t < s; ++t) mbar_wait_sleep(&full[t % kStages], (t / kStages) & 1);
+    return;
+  }
 
+  // ---------------- consumers
   // score role: (column-in-pass, head, group)
   const int hg = tid % HG, jsub = tid / HG;
-  const int cpp = kThreads / HG;  // columns per pass
+  const int cpp = kConsumerThreads / HG;  // columns per pass
   const int sh = hg / G;
-  float q[32];
+  // q of this thread's (head, group) as three int8 digits per element, so
+  // that q . codes is three integer dot products (dp4a):
+  //   q_k = 2^(E-21) (d2 2^16 + d1 2^8 + d0),  E = exponent of max |q_k|,
+  // exact for every element within 2^14 of the group's largest.
+  int qd[3][8];
+  float qsc;  // 2^(E-21) log2(e)/sqrt(dh)
   {
+    float q[32];
     const uint16_t* qp = a.q_new + (size_t)b * RB + hg * 32;
 #pragma unroll
     for (int v = 0; v < 4; ++v) {
@@ -312,18 +349,36 @@ __global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a)
         q[v * 8 + 2 * e + 1] = f.y;
       }
     }
+    float mx = 0.f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(q[e]));
+    const int E = mx > 0.f ? ilogbf(mx) : 0;
+    const float up = ldexpf(1.f, 21 - E);
+#pragma unroll
+    for (int v = 0; v < 8; ++v) qd[0][v] = qd[1][v] = qd[2][v] = 0;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const int Q = __float2int_rn(q[e] * up);  // |Q| < 2^22
+      const int c0 = ((Q + 128) & 255) - 128;
+      const int Q1 = (Q - c0) >> 8;
+      const int c1 = ((Q1 + 128) & 255) - 128;
+      const int c2 = (Q1 - c1) >> 8;
+      const int sh8 = (e & 3) * 8;
+      qd[0][e >> 2] |= (c0 & 255) << sh8;
+      qd[1][e >> 2] |= (c1 & 255) << sh8;
+      qd[2][e >> 2] |= (c2 & 255) << sh8;
+    }
+    qsc = ldexpf(a.kscale, E - 21);
   }
+  // the two 16-byte halves of a lane's 32 codes: lanes of alternate 128-byte
+  // windows read them in opposite order, so each load spreads over all banks
+  const bool swap = (lane >> 2) & 1;
   // weighted-sum role: outputs [o, o + EPT) of head oh
   const int o = tid * EPT, oh = o / DH;
   float acc[EPT];
 #pragma unroll
   for (int e = 0; e < EPT; ++e) acc[e] = 0.f;
 
-  int issued = 0;  // thread 0 only
-  if (tid == 0)
-    for (; issued < kStages - 1 && issued < total; ++issued) issue(issued);
-
-  bool ok = true;
   int s = 0;  // stage sequence number
   for (int ch = 0; ch < nchunks; ++ch) {
     const int chunk0 = c_begin + ch * kChunkCols;
@@ -331,85 +386,96 @@ __global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a)
     const int ns = (n + kStageCols - 1) / kStageCols;
     for (int phase = 0; phase < 2; ++phase) {
       for (int st = 0; st < ns; ++st, ++s) {
-        if (tid == 0 && !s_abort && s + kStages - 1 < total) issue(issued++);
-        if (ok && !s_abort) {
-          if (!mbar_wait(&full[s % kStages], (s / kStages) & 1)) {
+        const int buf = s % kStages;
+        int ok = 0;
+        if (lane == 0 && !s_abort) {
+          ok = mbar_wait_sleep(&full[buf], (s / kStages) & 1) ? 1 : 0;
+          if (!ok) {
             set_error(a.err, kDevErrTimeout);
             s_abort = 1;
-            ok = false;
           }
         }
-        const uint8_t* buf = ring + (size_t)(s % kStages) * stage_bytes;
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        const uint8_t* sb = ring + (size_t)buf * stage_bytes;
+        const uint16_t* scl = reinterpret_cast<const uint16_t*>(sb + kStageCols * RB);
         const int nv = min(kStageCols, n - st * kStageCols);
-        // one decision per warp: the shuffles below need every lane
-        if (__all_sync(0xffffffffu, ok && !s_abort)) {
+        if (ok) {
           if (phase == 0) {
-            for (int p0 = 0; p0 < kStageCols; p0 += cpp) {
+            for (int p0 = 0; p0 < kStageCols; p0 += cpp) {  // the same trip count in every lane
               const int jj = p0 + jsub;
               float part = 0.f;
               if (jj < nv) {
-                const uint8_t* row = buf + (size_t)jj * RB + hg * 32;
-                // odd lanes read the second 16 bytes first: the two loads of
-                // a warp then spread over all banks
-                const bool odd = lane & 1;
-                const uint4 ca = *reinterpret_cast<const uint4*>(row + (odd ? 16 : 0));
-                const uint4 cb = *reinterpret_cast<const uint4*>(row + (odd ? 0 : 16));
-                const uint4 c0 = odd ? cb : ca, c1 = odd ? ca : cb;
-                const uint32_t w0[4] = {c0.x ^ 0x80808080u, c0.y ^ 0x80808080u, c0.z ^ 0x80808080u,
-                                        c0.w ^ 0x80808080u};
-                const uint32_t w1[4] = {c1.x ^ 0x80808080u, c1.y ^ 0x80808080u, c1.z ^ 0x80808080u,
-                                        c1.w ^ 0x80808080u};
-                float d0 = 0.f, d1 = 0.f;
+                const uint8_t* row = sb + (size_t)jj * RB + hg * 32;
+                const uint4 ca = *reinterpret_cast<const uint4*>(row + (swap ? 16 : 0));
+                const uint4 cb = *reinterpret_cast<const uint4*>(row + (swap ? 0 : 16));
+                const uint4 c0 = swap ? cb : ca, c1 = swap ? ca : cb;
+                const int cw[8] = {(int)c0.x, (int)c0.y, (int)c0.z, (int)c0.w,
+                                   (int)c1.x, (int)c1.y, (int)c1.z, (int)c1.w};
+                int D0 = 0, D1 = 0, D2 = 0;
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                  d0 = fmaf(q[e], i8_at(w0[e >> 2], e & 3), d0);
-                  d1 = fmaf(q[16 + e], i8_at(w1[e >> 2], e & 3), d1);
+                for (int v = 0; v < 8; ++v) {
+                  D0 = __dp4a(cw[v], qd[0][v], D0);
+                  D1 = __dp4a(cw[v], qd[1][v], D1);
+                  D2 = __dp4a(cw[v], qd[2][v], D2);
                 }
-                const uint16_t* scl = reinterpret_cast<const uint16_t*>(buf + kStageCols * RB);
-                part = (d0 + d1) * half_bits_f(scl[jj * HG + hg]);
+                // |D0 + 256 D1| < 2^27: exact in int32; the 2^16 digit joins in float
+                const float dot = fmaf(static_cast<float>(D2), 65536.f, static_cast<float>(D0 + D1 * 256));
+                part = dot * half_bits_f(scl[jj * HG + hg]) * qsc;  // qsc differs per group
               }
 #pragma unroll
               for (int off = 1; off < G; off <<= 1) part += __shfl_xor_sync(0xffffffffu, part, off);
-              if (jj < nv && (hg % G) == 0) sc[sh * kChunkCols + st * kStageCols + jj] = part * a.kscale;
+              if (jj < nv && (hg % G) == 0) sc[sh * kScRow + st * kStageCols + jj] = part;
             }
           } else {
-            const uint16_t* scl = reinterpret_cast<const uint16_t*>(buf + kStageCols * RB);
-            for (int jj = 0; jj < nv; ++jj) {
-              const float f = sc[oh * kChunkCols + st * kStageCols + jj] * half_bits_f(scl[jj * HG + o / 32]);
-              const uint8_t* src = buf + (size_t)jj * RB + o;
-              if constexpr (EPT >= 4) {
+            const float* wrow = sc + oh * kScRow + st * kStageCols;
 #pragma unroll
-                for (int v = 0; v < EPT / 4; ++v) {
-                  const uint32_t u = reinterpret_cast<const uint32_t*>(src)[v] ^ 0x80808080u;
+            for (int jj = 0; jj < kStageCols; ++jj) {
+              if (jj < nv) {
+                const float f = wrow[jj] * half_bits_f(scl[jj * HG + o / 32]);
+                const uint8_t* src = sb + (size_t)jj * RB + o;
+                if constexpr (EPT == 8) {
+                  const uint2 w2 = *reinterpret_cast<const uint2*>(src);
+                  const uint32_t uu[2] = {w2.x ^ 0x80808080u, w2.y ^ 0x80808080u};
 #pragma unroll
-                  for (int e = 0; e < 4; ++e) acc[4 * v + e] = fmaf(f, i8_at(u, e), acc[4 * v + e]);
+                  for (int v = 0; v < 2; ++v)
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[4 * v + e] = fmaf(f, i8_at(uu[v], e), acc[4 * v + e]);
+                } else if constexpr (EPT >= 4) {
+#pragma unroll
+                  for (int v = 0; v < EPT / 4; ++v) {
+                    const uint32_t u = reinterpret_cast<const uint32_t*>(src)[v] ^ 0x80808080u;
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[4 * v + e] = fmaf(f, i8_at(u, e), acc[4 * v + e]);
+                  }
+                } else {
+#pragma unroll
+                  for (int e = 0; e < EPT; ++e)
+                    acc[e] = fmaf(f, static_cast<float>(reinterpret_cast<const int8_t*>(src)[e]), acc[e]);
                 }
-              } else {
-#pragma unroll
-                for (int e = 0; e < EPT; ++e)
-                  acc[e] = fmaf(f, static_cast<float>(reinterpret_cast<const int8_t*>(src)[e]), acc[e]);
               }
             }
           }
         }
-        __syncthreads();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[buf]);
       }
       if (phase == 0) {
         // online softmax over this chunk: new running max, rescale factor,
         // weights in place of the scores, raw scores kept for the selection
-        for (int h = warp; h < H; h += kThreads / 32) {
+        named_bar_sync(kConsumerBar, kConsumerThreads);
+        for (int h = warp; h < H; h += kDenseConsumers) {
           float mx = -INFINITY;
-          for (int jc = lane; jc < n; jc += 32) mx = fmaxf(mx, sc[h * kChunkCols + jc]);
+          for (int jc = lane; jc < n; jc += 32) mx = fmaxf(mx, sc[h * kScRow + jc]);
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
           const float m_new = fmaxf(run_m[h], mx);
           float z = 0.f;
           float* srow = a.scores + ((size_t)b * H + h) * a.P1 + chunk0;
           for (int jc = lane; jc < n; jc += 32) {
-            const float sv = sc[h * kChunkCols + jc];
+            const float sv = sc[h * kScRow + jc];
             srow[jc] = sv;
             const float e = ex2(sv - m_new);
-            sc[h * kChunkCols + jc] = e;
+            sc[h * kScRow + jc] = e;
             z += e;
           }
 #pragma unroll
@@ -421,33 +487,31 @@ __global__ void __launch_bounds__(kThreads, 2) decode_dense_kernel(DecodeArgs a)
             run_m[h] = m_new;
           }
         }
-        __syncthreads();
+        named_bar_sync(kConsumerBar, kConsumerThreads);
         const float al = alpha[oh];
 #pragma unroll
         for (int e = 0; e < EPT; ++e) acc[e] *= al;
+      } else {
+        // the next chunk's scores overwrite sc: every warp is done with its weights
+        named_bar_sync(kConsumerBar, kConsumerThreads);
       }
     }
   }
   // partials of this range
   const size_t pr = (size_t)b * a.nsplit + blockIdx.x;
-  for (int h = tid; h < H; h += kThreads) {
+  for (int h = tid; h < H; h += kConsumerThreads) {
     a.part_m[pr * H + h] = run_m[h];
     a.part_Z[pr * H + h] = run_z[h];
   }
 #pragma unroll
   for (int e = 0; e < EPT; ++e) a.part_N[pr * RB + o + e] = acc[e];
-  // a wait that gave up may leave a copy in flight: let it land first
-  if (tid == 0 && s_abort) {
-    for (int t = max(0, issued - kStages); t < issued; ++t) mbar_wait(&full[t % kStages], (t / kStages) & 1);
-  }
 }
 
-// Combine the ranges of each (sequence, head): state slot 0, O, and the
-// loop-1 probabilities of every column 0..S.
+// Combine the ranges of each (sequence, head): state slot 0 and O.  (The
+// loop-1 probabilities are made from the kept scores by the selection.)
 template <int DH>
 __global__ void __launch_bounds__(kThreads) decode_dense_merge_kernel(DecodeArgs a, float* m_out, float* z_out,
-                                                                      float* n_out, uint16_t* o_out,
-                                                                      float* probs) {
+                                                                      float* n_out, uint16_t* o_out) {
   const int bh = blockIdx.x, b = bh / a.H, h = bh - b * a.H;
   __shared__ float s_m, s_z;
   __shared__ float red[kThreads / 32];
@@ -484,91 +548,120 @@ __global__ void __launch_bounds__(kThreads) decode_dense_merge_kernel(DecodeArgs
     m_out[bh] = m;
     z_out[bh] = z;
   }
-  const float rz = 1.f / z;
-  const float* srow = a.scores + (size_t)bh * a.P1;
-  float* prow = probs + (size_t)bh * a.P1;
-  for (int j = tid; j < a.P1; j += kThreads) prow[j] = ex2(srow[j] - m) * rz;
 }
 
 // ---------------------------------------------------------------------------
 // Loop r >= 2, sparse: block (range, b*H + h) takes kSparseCols of the
-// selected columns.  8 lanes per column (each lane DH/8 elements), 16
-// columns per block step.  Pass 1 rebuilds K^(r-1) and K^(r) of each column
-// from the packed streams and keeps both scores; pass 2 rebuilds V^(r-1),
-// V^(r) and sums e_new V^(r) - e_old V^(r-1) against the block's own
-// reference max.
+// selected columns.  The block first resolves every column's rows (base row
+// and the residual row of each loop 2..r, or the token's rows) into shared
+// memory.  The columns' K and V bytes of every stream are then gathered by
+// cp.async into a ring of kSparseStages stages of kSparseStageCols columns
+// (8 threads per column), so that several stages are in flight while one is
+// used.  From a stage, 8 lanes per column (DH/8 elements each) rebuild
+// Khat^(r-1), Khat^(r), Vhat^(r-1), Vhat^(r) and fold
+// e_new Vhat^(r) - e_old Vhat^(r-1) into an online sum with a running
+// reference max per column group.
 // ---------------------------------------------------------------------------
 // acc[e] += code(e) * s for E8 consecutive BITS-bit two's-complement codes
-// starting at src (E8 * BITS / 8 bytes, aligned to their size).
-template <int E8, int BITS>
-__device__ __forceinline__ void add_res(const uint8_t* src, float s, float (&acc)[E8]) {
-  constexpr int NB = E8 * BITS / 8;
+// held in little-endian words w.
+// The sign bit of every field is flipped first (c + 2^(BITS-1), unsigned);
+// the field then lands in the mantissa of 2^23 and 2^23 + 2^(BITS-1) comes
+// off again: the exact code as a float, with no int-to-float conversion.
+template <int E8, int BITS, int NW>
+__device__ __forceinline__ void add_codes(const uint32_t (&w)[NW], float s, float (&acc)[E8]) {
   constexpr int PW = 32 / BITS;
-  uint32_t words[(NB + 3) / 4];
-  if constexpr (NB >= 4) {
+  constexpr uint32_t kSign = BITS == 8 ? 0x80808080u : BITS == 4 ? 0x88888888u : 0xAAAAAAAAu;
+  constexpr float kBias = 8388608.0f + (1 << (BITS - 1));
+  uint32_t u[NW];
 #pragma unroll
-    for (int v = 0; v < NB / 4; ++v) words[v] = reinterpret_cast<const uint32_t*>(src)[v];
-  } else if constexpr (NB == 2) {
-    words[0] = *reinterpret_cast<const uint16_t*>(src);
-  } else {
-    words[0] = *src;
-  }
+  for (int v = 0; v < NW; ++v) u[v] = w[v] ^ kSign;
 #pragma unroll
   for (int e = 0; e < E8; ++e) {
-    int c = static_cast<int>((words[e / PW] >> ((e % PW) * BITS)) & ((1u << BITS) - 1u));
-    if (c >= (1 << (BITS - 1))) c -= (1 << BITS);
-    acc[e] = acc[e] + static_cast<float>(c) * s;
+    const uint32_t f = ((u[e / PW] >> ((e % PW) * BITS)) & ((1u << BITS) - 1u)) | 0x4B000000u;
+    acc[e] = fmaf(__uint_as_float(f) - kBias, s, acc[e]);
   }
 }
 
-// Rows: a token column reads row b of every token stream; a context column
-// reads base row t and residual rows cslot[l-1][t].
+__device__ __forceinline__ void cp_async8(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(smem)), "l"(gmem));
+}
+
+// Shared-memory layout of one gather stage of kSparseStageCols columns:
+// K and V codes of every stream (base, then loop 2..LOOP residuals), then the
+// K and V scales of every stream.  Offsets depend on the loops' code widths.
+template <int DH, int LOOP>
+struct SparseStage {
+  static constexpr int G = DH / 32;
+  int rb[LOOP];               // code bytes of one column in stream l (0 = base)
+  int off_k[LOOP], off_v[LOOP];
+  int off_ks, off_vs, bytes;
+  __host__ __device__ SparseStage(const int* bits) {
+    int off = 0;
+#pragma unroll
+    for (int l = 0; l < LOOP; ++l) {
+      rb[l] = l == 0 ? DH : DH * bits[l] / 8;
+      off_k[l] = off;
+      off += kSparseStageCols * rb[l];
+      off_v[l] = off;
+      off += kSparseStageCols * rb[l];
+    }
+    off_ks = off;
+    off += LOOP * kSparseStageCols * G * 2;
+    off_vs = off;
+    off += LOOP * kSparseStageCols * G * 2;
+    bytes = off;
+  }
+};
+
+// E8 codes (this lane's slice, element e0 on) of one column of stream l in
+// a stage, added times s to acc (l = 0: the INT8 base, assigned).
 template <int E8>
-__device__ __forceinline__ void rebuild(const KVStreams& kv, const DecodeArgs& a, bool tok, int b, size_t t,
-                                        int h, int DH, int e0, float (&old_v)[E8], float (&new_v)[E8]) {
-  const int H = a.H, loop = a.loop;
-  const size_t base_row = tok ? (size_t)b : t;
-  {
-    const int8_t* src = kv.base_codes + (base_row * H + h) * DH + e0;
-    const float s = half_bits_f(kv.base_scales[(base_row * H + h) * (DH / 32) + e0 / 32]);
+__device__ __forceinline__ void stage_codes(const uint8_t* row, int bits, int e0, float s, float (&acc)[E8],
+                                            bool assign) {
+  const int nb = E8 * bits / 8;
+  const uint8_t* src = row + (e0 * bits) / 8;
+  uint32_t w[E8 / 4];
+#pragma unroll
+  for (int v = 0; v < E8 / 4; ++v) w[v] = 0u;
+  if constexpr (E8 >= 16) {
+    if (nb == 16) {
+      const uint4 t = *reinterpret_cast<const uint4*>(src);
+      w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+    }
+  }
+  if (nb == 16) {
+  } else if (nb == 8) {
+    const uint2 t = *reinterpret_cast<const uint2*>(src);
+    w[0] = t.x; w[1] = t.y;
+  } else if (nb == 4) {
+    w[0] = *reinterpret_cast<const uint32_t*>(src);
+  } else {
+    w[0] = *reinterpret_cast<const uint16_t*>(src);
+  }
+  if (assign) {  // the base: INT8
 #pragma unroll
     for (int v = 0; v < E8 / 4; ++v) {
-      const uint32_t u = reinterpret_cast<const uint32_t*>(src)[v] ^ 0x80808080u;
+      const uint32_t u = w[v] ^ 0x80808080u;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) old_v[4 * v + e] = i8_at(u, e) * s;
+      for (int e = 0; e < 4; ++e) acc[4 * v + e] = i8_at(u, e) * s;
     }
+    return;
   }
-  for (int l = 2; l <= loop; ++l) {
-    const int sl = tok ? b : a.cslot[l - 1][t];
-    if (l == loop) {
-#pragma unroll
-      for (int e = 0; e < E8; ++e) new_v[e] = old_v[e];
-    }
-    if (sl < 0) continue;
-    const int bb = a.bits[l - 1];
-    const uint8_t* row = kv.res_codes[l - 1] + ((size_t)sl * H + h) * (DH * bb / 8);
-    const float s = half_bits_f(kv.res_scales[l - 1][((size_t)sl * H + h) * (DH / 32) + e0 / 32]);
-    const uint8_t* src = row + (e0 * bb) / 8;
-    if (l < loop) {
-      if (bb == 2) add_res<E8, 2>(src, s, old_v);
-      else if (bb == 4) add_res<E8, 4>(src, s, old_v);
-      else add_res<E8, 8>(src, s, old_v);
-    } else {
-      if (bb == 2) add_res<E8, 2>(src, s, new_v);
-      else if (bb == 4) add_res<E8, 4>(src, s, new_v);
-      else add_res<E8, 8>(src, s, new_v);
-    }
-  }
-  if (loop == 1) {
-#pragma unroll
-    for (int e = 0; e < E8; ++e) new_v[e] = old_v[e];
-  }
+  if (bits == 2) add_codes<E8, 2>(w, s, acc);
+  else if (bits == 4) add_codes<E8, 4>(w, s, acc);
+  else add_codes<E8, 8>(w, s, acc);
 }
 
-template <int DH>
+template <int DH, int LOOP>
 __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArgs a) {
-  constexpr int E8 = DH / 8;
-  __shared__ float s_old[kSparseCols], s_new[kSparseCols];
+  constexpr int E8 = DH / 8, G = DH / 32;
+  const SparseStage<DH, LOOP> L(a.bits);
+  extern __shared__ __align__(16) uint8_t sm[];
+  int* srow = reinterpret_cast<int*>(sm + (size_t)kSparseStages * L.bytes);  // [LOOP][kSparseCols]
+  uint8_t* stok = reinterpret_cast<uint8_t*>(srow + LOOP * kSparseCols);   // [kSparseCols]
   __shared__ float red[3][kSparseThreads / 32];
   __shared__ float nred[kSparseThreads / 32][DH];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -578,6 +671,69 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
   const int n = max(0, min(kSparseCols, a.k - c_begin));
   const int e0 = u * E8;
   const int d = a.H * DH;
+
+  // rows of every column: base row and the residual row of loops 2..LOOP
+  const int32_t* cols = a.cols + (size_t)bh * a.k + c_begin;
+  for (int i = tid; i < n; i += kSparseThreads) {
+    int j = cols[i];
+    if (j < 0 || j > a.S) {
+      set_error(a.err, FLASHLOOP_DEVERR_INDEX);
+      j = a.S;
+    }
+    const bool tok = j == a.S;
+    const size_t t = (size_t)b * a.S + j;
+    stok[i] = tok;
+    srow[i] = tok ? b : (int)t;
+#pragma unroll
+    for (int l = 2; l <= LOOP; ++l) srow[(l - 1) * kSparseCols + i] = tok ? b : a.cslot[l - 1][t];
+  }
+  __syncthreads();
+
+  // gather of stage st: 8 threads per column
+  const int nst = (n + kSparseStageCols - 1) / kSparseStageCols;
+  auto issue = [&](int st) {
+    const int c = st * kSparseStageCols + (tid >> 3);
+    const int cu = tid & 7;
+    if (c < n) {
+      uint8_t* buf = sm + (size_t)(st % kSparseStages) * L.bytes;
+      const int cl = tid >> 3;  // column within the stage
+      const bool tok = stok[c];
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const KVStreams& S = kv == 0 ? (tok ? a.tk : a.ck) : (tok ? a.tv : a.cv);
+        const int* off = kv == 0 ? L.off_k : L.off_v;
+#pragma unroll
+        for (int l = 0; l < LOOP; ++l) {
+          const int row = srow[l * kSparseCols + c];
+          const int nch = L.rb[l] / 16;
+          if (row >= 0 && cu < nch) {
+            const uint8_t* src = (l == 0 ? reinterpret_cast<const uint8_t*>(S.base_codes)
+                                         : S.res_codes[l]) +
+                                 ((size_t)row * a.H + h) * L.rb[l] + cu * 16;
+            cp_async16(buf + off[l] + cl * L.rb[l] + cu * 16, src, 16);
+          }
+        }
+      }
+      // scales: 2*LOOP copies of G fp16 per column, two per thread
+#pragma unroll
+      for (int i = cu; i < 2 * LOOP; i += 8) {
+        const int kv = i / LOOP, l = i - kv * LOOP;
+        const KVStreams& S = kv == 0 ? (tok ? a.tk : a.ck) : (tok ? a.tv : a.cv);
+        const int row = srow[l * kSparseCols + c];
+        uint8_t* dst = buf + (kv == 0 ? L.off_ks : L.off_vs) + ((size_t)l * kSparseStageCols + cl) * G * 2;
+        if (row < 0) {  // no residual at this loop: scale 0 adds nothing
+          if constexpr (G == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
+          else *reinterpret_cast<uint32_t*>(dst) = 0u;
+        } else {
+          const uint16_t* src = (l == 0 ? S.base_scales : S.res_scales[l]) + ((size_t)row * a.H + h) * G;
+          if constexpr (G == 4) cp_async8(dst, src);
+          else cp_async4(dst, src);
+        }
+      }
+    }
+    cp_async_commit();
+  };
+
   float qo[E8], qn[E8];
   {
     const uint16_t* po = a.q_old + (size_t)b * d + h * DH + e0;
@@ -590,101 +746,116 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
       qn[2 * v] = fn.x; qn[2 * v + 1] = fn.y;
     }
   }
-  const int32_t* cols = a.cols + (size_t)bh * a.k + c_begin;
-  auto column = [&](int jl, bool& tok) -> size_t {
-    int j = cols[jl];
-    if (j < 0 || j > a.S) {
-      set_error(a.err, FLASHLOOP_DEVERR_INDEX);
-      j = a.S;
-    }
-    tok = j == a.S;
-    return (size_t)b * a.S + j;
-  };
-  const int steps = (n + 15) / 16;
-  float mu = -INFINITY, mxn = -INFINITY;
-  for (int it = 0; it < steps; ++it) {
-    const int jl = it * 16 + grp;
-    float dol = 0.f, dnw = 0.f;
-    if (jl < n) {
-      bool tok;
-      const size_t t = column(jl, tok);
-      float ko[E8], kn[E8];
-      rebuild<E8>(tok ? a.tk : a.ck, a, tok, b, t, h, DH, e0, ko, kn);
 #pragma unroll
-      for (int e = 0; e < E8; ++e) {
-        dol = fmaf(qo[e], ko[e], dol);
-        dnw = fmaf(qn[e], kn[e], dnw);
-      }
+  for (int st = 0; st < kSparseStages - 1; ++st) {
+    if (st < nst) issue(st);
+    else cp_async_commit();
+  }
+
+  float mu = -INFINITY, mxn = -INFINITY, zn = 0.f, zo = 0.f;
+  float acc[E8];
+#pragma unroll
+  for (int e = 0; e < E8; ++e) acc[e] = 0.f;
+  const int g = e0 / 32;
+  for (int st = 0; st < nst; ++st) {
+    cp_async_wait<kSparseStages - 2>();
+    __syncthreads();  // stage st landed for every thread; stage st-1 is free
+    if (st + kSparseStages - 1 < nst) issue(st + kSparseStages - 1);
+    else cp_async_commit();
+    const uint8_t* buf = sm + (size_t)(st % kSparseStages) * L.bytes;
+    const int jl = st * kSparseStageCols + grp;
+    const bool valid = jl < n;
+    // K: Khat^(LOOP-1) and Khat^(LOOP) of this lane's slice
+    float xo[E8], xn[E8];
+    {
+      const uint16_t* ks = reinterpret_cast<const uint16_t*>(buf + L.off_ks);
+      stage_codes<E8>(buf + L.off_k[0] + grp * L.rb[0], 8, e0, half_bits_f(ks[grp * G + g]), xo, true);
+#pragma unroll
+      for (int l = 1; l < LOOP - 1; ++l)
+        stage_codes<E8>(buf + L.off_k[l] + grp * L.rb[l], a.bits[l], e0,
+                        half_bits_f(ks[(l * kSparseStageCols + grp) * G + g]), xo, false);
+#pragma unroll
+      for (int e = 0; e < E8; ++e) xn[e] = xo[e];
+      stage_codes<E8>(buf + L.off_k[LOOP - 1] + grp * L.rb[LOOP - 1], a.bits[LOOP - 1], e0,
+                      half_bits_f(ks[((LOOP - 1) * kSparseStageCols + grp) * G + g]), xn, false);
+    }
+    float dol = 0.f, dnw = 0.f;
+#pragma unroll
+    for (int e = 0; e < E8; ++e) {
+      dol = fmaf(qo[e], xo[e], dol);
+      dnw = fmaf(qn[e], xn[e], dnw);
     }
 #pragma unroll
     for (int off = 1; off < 8; off <<= 1) {
       dol += __shfl_xor_sync(0xffffffffu, dol, off);
       dnw += __shfl_xor_sync(0xffffffffu, dnw, off);
     }
-    if (jl < n) {
-      dol *= a.kscale;
-      dnw *= a.kscale;
-      if (u == 0) {
-        s_old[jl] = dol;
-        s_new[jl] = dnw;
+    if (valid) {
+      const float so = dol * a.kscale, sn = dnw * a.kscale;
+      const float m_new = fmaxf(mu, fmaxf(so, sn));
+      if (m_new > mu) {  // same decision in the column's 8 lanes
+        const float rho = ex2(mu - m_new);  // 0 while mu is -inf
+#pragma unroll
+        for (int e = 0; e < E8; ++e) acc[e] *= rho;
+        zn *= rho;
+        zo *= rho;
+        mu = m_new;
       }
-      mu = fmaxf(mu, fmaxf(dol, dnw));
-      mxn = fmaxf(mxn, dnw);
-    }
-  }
+      const float en = ex2(sn - mu), eo = ex2(so - mu);
+      const uint16_t* vs = reinterpret_cast<const uint16_t*>(buf + L.off_vs);
+      stage_codes<E8>(buf + L.off_v[0] + grp * L.rb[0], 8, e0, half_bits_f(vs[grp * G + g]), xo, true);
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    mu = fmaxf(mu, __shfl_xor_sync(0xffffffffu, mu, off));
-    mxn = fmaxf(mxn, __shfl_xor_sync(0xffffffffu, mxn, off));
-  }
-  if (lane == 0) {
-    red[0][warp] = mu;
-    red[1][warp] = mxn;
-  }
-  __syncthreads();
-  mu = red[0][0];
-  mxn = red[1][0];
+      for (int l = 1; l < LOOP - 1; ++l)
+        stage_codes<E8>(buf + L.off_v[l] + grp * L.rb[l], a.bits[l], e0,
+                        half_bits_f(vs[(l * kSparseStageCols + grp) * G + g]), xo, false);
 #pragma unroll
-  for (int w = 1; w < kSparseThreads / 32; ++w) {
-    mu = fmaxf(mu, red[0][w]);
-    mxn = fmaxf(mxn, red[1][w]);
-  }
-  float acc[E8];
+      for (int e = 0; e < E8; ++e) xn[e] = xo[e];
+      stage_codes<E8>(buf + L.off_v[LOOP - 1] + grp * L.rb[LOOP - 1], a.bits[LOOP - 1], e0,
+                      half_bits_f(vs[((LOOP - 1) * kSparseStageCols + grp) * G + g]), xn, false);
 #pragma unroll
-  for (int e = 0; e < E8; ++e) acc[e] = 0.f;
-  float zn = 0.f, zo = 0.f;
-  for (int it = 0; it < steps; ++it) {
-    const int jl = it * 16 + grp;
-    if (jl < n) {
-      bool tok;
-      const size_t t = column(jl, tok);
-      float vo[E8], vn[E8];
-      rebuild<E8>(tok ? a.tv : a.cv, a, tok, b, t, h, DH, e0, vo, vn);
-      const float en = ex2(s_new[jl] - mu), eo = ex2(s_old[jl] - mu);
-#pragma unroll
-      for (int e = 0; e < E8; ++e) acc[e] = fmaf(en, vn[e], fmaf(-eo, vo[e], acc[e]));
+      for (int e = 0; e < E8; ++e) acc[e] = fmaf(en, xn[e], fmaf(-eo, xo[e], acc[e]));
       zn += en;
       zo += eo;
+      mxn = fmaxf(mxn, sn);
     }
   }
-  // reduce the 4 column groups of each warp, then the warps
+  cp_async_wait<0>();
+  // block reference: the largest group reference; every group rescales to it
+  float mb = mu, mx = mxn;
+#pragma unroll
+  for (int off = 8; off < 32; off <<= 1) {
+    mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, off));
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+  }
+  if (lane == 0) {
+    red[0][warp] = mb;
+    red[1][warp] = mx;
+  }
+  __syncthreads();
+  mb = red[0][0];
+  mx = red[1][0];
+#pragma unroll
+  for (int w = 1; w < kSparseThreads / 32; ++w) {
+    mb = fmaxf(mb, red[0][w]);
+    mx = fmaxf(mx, red[1][w]);
+  }
+  __syncthreads();
+  const float f = mu == -INFINITY ? 0.f : ex2(mu - mb);
 #pragma unroll
   for (int e = 0; e < E8; ++e) {
+    acc[e] *= f;
     acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 8);
     acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], 16);
   }
-  zn += __shfl_xor_sync(0xffffffffu, zn, 8);
-  zn += __shfl_xor_sync(0xffffffffu, zn, 16);
-  zo += __shfl_xor_sync(0xffffffffu, zo, 8);
-  zo += __shfl_xor_sync(0xffffffffu, zo, 16);
+  float zd = (zn - zo) * f;  // identical in the 8 lanes of a group: count lane u == 0 only
+  zd = u == 0 ? zd : 0.f;
+#pragma unroll
+  for (int off = 8; off < 32; off <<= 1) zd += __shfl_xor_sync(0xffffffffu, zd, off);
   if (lane < 8) {
 #pragma unroll
     for (int e = 0; e < E8; ++e) nred[warp][e0 + e] = acc[e];
   }
-  if (lane == 0) {
-    red[0][warp] = zn;
-    red[1][warp] = zo;
-  }
+  if (lane == 0) red[2][warp] = zd;
   __syncthreads();
   const size_t pi = (size_t)bh * gridDim.x + blockIdx.x;
   for (int e = tid; e < DH; e += kSparseThreads) {
@@ -694,16 +865,27 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
     a.part_N[pi * DH + e] = v;
   }
   if (tid == 0) {
-    float zsn = 0.f, zso = 0.f;
+    float z = 0.f;
 #pragma unroll
-    for (int w = 0; w < kSparseThreads / 32; ++w) {
-      zsn += red[0][w];
-      zso += red[1][w];
-    }
-    a.part_m[pi] = mxn;
-    a.part_mu[pi] = mu;
-    a.part_Z[pi] = zsn - zso;
+    for (int w = 0; w < kSparseThreads / 32; ++w) z += red[2][w];
+    a.part_m[pi] = mx;
+    a.part_mu[pi] = mb;
+    a.part_Z[pi] = z;
   }
+}
+
+template <int DH, int LOOP>
+static int launch_sparse_t(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
+  const SparseStage<DH, LOOP> L(a.bits);
+  const size_t smem = (size_t)kSparseStages * L.bytes + (size_t)LOOP * kSparseCols * 4 + kSparseCols;
+  static size_t attr = 0;
+  if (smem > attr) {
+    FL_TRY(cudaFuncSetAttribute(decode_sparse_kernel<DH, LOOP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem));
+    attr = smem;
+  }
+  decode_sparse_kernel<DH, LOOP><<<grid, kSparseThreads, smem, stream>>>(a);
+  return launch_status();
 }
 
 // Fold the ranges into the running state: m' = max(m, max s_new),
@@ -774,7 +956,7 @@ DecodeLayout decode_layout(const flashloop_params* p) {
 
 size_t decode_dense_smem(const flashloop_params* p) {
   const int H = p->n_heads, RB = H * p->head_dim, SB = H * (p->head_dim / 32) * 2;
-  return 128 + (size_t)kStages * kStageCols * (RB + SB) + ((size_t)H * kChunkCols + 3 * H) * sizeof(float);
+  return 128 + (size_t)kStages * kStageCols * (RB + SB) + ((size_t)H * kScRow + 3 * H) * sizeof(float);
 }
 
 static DecodeArgs make_args(const flashloop_params* p, int loop, const flashloop_state* ctx,
@@ -817,7 +999,7 @@ static int launch_dense_t(const DecodeArgs& a, size_t smem, cudaStream_t stream)
                                 (int)smem));
     attr = true;
   }
-  decode_dense_kernel<DH, EPT><<<dim3(a.nsplit, a.B), kThreads, smem, stream>>>(a);
+  decode_dense_kernel<DH, EPT><<<dim3(a.nsplit, a.B), kDenseThreads, smem, stream>>>(a);
   return launch_status();
 }
 
@@ -838,61 +1020,69 @@ int launch_decode_attn(const flashloop_params* p, int loop, const flashloop_stat
     if (rc != FLASHLOOP_OK) return rc;
     if (dh == 128)
       decode_dense_merge_kernel<128><<<B * H, kThreads, 0, stream>>>(a, ds->m[0], ds->Z[0], ds->N[0],
-                                                                     reinterpret_cast<uint16_t*>(ds->O), ds->probs);
+                                                                     reinterpret_cast<uint16_t*>(ds->O));
     else
       decode_dense_merge_kernel<64><<<B * H, kThreads, 0, stream>>>(a, ds->m[0], ds->Z[0], ds->N[0],
-                                                                    reinterpret_cast<uint16_t*>(ds->O), ds->probs);
-    rc = launch_status();
-    if (rc != FLASHLOOP_OK || p->n_loops < 2) return rc;
-    // fused selection: top-k of each (sequence, head) row of probabilities
-    flashloop_params ps = *p;
-    ps.n_heads = B * H;
-    ps.seq = p->seq + 1;
-    return launch_topk(&ps, ds->probs, nullptr, 0, a.k, ds->cols, ds->err_word, stream);
+                                                                    reinterpret_cast<uint16_t*>(ds->O));
+    return launch_status();
   }
   const int si = slot_of_loop(loop - 1), so = slot_of_loop(loop);
+  const dim3 grid(L.nblk, B * H);
+  int rc = FLASHLOOP_ERR_UNSUPPORTED;
+#define FL_SPARSE(D, LP) \
+  if (dh == D && loop == LP) rc = launch_sparse_t<D, LP>(a, grid, stream);
+  FL_SPARSE(128, 2) FL_SPARSE(128, 3) FL_SPARSE(128, 4) FL_SPARSE(128, 5) FL_SPARSE(128, 6)
+  FL_SPARSE(128, 7) FL_SPARSE(128, 8)
+  FL_SPARSE(64, 2) FL_SPARSE(64, 3) FL_SPARSE(64, 4) FL_SPARSE(64, 5) FL_SPARSE(64, 6)
+  FL_SPARSE(64, 7) FL_SPARSE(64, 8)
+#undef FL_SPARSE
+  if (rc != FLASHLOOP_OK) return rc;
   if (dh == 128) {
-    decode_sparse_kernel<128><<<dim3(L.nblk, B * H), kSparseThreads, 0, stream>>>(a);
     decode_sparse_merge_kernel<128><<<B * H, 128, 0, stream>>>(a, L.nblk, ds->m[si], ds->Z[si], ds->N[si], ds->m[so],
                                                                ds->Z[so], ds->N[so], reinterpret_cast<uint16_t*>(ds->O));
   } else {
-    decode_sparse_kernel<64><<<dim3(L.nblk, B * H), kSparseThreads, 0, stream>>>(a);
     decode_sparse_merge_kernel<64><<<B * H, 64, 0, stream>>>(a, L.nblk, ds->m[si], ds->Z[si], ds->N[si], ds->m[so],
                                                              ds->Z[so], ds->N[so], reinterpret_cast<uint16_t*>(ds->O));
   }
   return launch_status();
 }
 
+// Selection of the decode token: per (sequence, head) the topk[1] columns of
+// largest loop-1 probability, the same radix select as the prefill's, its
+// keys made from the kept scores (and written to probs) as they are loaded.
+int launch_decode_select(const flashloop_params* p, flashloop_decode_state* ds, cudaStream_t stream) {
+  flashloop_params ps = *p;
+  ps.n_heads = p->batch * p->n_heads;
+  ps.seq = p->seq + 1;
+  const DecodeLayout L = decode_layout(p);
+  return launch_topk(&ps, ws_ptr<float>(ds->workspace, L.scores), nullptr, 0, p->topk[1], ds->cols, ds->err_word,
+                     stream, ds->m[0], ds->Z[0], ds->probs);
+}
+
 int launch_decode_gemv(const flashloop_params* p, const uint16_t* x, const uint16_t* w, int mode,
                        const float* rope_cs, uint16_t* q_out, float* k_out, float* v_out, uint16_t* y_out,
                        cudaStream_t stream) {
   const int d = p->d_model, N = mode == 0 ? 3 * d : d;
-  const size_t smem = (size_t)kGemvRows * d * sizeof(float);
-  static size_t attr = 0;
-  if (smem > attr) {
-    FL_TRY(cudaFuncSetAttribute(decode_gemv_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-    attr = smem;
-  }
-  const int pairs = N / 2, warps = kThreads / 32;
-  decode_gemv_kernel<<<(pairs + warps - 1) / warps, kThreads, smem, stream>>>(
-      x, w, p->batch, d, N, p->head_dim, p->n_heads, mode, rope_cs, q_out, k_out, v_out, y_out);
+  const dim3 grid(N / 32, (p->batch + 7) / 8);
+  decode_gemv_kernel<<<grid, kGemvWarps * 32, 0, stream>>>(x, w, p->batch, d, N, p->head_dim, p->n_heads, mode,
+                                                           rope_cs, q_out, k_out, v_out, y_out);
   return launch_status();
 }
 
-int launch_decode_step(const flashloop_params* p, int loop, const uint16_t* x_tok, const uint16_t* w_qkv,
-                       const uint16_t* w_o, const flashloop_state* ctx, flashloop_decode_state* ds,
-                       cudaStream_t stream) {
+int launch_decode_qkv(const flashloop_params* p, int loop, const uint16_t* x_tok, const uint16_t* w_qkv,
+                      flashloop_decode_state* ds, cudaStream_t stream) {
   const DecodeLayout L = decode_layout(p);
   float* k_new = ws_ptr<float>(ds->workspace, L.k_new);
   float* v_new = ws_ptr<float>(ds->workspace, L.v_new);
   int rc = launch_decode_gemv(p, x_tok, w_qkv, 0, ds->rope_cs,
                               reinterpret_cast<uint16_t*>(ds->q[slot_of_loop(loop)]), k_new, v_new, nullptr, stream);
   if (rc != FLASHLOOP_OK) return rc;
-  rc = launch_kv_quant_rows(p->head_dim, loop, p->batch, p->n_heads, p->bits, k_new, v_new, ds->k, ds->v,
-                            ds->err_word, stream);
-  if (rc != FLASHLOOP_OK) return rc;
-  rc = launch_decode_attn(p, loop, ctx, ds, stream);
-  if (rc != FLASHLOOP_OK) return rc;
+  return launch_kv_quant_rows(p->head_dim, loop, p->batch, p->n_heads, p->bits, k_new, v_new, ds->k, ds->v,
+                              ds->err_word, stream);
+}
+
+int launch_decode_out(const flashloop_params* p, const uint16_t* w_o, flashloop_decode_state* ds,
+                      cudaStream_t stream) {
   return launch_decode_gemv(p, reinterpret_cast<const uint16_t*>(ds->O), w_o, 1, nullptr, nullptr, nullptr,
                             nullptr, reinterpret_cast<uint16_t*>(ds->Y), stream);
 }

@@ -44,6 +44,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait with a suspend-time hint: the thread may sleep in the
+// instruction up to `ns` nanoseconds for the phase to complete, instead of
+// spinning (fewer issued instructions while a stage is still in flight).
+__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(ns)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait that sleeps in try_wait (up to 20 us a try, at most ~2^16
+// tries, about 1.3 s in all) rather than spinning.
+__device__ __forceinline__ bool mbar_wait_sleep(uint64_t* bar, uint32_t parity) {
+  for (uint32_t i = 0; i < (1u << 16); ++i)
+    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+  return false;
+}
+
 // Wait until the phase of parity `parity` has completed.  Bounded: returns
 // false after kWaitLimit polls (the caller records the error and unwinds).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {

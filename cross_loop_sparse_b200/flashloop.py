@@ -104,6 +104,9 @@ _SIG = {
     "flashloop_decode_workspace_bytes": (c_size_t, [_P]),
     "flashloop_decode_attn": (_I, [_P, _I, _S, _D, _V]),
     "flashloop_decode_step": (_I, [_P, _I, _V, _V, _V, _S, _D, _V]),
+    "flashloop_decode_qkv": (_I, [_P, _I, _V, _V, _D, _V]),
+    "flashloop_decode_select": (_I, [_P, _D, _V]),
+    "flashloop_decode_out": (_I, [_P, _V, _D, _V]),
     "flashloop_selection_loop": (_I, [_P, _I]),
     "flashloop_check_error_word": (_I, [_V, POINTER(c_int32), _V]),
     "flashloop_status_string": (ctypes.c_char_p, [_I]),
@@ -251,6 +254,21 @@ def flashloop_decode_workspace_bytes(params: Params) -> int:
 def flashloop_decode_attn(params, loop, ctx, dstate, stream=None):
     return _check("flashloop_decode_attn", _lib.flashloop_decode_attn(
         ctypes.byref(params), loop, ctypes.byref(ctx.c), ctypes.byref(dstate.c), _stream(stream)))
+
+
+def flashloop_decode_qkv(params, loop, x_tok, w_qkv, dstate, stream=None):
+    return _check("flashloop_decode_qkv", _lib.flashloop_decode_qkv(
+        ctypes.byref(params), loop, _ptr(x_tok), _ptr(w_qkv), ctypes.byref(dstate.c), _stream(stream)))
+
+
+def flashloop_decode_select(params, dstate, stream=None):
+    return _check("flashloop_decode_select", _lib.flashloop_decode_select(
+        ctypes.byref(params), ctypes.byref(dstate.c), _stream(stream)))
+
+
+def flashloop_decode_out(params, w_o, dstate, stream=None):
+    return _check("flashloop_decode_out", _lib.flashloop_decode_out(
+        ctypes.byref(params), _ptr(w_o), ctypes.byref(dstate.c), _stream(stream)))
 
 
 def flashloop_decode_step(params, loop, x_tok, w_qkv, w_o, ctx, dstate, stream=None):

@@ -203,7 +203,7 @@ int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t*
 /* (a4) Column selection [FlashLoop §3.2, §4.2, App. D.2].  Per head h: the k
  * candidates of largest float32 mass[h, j] (ties to the lower index, -0 == +0),
  * written ascending to out[h*k ...].  candidates = NULL: all j in [0, S);
- * otherwise candidates[h*n_cand ...] ascending.  n_cand <= 53248. */
+ * otherwise candidates[h*n_cand ...] ascending.  n (S or n_cand) <= 49152. */
 int flashloop_topk_columns(const flashloop_params* p, const float* mass, const int32_t* candidates,
                            int32_t n_cand, int32_t k, int32_t* out, void* stream);
 
@@ -280,7 +280,7 @@ typedef struct flashloop_decode_state {
   float* m[3];               /* [B, H] */
   float* Z[3];               /* [B, H] */
   float* N[3];               /* [B, H, dh] */
-  float* probs;              /* [B, H, S+1] float32 loop-1 attention probabilities of the token */
+  float* probs;              /* [B, H, S+1] float32 loop-1 attention probabilities (flashloop_decode_select) */
   int32_t* cols;             /* [B, H, topk[1]] ascending selected columns in [0, S] (S = the token) */
   uint16_t* O;               /* bf16 [B, d_model] */
   uint16_t* Y;               /* bf16 [B, d_model] */
@@ -304,9 +304,8 @@ size_t flashloop_decode_workspace_bytes(const flashloop_params* p);
  * ctx->v and ctx->slot are read.  Columns 0..S-1 are the context, column S is
  * the token itself (its streams in ds).
  * loop 1: dense attention of q (slot 0) over Khat^(1), Vhat^(1) of columns
- *   0..S (base codes dequantised in the loads): state slot 0, O, probs; then
- *   cols = per (sequence, head) the topk[1] columns of largest float32
- *   probability (ties to the lower index), ascending.
+ *   0..S (base codes dequantised in the loads): state slot 0, O; the scores
+ *   stay in the workspace for flashloop_decode_select.
  * loop r >= 2: for the selected columns j,
  *   s_old = q^(r-1).Khat_j^(r-1)/sqrt(dh), s_new = q^(r).Khat_j^(r)/sqrt(dh),
  *   m' = max(m, max s_new), Z' = e^(m-m') Z - sum e^(s_old-m') + sum e^(s_new-m'),
@@ -317,12 +316,30 @@ size_t flashloop_decode_workspace_bytes(const flashloop_params* p);
 int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
                           flashloop_decode_state* ds, void* stream);
 
-/* (a8) One loop of the decode token, B sequences: q, k, v = x_tok W_qkv^T
+/* (a8) Projections of the decode token at loop `loop`: q, k, v = x_tok W_qkv^T
  * (x_tok bf16 [B, d_model], float32 accumulation, RoPE at position S on q and
- * k, q -> ds->q slot); k and v quantised into the token streams (INT8 base at
- * loop 1, the residual against the reconstructed previous loop after it,
- * the arithmetic of flashloop_kv_quant_residual); flashloop_decode_attn; then
- * Y = bf16(O W_o^T).  The token is active at every loop (no gate). */
+ * k; q -> ds->q slot of the loop); k and v quantised into the token streams
+ * (INT8 base at loop 1, the residual against the reconstructed previous loop
+ * after it, the arithmetic of flashloop_kv_quant_residual).  The token is
+ * active at every loop (no gate). */
+int flashloop_decode_qkv(const flashloop_params* p, int32_t loop, const uint16_t* x_tok, const uint16_t* w_qkv,
+                         flashloop_decode_state* ds, void* stream);
+
+/* (a8) Fused sparse decode selection [FlashLoop App. G]: cols = per
+ * (sequence, head) the topk[1] columns of largest float32 loop-1 probability
+ * (ties to the lower index, written ascending), and probs = those
+ * probabilities, 2^(s_j - m) / Z from the loop-1 scores kept in the
+ * workspace by flashloop_decode_attn (call it first).  Needs S + 1 <= 49152. */
+int flashloop_decode_select(const flashloop_params* p, flashloop_decode_state* ds, void* stream);
+
+/* (a8) Output projection of the decode tokens: Y = bf16(O W_o^T), float32
+ * accumulation. */
+int flashloop_decode_out(const flashloop_params* p, const uint16_t* w_o, flashloop_decode_state* ds,
+                         void* stream);
+
+/* (a8) One loop of the decode token, B sequences: flashloop_decode_qkv,
+ * flashloop_decode_attn, flashloop_decode_select (loop 1, when R >= 2),
+ * flashloop_decode_out. */
 int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_t* x_tok,
                           const uint16_t* w_qkv, const uint16_t* w_o, const flashloop_state* ctx,
                           flashloop_decode_state* ds, void* stream);

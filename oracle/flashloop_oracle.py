@@ -536,8 +536,16 @@ class OracleDecode:
         self.q = {}
         self.probs = None
 
+    def prepare_context(self):
+        """The context tokens' part of every loop (gate, k/v), which depends on
+        the context alone: a decode reads it from the cache its prefill left."""
+        self._ctx_kv = {r: self._context_kv(r) for r in range(1, self.cfg.n_loops + 1)}
+        return self
+
     def _context_kv(self, r):
-        """Context tokens' part of loop r: gate, k/v, cache write (no attention)."""
+        """Context tokens' part of loop r: gate, k/v (no attention)."""
+        if getattr(self, "_ctx_kv", None) and r in self._ctx_kv:
+            return self._ctx_kv[r]
         cfg = self.cfg
         S = cfg.seq
         if r == 1:

@@ -133,6 +133,8 @@ def test_decode_attention_staged(seq, batch):
             ds[f"Z{ip}"].copy_(torch.from_numpy(np.stack([o.state[r - 1][1] for o in orcs]).astype(np.float32)))
             ds[f"N{ip}"].copy_(torch.from_numpy(np.stack([o.state[r - 1][2] for o in orcs]).astype(np.float32)))
         F.flashloop_decode_attn(p, r, ctx, ds)
+        if r == 1:
+            F.flashloop_decode_select(p, ds)
         torch.cuda.synchronize()
         og = bf16_rows(torch_to_bf16_bits(ds["O"]))
         oo = bf16_rows(np.stack([o.O[r] for o in orcs]))
