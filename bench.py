@@ -34,8 +34,9 @@ DECODE_METRIC = "decode tokens/s (B sequences x 1 token x R loops) at S_ctx=32K,
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures summarised
 # under profiles/; None once the kernel changes until it is re-captured.
-ATTN_LOOP2_TRAFFIC = {"attn_tc_kernel<128>": 731.3e6}
-DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": None}
+ATTN_LOOP2_TRAFFIC = {"attn_tc_kernel<128>": 731.7e6}
+# captured on 2 sequences and scaled by 4 (traffic in proportion to the columns read)
+DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": 1169.5e6}
 
 
 def max_over_ranks(value, device=None):
@@ -382,9 +383,9 @@ def run_decode_cuda(args, cfg, rank, world, local_rank):
         per_loop.setdefault(r, []).append(e0.elapsed_time(e1))
     peaks, peak_kind = load_peaks()
     # loop 1 (the dominant pass): the INT8 base codes + scales of K and V of
-    # every column 0..S of every (sequence, head), and the probabilities written
+    # every column 0..S of every (sequence, head)
     P1 = S + 1
-    bytes1 = decode_stream_bytes(cfg, B * H * P1, 1) + B * H * P1 * 4
+    bytes1 = decode_stream_bytes(cfg, B * H * P1, 1)
     ms1 = statistics.mean(per_loop[1])
     achieved = bytes1 / (ms1 * 1e-3) / 1e9
     n_ctx = ctx["n_active"].cpu().numpy()
@@ -401,11 +402,12 @@ def run_decode_cuda(args, cfg, rank, world, local_rank):
                               "bytes": int(b_r)}
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": DECODE_DENSE_TRAFFIC.get(f"decode_dense_kernel<{dh},{H * dh // 256}>"),
+                "traffic": (DECODE_DENSE_TRAFFIC.get(f"decode_dense_kernel<{dh},{H * dh // 256}>")
+                            if (B, S, H, dh) == (8, 32768, 16, 128) else None),
                 "kernel": f"decode_dense_kernel<{dh},{H * dh // 256}> + decode_dense_merge_kernel "
                           "(loop-1 pass, timed together)",
                 "algorithmic": f"K and V INT8 base codes + fp16 scales of {B}x{H}x{P1} (sequence, head, column) "
-                               f"entries + float32 probabilities = {bytes1:.4g} B",
+                               f"entries = {bytes1:.4g} B",
                 "peak_source": f"{peak_kind} HBM copy bandwidth",
                 "per_loop": {"loop1": {"ms": round(ms1, 4), "gbs": round(achieved, 1)}, **sparse},
                 "attn_share_of_step": round(sum(sum(v) for v in per_loop.values()) / ms, 4)}
@@ -584,8 +586,14 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--config", default="prefill_32k", choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="decode workloads: sequences per GPU (a smaller case for profiler captures)")
     args = ap.parse_args()
     cfg = CONFIGS[args.config]
+    if args.batch is not None:
+        if not cfg.decode:
+            ap.error("--batch applies to decode workloads only")
+        cfg = cfg.with_(batch=args.batch)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
