@@ -240,31 +240,66 @@ def run_cuda(args, cfg, rank, world, local_rank):
                              for r, v in sorted(per_loop.items())},
                 "attn_share_of_step": round(attn_ms / ms, 4)}
 
-    # End to end through the public API with host buffers: H2D of the step's
-    # hidden states X_2..X_R from pinned memory, loop_step for loops 2..R,
-    # D2H of Y.
+    # End to end through the public API with host buffers, pipelined the way a
+    # serving loop runs it: every step copies its hidden states X_2..X_R from
+    # pinned host memory on a copy stream into one of two device buffer sets
+    # (the next step's copies overlap this step's compute), loop_step r waits
+    # for X_r only, and Y goes back to the host on a second copy stream once
+    # loop R is done.  Y alternates between two device buffers (the second
+    # starts as a copy of the first, so rows a step leaves untouched agree)
+    # so that the next step need not wait for the read-back.
     host_x = [torch.from_numpy(X[r - 1].view(np.int16)).view(torch.bfloat16).pin_memory()
               for r in range(2, R + 1)]
     host_y = torch.empty((S, d), dtype=torch.bfloat16).pin_memory()
-    e2e_steps = max(1, min(args.steps, 10))
+    e2e_steps = max(2, min(args.steps, 10))
+    xbuf = [[torch.empty_like(xs[r - 1]) for r in range(2, R + 1)] for _ in range(2)]
+    ybuf = [st["Y"], st["Y"].clone()]
+    h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    set_free = [None, None]  # the last compute that read each X buffer set
+    y_free = [None, None]    # the last read-back of each Y buffer
 
-    def e2e_step():
+    def e2e_step(sidx):
+        b = sidx % 2
+        ready = []
+        if set_free[b] is not None:
+            h2d.wait_event(set_free[b])
+        with torch.cuda.stream(h2d):
+            for i in range(R - 1):
+                xbuf[b][i].copy_(host_x[i], non_blocking=True)
+                ev = torch.cuda.Event()
+                ev.record(h2d)
+                ready.append(ev)
+        if y_free[b] is not None:
+            stream.wait_event(y_free[b])
+        st.c.Y = ybuf[b].data_ptr()
         for i, r in enumerate(range(2, R + 1)):
-            xs[r - 1].copy_(host_x[i], non_blocking=True)
-        for r in range(2, R + 1):
-            F.flashloop_loop_step(p, r, xs[r - 1], xs[r - 2], wqkv, wo, st)
-        host_y.copy_(st["Y"], non_blocking=True)
+            stream.wait_event(ready[i])
+            x_prev = xs[0] if r == 2 else xbuf[b][i - 1]
+            F.flashloop_loop_step(p, r, xbuf[b][i], x_prev, wqkv, wo, st, stream)
+        done = torch.cuda.Event()
+        done.record(stream)
+        set_free[b] = done
+        d2h.wait_event(done)
+        with torch.cuda.stream(d2h):
+            host_y.copy_(ybuf[b], non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(d2h)
+        y_free[b] = ev
 
-    e2e_step()
+    e2e_step(0)
     torch.cuda.synchronize()
     barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        e2e_step()
+    h2d.wait_event(e0)
+    for i in range(e2e_steps):
+        e2e_step(i + 1)
+    for ev in y_free:
+        stream.wait_event(ev)
     e1.record(stream)
     torch.cuda.synchronize()
+    st.c.Y = ybuf[0].data_ptr()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     barrier()
 

@@ -151,7 +151,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         const int h = item / row_tiles, rt = item % row_tiles;
         const int nt = at_tiles(g, h, rt, n_rows);
         for (int t = 0; t < nt && !*abort_flag; ++t) {
-          if (!mbar_wait(&kv_empty[stage], phase ^ 1)) {
+          if (!mbar_wait_sleep(&kv_empty[stage], phase ^ 1)) {
             set_error(g.err, kDevErrTimeout);
             *abort_flag = 1;
             break;
@@ -190,7 +190,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x, ++item_no) {
         const int h = item / row_tiles, rt = item % row_tiles;
         const int nt = at_tiles(g, h, rt, n_rows);
-        if (!mbar_wait(q_ready, item_no & 1)) {
+        if (!mbar_wait_sleep(q_ready, item_no & 1)) {
           set_error(g.err, kDevErrTimeout);
           *abort_flag = 1;
           break;
@@ -200,7 +200,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         for (int t = 0; t <= nt; ++t) {
           if (t < nt) {
             // S(t) into buffer u & 1
-            if (!mbar_wait(&kv_full[stage], phase)) {
+            if (!mbar_wait_sleep(&kv_full[stage], phase)) {
               set_error(g.err, kDevErrTimeout);
               *abort_flag = 1;
               ok = false;
@@ -222,7 +222,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           if (t > 0) {
             // P(t-1).V into N
             const uint32_t up = u - 1;
-            if (!mbar_wait(&p_full[up & 1], (up >> 1) & 1)) {
+            if (!mbar_wait_sleep(&p_full[up & 1], (up >> 1) & 1)) {
               set_error(g.err, kDevErrTimeout);
               *abort_flag = 1;
               ok = false;
@@ -274,7 +274,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
     auto wait_or_die = [&](uint64_t* bar, uint32_t parity) {
       if (!dead && __any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
       if (dead) return;
-      if (!__all_sync(0xffffffffu, mbar_wait(bar, parity))) {
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar, parity))) {
         set_error(g.err, kDevErrTimeout);
         *abort_flag = 1;
         dead = true;
@@ -377,19 +377,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           tmem_ld32(sbase + first, rn);
           if (has_old) tmem_ld32(sbase + 64 + first, ro);
           tmem_wait_ld();
-          if (nvalid >= first + 32) {
-#pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, __uint_as_float(rn[e]));
-          } else {
+          if (nvalid < first + 32) {
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               if (first + e >= nvalid) {
                 rn[e] = 0xff800000u;  // -inf
                 ro[e] = 0xff800000u;
               }
-              mx = fmaxf(mx, __uint_as_float(rn[e]));
             }
           }
+          // tree reduction: 5 dependent steps instead of a 32-long chain
+          float t16[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) t16[e] = fmaxf(__uint_as_float(rn[e]), __uint_as_float(rn[e + 16]));
+#pragma unroll
+          for (int w = 8; w > 0; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e) t16[e] = fmaxf(t16[e], t16[e + w]);
+          mx = t16[0];
         }
         float* xm = xchg + (b * 2) * 128;  // [half][128] of this parity
         xm[half * 128 + row] = mx;
@@ -422,28 +427,32 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           m_ref = new_ref;
         }
         uint32_t pk[16];
-        float zs = 0.f;
+        // four independent partial sums per matrix (short dependency chains)
+        float za[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
           const float p0 = ex2(__uint_as_float(rn[2 * e2]) - m_ref);
           const float p1 = ex2(__uint_as_float(rn[2 * e2 + 1]) - m_ref);
-          zs += p0 + p1;
+          za[e2 & 3] += p0 + p1;
           pk[e2] = pack_half2(p0, p1);
         }
         __syncwarp();
         tmem_st16(sbase + half * 16, pk);
         if (has_old) {
+          float zb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
             const float p0 = ex2(__uint_as_float(ro[2 * e2]) - m_ref);
             const float p1 = ex2(__uint_as_float(ro[2 * e2 + 1]) - m_ref);
-            zs -= p0 + p1;
+            zb[e2 & 3] += p0 + p1;
             pk[e2] = pack_half2(-p0, -p1);
           }
           __syncwarp();
           tmem_st16(sbase + 32 + half * 16, pk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) za[i] -= zb[i];
         }
-        z += zs;
+        z += (za[0] + za[1]) + (za[2] + za[3]);
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);

@@ -18,8 +18,8 @@ from gpu_helpers import bf16_rows, bf16_to_torch, row_rel_l2, torch_to_bf16_bits
 TOL = 1e-2
 
 
-def run_gpu(cfg, W, X, stream=None):
-    p = F.Params.from_config(cfg)
+def run_gpu(cfg, W, X, stream=None, topk=None):
+    p = F.Params.from_config(cfg, topk=topk)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
@@ -99,7 +99,7 @@ def check_caches(cfg, orc, st, heads):
     return flipped
 
 
-def compare(cfg, orc, snaps, st, heads, check_y):
+def compare(cfg, orc, snaps, st, heads, check_y, topk=None):
     """Per loop: sets exact, selections exact up to near-ties, O (and Y)
     within 1e-2 per row for at least 99.5% of the active rows and within
     5e-2 for all, every row above 1e-2 explained by a quantiser rounding flip
@@ -108,7 +108,8 @@ def compare(cfg, orc, snaps, st, heads, check_y):
     cols = np.concatenate([np.arange(h * dh, (h + 1) * dh) for h in heads])
     flipped = check_caches(cfg, orc, st, heads)
     worst = {}
-    sel_loop = {r: F.flashloop_selection_loop(F.Params.from_config(cfg), r) for r in range(2, cfg.n_loops + 1)}
+    sel_loop = {r: F.flashloop_selection_loop(F.Params.from_config(cfg, topk=topk), r)
+                for r in range(2, cfg.n_loops + 1)}
     for r in range(1, cfg.n_loops + 1):
         s = snaps[r]
         act = orc.active[r]
@@ -117,7 +118,10 @@ def compare(cfg, orc, snaps, st, heads, check_y):
         swapped = {}
         if r >= 2:
             for a, h in enumerate(heads):
-                swapped[a] = check_selection(s["cols"][h], orc.T[sel_loop[r]][a], orc.colmass[1][a])
+                # the mass that loop's selection ranked: the dense loop-1 mass, or the
+                # previous sparse loop's for a shrinking budget
+                mass = orc.colmass[sel_loop[r] - 1][a]
+                swapped[a] = check_selection(s["cols"][h], orc.T[sel_loop[r]][a], mass)
         og = bf16_rows(s["O"][act][:, cols]).reshape(act.size, len(heads), dh)
         oo = bf16_rows(orc.O_hist[r][act]).reshape(act.size, len(heads), dh)
         e = row_rel_l2(og.reshape(act.size, -1), oo.reshape(act.size, -1))
@@ -197,3 +201,23 @@ def test_loop_steps_are_repeatable():
         torch.cuda.synchronize()
         outs.append((torch_to_bf16_bits(st["O"]).copy(), torch_to_bf16_bits(st["Y"]).copy()))
     assert np.array_equal(outs[0][0], outs[1][0]) and np.array_equal(outs[0][1], outs[1][1])
+
+
+def test_loop_step_shrinking_budgets():
+    """Nested selections with shrinking budgets (40, 26, 13 columns): loops 3
+    and 4 rank the previous sparse loop's column mass over its selection."""
+    cfg = CONFIGS["tiny"]
+    topk = [cfg.seq, 40, 26, 13]
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    orc = O.OracleSequence(cfg, W, X, topk=topk).run()
+    p, st, snaps = run_gpu(cfg, W, X, topk=topk)
+    assert [F.flashloop_selection_loop(p, r) for r in (2, 3, 4)] == [2, 3, 4]
+    for r in (3, 4):
+        cols = snaps[r]["cols"]
+        prev = snaps[r - 1]["cols"]
+        for h in range(cfg.n_heads):
+            assert set(cols[h].tolist()) <= set(prev[h].tolist())  # nested
+            assert cols[h].size == topk[r - 1] and np.all(np.diff(cols[h]) > 0)
+    worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True, topk=topk)
+    print("shrinking", worst)
