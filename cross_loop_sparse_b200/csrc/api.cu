@@ -11,13 +11,16 @@
 namespace fl {
 int launch_gate(const flashloop_params*, const uint16_t*, const uint16_t*, const int32_t*,
                 const int32_t*, int, int32_t*, int32_t*, int32_t*, int, void*, int32_t*, cudaStream_t);
+int launch_gate_topk(const flashloop_params*, const uint16_t*, const uint16_t*, const int32_t*, const int32_t*,
+                     int, int, int32_t*, int32_t*, int32_t*, void*, int32_t*, cudaStream_t);
 int launch_kv_quant(const flashloop_params*, int, const float*, const float*, const int32_t*,
                     const int32_t*, flashloop_state*, cudaStream_t);
 int launch_selcol_dequant(const flashloop_params*, int, const int32_t*, int, int, flashloop_state*,
                           __half*, __half*, __half*, __half*, cudaStream_t);
 int launch_topk(const flashloop_params*, const float*, const int32_t*, int, int, int32_t*, int32_t*,
                 cudaStream_t, const float* row_m = nullptr, const float* row_z = nullptr,
-                float* probs_out = nullptr);
+                float* probs_out = nullptr, const int32_t* n_dev = nullptr, int32_t* k_out = nullptr,
+                const int32_t* out_map = nullptr);
 int launch_qkv_gemm(const flashloop_params*, const uint16_t*, const int32_t*, const int32_t*, int,
                     const uint16_t*, const float*, uint16_t*, float*, float*, int32_t*, cudaStream_t);
 int launch_out_gemm(const flashloop_params*, const uint16_t*, const int32_t*, const int32_t*, int,
@@ -159,6 +162,23 @@ int flashloop_gate(const flashloop_params* p, const uint16_t* x_cur, const uint1
     return FLASHLOOP_ERR_INVALID_ARG;
   return launch_gate(p, x_cur, x_prev, prev_active, n_prev, prev_capacity, active_out, slot_out,
                      n_active_out, out_capacity, workspace, err_word, as_stream(stream));
+}
+
+int flashloop_gate_topk(const flashloop_params* p, const uint16_t* x_cur, const uint16_t* x_prev,
+                        const int32_t* prev_active, const int32_t* n_prev, int32_t prev_capacity,
+                        int32_t budget, int32_t* active_out, int32_t* slot_out, int32_t* n_active_out,
+                        int32_t out_capacity, void* workspace, int32_t* err_word, void* stream) {
+  int rc = check_common(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (!x_cur || !x_prev || !active_out || !slot_out || !n_active_out || !workspace) return FLASHLOOP_ERR_INVALID_ARG;
+  if (prev_active != nullptr && n_prev == nullptr) return FLASHLOOP_ERR_INVALID_ARG;
+  if (prev_capacity < 1 || prev_capacity > p->seq || out_capacity < 1 || out_capacity > p->seq)
+    return FLASHLOOP_ERR_INVALID_ARG;
+  if (prev_active == nullptr && prev_capacity != p->seq) return FLASHLOOP_ERR_INVALID_ARG;
+  if (budget < 0 || budget > out_capacity) return FLASHLOOP_ERR_INVALID_ARG;
+  if (prev_capacity > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
+  return launch_gate_topk(p, x_cur, x_prev, prev_active, n_prev, prev_capacity, budget, active_out, slot_out,
+                          n_active_out, workspace, err_word, as_stream(stream));
 }
 
 int flashloop_qkv_gathered(const flashloop_params* p, const uint16_t* x, const int32_t* active,
@@ -342,6 +362,7 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   if (loop < 1 || loop > p->n_loops || !x_cur || !w_qkv || !w_o || !st || !st->Y || !st->rope_cs)
     return FLASHLOOP_ERR_INVALID_ARG;
   if (loop >= 2 && !x_prev) return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop >= 2 && p->gate_topk && p->seq > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
   rc = check_state(p, st, loop);
   if (rc != FLASHLOOP_OK) return rc;
   cudaStream_t s = as_stream(stream);
@@ -360,8 +381,12 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   int32_t* n_act = st->n_active + (loop - 1);
   const int32_t* prev_act = loop == 2 ? nullptr : st->active[loop - 2];
   const int32_t* n_prev = loop == 2 ? nullptr : st->n_active + (loop - 2);
-  rc = launch_gate(p, x_cur, x_prev, prev_act, n_prev, capacity_of(p, loop - 1), act,
-                   st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
+  if (p->gate_topk)
+    rc = launch_gate_topk(p, x_cur, x_prev, prev_act, n_prev, capacity_of(p, loop - 1), cap, act,
+                          st->slot[loop - 1], n_act, st->workspace, st->err_word, s);
+  else
+    rc = launch_gate(p, x_cur, x_prev, prev_act, n_prev, capacity_of(p, loop - 1), act,
+                     st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
   if (rc != FLASHLOOP_OK) return rc;
   rc = launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, st->q[cur], s);
   if (rc != FLASHLOOP_OK) return rc;
@@ -388,7 +413,7 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
 
 size_t flashloop_kv_workspace_bytes(const flashloop_params* p) {
   if (check_params(p) != FLASHLOOP_OK) return 0;
-  return workspace_layout(p).flags + (size_t)p->seq;
+  return workspace_layout(p).keys + (size_t)p->seq * sizeof(float);
 }
 
 int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur, const uint16_t* x_prev,
@@ -403,6 +428,7 @@ int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x
   if (loop == 1) return launch_qkv_quant_gemm(p, 1, x_cur, nullptr, nullptr, p->seq, w_qkv, st, nullptr, s);
   if (!x_prev || !st->n_active || !st->workspace || st->workspace_bytes < flashloop_kv_workspace_bytes(p))
     return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->gate_topk && p->seq > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
   for (int l = 2; l <= loop; ++l)
     if (!st->active[l - 1] || !st->slot[l - 1] || !st->k.res_codes[l - 1] || !st->k.res_scales[l - 1] ||
         !st->v.res_codes[l - 1] || !st->v.res_scales[l - 1])
@@ -410,9 +436,14 @@ int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x
   int32_t* act = st->active[loop - 1];
   int32_t* n_act = st->n_active + (loop - 1);
   const int cap = capacity_of(p, loop);
-  rc = launch_gate(p, x_cur, x_prev, loop == 2 ? nullptr : st->active[loop - 2],
-                   loop == 2 ? nullptr : st->n_active + (loop - 2), capacity_of(p, loop - 1), act,
-                   st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
+  if (p->gate_topk)
+    rc = launch_gate_topk(p, x_cur, x_prev, loop == 2 ? nullptr : st->active[loop - 2],
+                          loop == 2 ? nullptr : st->n_active + (loop - 2), capacity_of(p, loop - 1), cap, act,
+                          st->slot[loop - 1], n_act, st->workspace, st->err_word, s);
+  else
+    rc = launch_gate(p, x_cur, x_prev, loop == 2 ? nullptr : st->active[loop - 2],
+                     loop == 2 ? nullptr : st->n_active + (loop - 2), capacity_of(p, loop - 1), act,
+                     st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
   if (rc != FLASHLOOP_OK) return rc;
   return launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, nullptr, s);
 }

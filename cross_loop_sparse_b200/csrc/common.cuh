@@ -55,6 +55,7 @@ __device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w) {
 struct Workspace {
   size_t ticket;    // uint32 counter of the last-block compaction (gate)
   size_t flags;     // uint8 [S] per-candidate gate decisions
+  size_t keys;      // float [S] per-candidate change ratios (top-k retention)
   size_t k_new;     // float [S, H, dh] projected keys of the active rows (compact)
   size_t v_new;     // float [S, H, dh]
   size_t cols_kv;   // fp16 dequantised selected columns: 4 x [H, kmax, dh] or 2 x [H, S, dh]
@@ -76,6 +77,7 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   size_t off = 0;
   w.ticket = off; off = align256(off + 16);
   w.flags = off; off = align256(off + S);
+  w.keys = off; off = align256(off + S * sizeof(float));
   w.k_new = off; off = align256(off + S * H * dh * sizeof(float));
   w.v_new = off; off = align256(off + S * H * dh * sizeof(float));
   size_t sel = 4 * H * (size_t)pad8(max_topk(p)) * dh;

@@ -36,7 +36,8 @@ int launch_kv_quant_rows(int dh, int loop, int n_rows, int H, const int* bits, c
                          cudaStream_t stream);
 int launch_topk(const flashloop_params* p, const float* mass, const int32_t* cand, int n_cand, int k,
                 int32_t* out, int32_t* err, cudaStream_t stream, const float* row_m = nullptr,
-                const float* row_z = nullptr, float* probs_out = nullptr);
+                const float* row_z = nullptr, float* probs_out = nullptr, const int32_t* n_dev = nullptr,
+                int32_t* k_out = nullptr, const int32_t* out_map = nullptr);
 
 namespace {
 

@@ -29,17 +29,22 @@ __device__ __forceinline__ uint32_t order_key(float v) {
 __global__ void __launch_bounds__(kTopkThreads)
 topk_kernel(const float* __restrict__ mass, int S, const int32_t* __restrict__ cand, int n_cand,
             int k, int32_t* __restrict__ out, int32_t* err, const float* __restrict__ row_m,
-            const float* __restrict__ row_z, float* __restrict__ probs_out) {
-  extern __shared__ uint32_t keys[];  // [n], then the warps' histograms [kTopkWarps][256]
+            const float* __restrict__ row_z, float* __restrict__ probs_out, const int32_t* __restrict__ n_dev,
+            int32_t* __restrict__ k_out, const int32_t* __restrict__ out_map) {
+  extern __shared__ uint32_t keys[];  // [n_alloc], then the warps' histograms [kTopkWarps][256]
   __shared__ int hist[256];
   __shared__ int warp_sums[32];
   __shared__ uint32_t s_prefix;
   __shared__ int s_remaining;
   const int h = blockIdx.x;
-  const int n = cand ? n_cand : S;
+  const int n_alloc = cand ? n_cand : S;
+  // a device count may shorten the list (keys n_dev.. are not candidates)
+  const int n = n_dev ? max(0, min(n_alloc, *n_dev)) : n_alloc;
+  if (k > n) k = n;
+  if (k_out != nullptr && threadIdx.x == 0) k_out[h] = k;
   const int32_t* hc = cand ? cand + (size_t)h * n_cand : nullptr;
   const float* hm = mass + (size_t)h * S;
-  int* whist = reinterpret_cast<int*>(keys + n);
+  int* whist = reinterpret_cast<int*>(keys + n_alloc);
   const bool probs = row_m != nullptr;
   const float pm = probs ? row_m[h] : 0.f;
   const float prz = probs ? 1.f / row_z[h] : 0.f;
@@ -181,7 +186,7 @@ topk_kernel(const float* __restrict__ mass, int S, const int32_t* __restrict__ c
           ++eq_rank;
         }
         if (keep) {
-          if (pos < k) out[(size_t)h * k + pos] = hc ? hc[c] : c;
+          if (pos < k) out[(size_t)h * k + pos] = out_map ? out_map[c] : (hc ? hc[c] : c);
           ++pos;
         }
       }
@@ -193,7 +198,8 @@ topk_kernel(const float* __restrict__ mass, int S, const int32_t* __restrict__ c
 
 int launch_topk(const flashloop_params* p, const float* mass, const int32_t* cand, int n_cand,
                 int k, int32_t* out, int32_t* err, cudaStream_t stream, const float* row_m,
-                const float* row_z, float* probs_out) {
+                const float* row_z, float* probs_out, const int32_t* n_dev, int32_t* k_out,
+                const int32_t* out_map) {
   const int n = cand ? n_cand : p->seq;
   const size_t smem = ((size_t)n + kTopkWarps * 256) * sizeof(uint32_t);
   static bool attr_set = false;
@@ -203,7 +209,7 @@ int launch_topk(const flashloop_params* p, const float* mass, const int32_t* can
     attr_set = true;
   }
   topk_kernel<<<p->n_heads, kTopkThreads, smem, stream>>>(mass, p->seq, cand, n_cand, k, out, err, row_m, row_z,
-                                                          probs_out);
+                                                          probs_out, n_dev, k_out, out_map);
   return launch_status();
 }
 

@@ -40,11 +40,12 @@ class Params(ctypes.Structure):
     _fields_ = [("seq", c_int32), ("d_model", c_int32), ("n_heads", c_int32), ("head_dim", c_int32),
                 ("n_loops", c_int32), ("batch", c_int32), ("tau", c_float), ("rope_theta", c_float),
                 ("topk", c_int32 * MAX_LOOPS), ("bits", c_int32 * MAX_LOOPS),
-                ("capacity", c_int32 * MAX_LOOPS)]
+                ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32)]
 
     @classmethod
-    def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None):
-        """Params of a workload.Config; capacities default to S (no overflow possible)."""
+    def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None):
+        """Params of a workload.Config; capacities default to S (no overflow possible).
+        token_budgets (per loop) selects top-k token retention with those budgets."""
         p = cls()
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
@@ -56,6 +57,10 @@ class Params(ctypes.Structure):
             p.topk[r] = ks[r]
             p.bits[r] = cfg.bits[r]
             p.capacity[r] = p.seq if capacity is None else capacity[r]
+        if token_budgets is not None:
+            p.gate_topk = 1
+            for r in range(1, cfg.n_loops):
+                p.capacity[r] = token_budgets[r]
         return p
 
 
@@ -91,6 +96,7 @@ _SIG = {
     "flashloop_rope_table": (_I, [_P, _I, _V, _V]),
     "flashloop_gate": (_I, [_P, _V, _V, _V, _V, _I, _V, _V, _V, _I, _V, _V, _V]),
     "flashloop_gate_noalloc": (_I, [_P, _V, _V, _V, _V, _I, _V, _V, _V, _I, _V, _V]),
+    "flashloop_gate_topk": (_I, [_P, _V, _V, _V, _V, _I, _I, _V, _V, _V, _I, _V, _V, _V]),
     "flashloop_qkv_gathered": (_I, [_P, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V]),
     "flashloop_kv_quant_residual": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
     "flashloop_qkv_quant": (_I, [_P, _I, _V, _V, _V, _V, _S, _V, _V]),
@@ -179,6 +185,14 @@ def flashloop_gate(params, x_cur, x_prev, prev_active, n_prev, prev_capacity, ac
         ctypes.byref(params), _ptr(x_cur), _ptr(x_prev), _ptr(prev_active), _ptr(n_prev),
         prev_capacity, _ptr(active_out), _ptr(slot_out), _ptr(n_active_out), out_capacity,
         _ptr(workspace), _ptr(err_word), _stream(stream)))
+
+
+def flashloop_gate_topk(params, x_cur, x_prev, prev_active, n_prev, prev_capacity, budget, active_out,
+                        slot_out, n_active_out, out_capacity, workspace, err_word, stream=None):
+    return _check("flashloop_gate_topk", _lib.flashloop_gate_topk(
+        ctypes.byref(params), _ptr(x_cur), _ptr(x_prev), _ptr(prev_active), _ptr(n_prev), prev_capacity,
+        budget, _ptr(active_out), _ptr(slot_out), _ptr(n_active_out), out_capacity, _ptr(workspace),
+        _ptr(err_word), _stream(stream)))
 
 
 def flashloop_gate_noalloc(params, x_cur, x_prev, prev_active, n_prev, prev_capacity, active_out,

@@ -69,6 +69,7 @@ typedef struct flashloop_params {
   int32_t topk[FLASHLOOP_MAX_LOOPS];     /* column budget k_r per loop (loop 1 unused), non-increasing */
   int32_t bits[FLASHLOOP_MAX_LOOPS];     /* code width per loop: bits[0] = 8 (base); 8, 4 or 2 after */
   int32_t capacity[FLASHLOOP_MAX_LOOPS]; /* rows allocated for loop r's active list and residual stream */
+  int32_t gate_topk; /* 0: the tau threshold gate; else top-k token retention keeping capacity[r-1] tokens */
 } flashloop_params;
 
 /* One quantised cache (K or V) of a sequence: the loop-1 base over every
@@ -125,6 +126,20 @@ size_t flashloop_cache_bytes(const flashloop_params* p, const int32_t* n_per_loo
 int flashloop_rope_table(const flashloop_params* p, int32_t n_pos, float* cs, void* stream);
 
 /* ---------------------------------------------------------------- the path */
+
+/* (a1, top-k retention) [FlashLoop §4.1 "top-k tokens retained", App. D.1]:
+ * instead of the tau threshold, keep the `budget` candidates of largest
+ * normalised change ||x_cur - x_prev||^2 / ||x_prev||^2 (float32 sums, IEEE
+ * division; a zero previous row counts as +inf if it changed, 0 if not),
+ * ties to the lower token.  Candidates are prev_active[0..*n_prev) (ascending),
+ * or every token when prev_active is NULL.  Writes the kept tokens ascending
+ * to active_out, every token's position to slot_out (-1 = not kept) and
+ * min(budget, n_prev) to *n_active_out.  budget <= out_capacity,
+ * prev_capacity <= 49152. */
+int flashloop_gate_topk(const flashloop_params* p, const uint16_t* x_cur, const uint16_t* x_prev,
+                        const int32_t* prev_active, const int32_t* n_prev, int32_t prev_capacity,
+                        int32_t budget, int32_t* active_out, int32_t* slot_out, int32_t* n_active_out,
+                        int32_t out_capacity, void* workspace, int32_t* err_word, void* stream);
 
 /* (a1) Token change gate and stream compaction [FlashLoop §3.1, §4.1, App. D.1].
  * For the n_prev candidates prev_active[0..n_prev) (ascending), a token is
@@ -243,6 +258,7 @@ int flashloop_out_proj(const flashloop_params* p, const uint16_t* o, const int32
 /* One loop of the sublayer: a1..a7 at loop >= 2 (gate against x_prev), or the
  * dense setup at loop == 1 (x_prev unused): every token active, INT8 base,
  * dense causal attention on the reconstructed base, column mass, W_o.
+ * With p->gate_topk the gate is flashloop_gate_topk with budget capacity[r-1]. 
  * [FlashLoop §4, App. D]. */
 int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur,
                         const uint16_t* x_prev, const uint16_t* w_qkv, const uint16_t* w_o,

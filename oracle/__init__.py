@@ -19,6 +19,7 @@ from .flashloop_oracle import (  # noqa: F401
     first_order_storage,
     gate,
     gate_norms,
+    gate_topk,
     out_projection,
     pack_codes,
     project_qkv,

@@ -92,6 +92,25 @@ def gate(x_cur_bits, x_prev_bits, candidates, tau):
     return candidates[keep]
 
 
+def gate_topk(x_cur_bits, x_prev_bits, candidates, budget):
+    """Active set A^(r) by top-k token retention [FL §4.1, App. D.1]: the
+    ``budget`` candidates of largest normalised change ||x_r - x_(r-1)||^2 /
+    ||x_(r-1)||^2 (the square ranks like the norm ratio), ties to the lower
+    token, returned ascending.  A zero previous row ranks first if it changed
+    and last if it did not.  Keys are ranked in float32, as a float32 kernel
+    would hold them.
+    """
+    candidates = np.asarray(candidates, dtype=np.int64)
+    if budget >= candidates.size:
+        return candidates
+    D, P = gate_norms(x_cur_bits, x_prev_bits, candidates)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        key = np.where(P > 0, D / np.where(P > 0, P, 1.0), np.where(D > 0, np.inf, 0.0))
+    dense = np.full(int(candidates.max()) + 1, -np.inf, dtype=np.float32)
+    dense[candidates] = key.astype(np.float32)
+    return topk_columns(dense, candidates, budget)
+
+
 # --------------------------------------------------------------------------
 # (a2) projections and RoPE  [FL §4.3 "post-RoPE keys", App. E; App. G]
 # --------------------------------------------------------------------------
@@ -382,8 +401,11 @@ class OracleSequence:
     """
 
     def __init__(self, cfg, W, X, heads=None, quantize=True, topk=None, tau=None,
-                 keep_history=True):
+                 keep_history=True, token_budgets=None):
+        """``token_budgets`` (per loop, index r-1) switches the gate from the
+        tau threshold to top-k token retention with those budgets."""
         self.cfg = cfg
+        self.token_budgets = None if token_budgets is None else list(token_budgets)
         self.W = W
         self.X = X
         self.S = cfg.seq
@@ -459,7 +481,10 @@ class OracleSequence:
         a4 column selection, a6 sparse update, a7 output projection."""
         assert r == self.loop + 1 and r >= 2
         S = self.S
-        rows = gate(self.X[r - 1], self.X[r - 2], self.active[r - 1], self.tau)
+        if self.token_budgets is None:
+            rows = gate(self.X[r - 1], self.X[r - 2], self.active[r - 1], self.tau)
+        else:
+            rows = gate_topk(self.X[r - 1], self.X[r - 2], self.active[r - 1], self.token_budgets[r - 1])
         self.active[r] = rows
         k, v = self._project(r, rows)
         self.Kc.write_residual(r, rows, k)

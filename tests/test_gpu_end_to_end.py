@@ -18,8 +18,8 @@ from gpu_helpers import bf16_rows, bf16_to_torch, row_rel_l2, torch_to_bf16_bits
 TOL = 1e-2
 
 
-def run_gpu(cfg, W, X, stream=None, topk=None):
-    p = F.Params.from_config(cfg, topk=topk)
+def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None):
+    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])

@@ -223,6 +223,66 @@ def test_gate_recovers_planted_nested_sets(name):
         act = act_new
 
 
+@pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
+def test_gate_topk_recovers_planted_nested_sets(name):
+    """Top-k token retention [FL §4.1, D.1] with the planted budgets keeps
+    exactly the planted (strongly changed) tokens, nested loop to loop."""
+    cfg = CONFIGS[name]
+    X, planted = make_hidden_states(cfg)
+    act = np.arange(cfg.seq)
+    for r in range(2, cfg.n_loops + 1):
+        act_new = O.gate_topk(X[r - 1], X[r - 2], act, cfg.n_active(r))
+        assert np.array_equal(act_new, planted[r - 1])
+        assert np.all(np.isin(act_new, act))
+        act = act_new
+
+
+def test_gate_topk_order_ties_and_degenerate_rows():
+    """Invariants of the top-k gate on random rows with planted ties: the
+    result is an ascending subset of the candidates of size min(budget, n);
+    every kept token changed at least as much as every dropped one; among
+    equal changes the lower tokens are kept; a zero previous row that changed
+    ranks above all, one that did not ranks below all."""
+    rng = np.random.default_rng(11)
+    d = 64
+    for trial in range(25):
+        S = int(rng.integers(4, 80))
+        prev = f32_to_bf16_bits(rng.standard_normal((S, d)).astype(np.float32))
+        cur = f32_to_bf16_bits(bf16_bits_to_f32(prev) + rng.standard_normal((S, d)).astype(np.float32)
+                               * np.float32(rng.choice([0.01, 0.1, 0.5])))
+        # duplicates: identical (prev, cur) rows have identical changes
+        for _ in range(int(rng.integers(0, 4))):
+            a, b = rng.choice(S, size=2, replace=False)
+            prev[b], cur[b] = prev[a], cur[a]
+        zero_changed = int(rng.integers(0, S))
+        prev[zero_changed] = 0
+        cur[zero_changed] = f32_to_bf16_bits(np.ones(d, np.float32))
+        zero_still = (zero_changed + 1) % S
+        prev[zero_still] = 0
+        cur[zero_still] = 0
+        cand = np.sort(rng.choice(S, size=int(rng.integers(1, S + 1)), replace=False))
+        budget = int(rng.integers(0, cand.size + 2))
+        got = O.gate_topk(cur, prev, cand, budget)
+        assert got.size == min(budget, cand.size)
+        assert np.all(np.diff(got) > 0) and np.all(np.isin(got, cand))
+        if got.size in (0, cand.size):
+            continue
+        D, P = O.gate_norms(cur, prev, cand)
+        with np.errstate(divide="ignore", invalid="ignore"):
+            key = np.where(P > 0, D / np.where(P > 0, P, 1), np.where(D > 0, np.inf, 0)).astype(np.float32)
+        kept = np.isin(cand, got)
+        assert key[kept].min() >= key[~kept].max()
+        thr = key[kept].min()
+        tied_kept = cand[kept & (key == thr)]
+        tied_dropped = cand[~kept & (key == thr)]
+        if tied_dropped.size:
+            assert tied_kept.max() < tied_dropped.min()
+        if zero_changed in cand:
+            assert zero_changed in got
+        if zero_still in cand and got.size < cand.size and np.sum(key[cand != zero_still] > 0) >= got.size:
+            assert zero_still not in got
+
+
 # ---------------------------------------------------------------- top-k
 def test_topk_brute_force_with_ties():
     rng = np.random.default_rng(2)
