@@ -39,7 +39,7 @@ int launch_decode_select(const flashloop_params*, flashloop_decode_state*, cudaS
 int launch_decode_qkv(const flashloop_params*, int, const uint16_t*, const uint16_t*, flashloop_decode_state*,
                       cudaStream_t);
 int launch_decode_out(const flashloop_params*, const uint16_t*, flashloop_decode_state*, cudaStream_t);
-int launch_colmass(const flashloop_params*, const ColmassArgs&, cudaStream_t);
+int launch_colmass_tc(const flashloop_params*, const ColmassArgs&, void*, void*, cudaStream_t);
 
 // ---------------------------------------------------------------------------
 // checks
@@ -338,7 +338,8 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
     c.out = dense ? st->colmass[0] : st->colmass[1];
     c.scale_log2 = 1.0f;  // the rebuilt keys already carry log2(e)/sqrt(dh)
     c.err = st->err_word;
-    rc = launch_colmass(p, c, s);
+    const Workspace w = workspace_layout(p);
+    rc = launch_colmass_tc(p, c, ws_ptr<void>(st->workspace, w.cm_q), ws_ptr<void>(st->workspace, w.cm_rows), s);
   }
   return rc;
 }

@@ -512,6 +512,334 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 }
 
 // ---------------------------------------------------------------------------
+// Column mass on the tensor cores [FlashLoop §4.2, App. D.2: the loop's
+// column statistics rank the next selection]:
+//   c[j] = sum over rows i with token_i >= token_j of 2^(s_ij - m_i) / Z_i,
+// s in log2 units (the rebuilt keys carry log2(e)/sqrt(dh)), m and Z the
+// rows' final state.  Transposed score tiles S^T = Khat_tile . q_tile^T put
+// one column in each TMEM lane, so a column's mass is a sum inside one
+// thread (no cross-lane reduction).  A work item = 128 selected columns of
+// one head; it walks 64-row tiles from the first row whose token reaches the
+// item's smallest column token.  Rows come prepared per head: fp16 q (the
+// same type as the keys, as kind::f16 requires), 2^-m scale as m in log2
+// units, 1/Z and the row token.
+// Roles: warps 0-7 reduce (two per TMEM lane quarter, each 32 of a tile's 64
+// rows) and load the item's keys into TMEM (A operand); warp 8 allocates TMEM
+// and streams the row tiles (TMA for q, bulk copies for m, 1/Z, tokens);
+// warp 9 issues the MMAs.  All waits are bounded.
+// ---------------------------------------------------------------------------
+constexpr int kCmtCols = 128, kCmtRows = 64, kCmtStages = 4, kCmtThreads = 320;
+constexpr int kCmtRowThreads = 256;
+
+template <int DH>
+struct CmtCfg {
+  static constexpr int kQBytes = kCmtRows * DH * 2;  // q tile: 64 rows x DH (DH/64 swizzle chunks)
+  static constexpr int kSideBytes = 1024;            // m2, rz, tokens of the tile (3 x 256 B), padded
+  static constexpr int kStageBytes = kQBytes + kSideBytes;
+  static constexpr int kSmem = 1024 + kCmtStages * kStageBytes + 256 + 2 * 128 * 4;
+  static constexpr uint32_t kColA = 0;       // keys, fp16 pairs: DH/2 columns
+  static constexpr uint32_t kColS = 64;      // two S^T buffers of 64 columns
+  static constexpr uint32_t kIdesc = f16_idesc(128, kCmtRows, 0);
+};
+
+struct CmtArgs {
+  int S, H, kc, kcp, n_cap;   // n_cap: rows allocated in the prepared arrays (multiple of 64)
+  const int32_t* n_rows;      // device count of rows (NULL: S)
+  int row_cap;
+  const int32_t* cols;        // [H, kc] ascending tokens (NULL: identity)
+  const int32_t* rtok;        // [n_cap] row tokens, -1 past the last row
+  const float* m2;            // [H, n_cap] row max, log2 units
+  const float* rz;            // [H, n_cap] 1 / Z
+  const __half* k;            // [H, kcp, DH] rebuilt keys
+  float* out;                 // [H, S], written at the column tokens
+  int32_t* err;
+};
+
+__device__ __forceinline__ int cmt_first_row(const CmtArgs& g, int n_rows, int tok) {
+  int lo = 0, hi = n_rows;  // first row whose token is >= tok (row tokens ascend)
+  while (lo < hi) {
+    const int mid = (lo + hi) >> 1;
+    if (__ldg(g.rtok + mid) < tok) lo = mid + 1;
+    else hi = mid;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kCmtThreads, 1)
+colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
+  using C = CmtCfg<DH>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCmtStages * C::kStageBytes);
+  uint64_t* full = bars;                       // [stages]
+  uint64_t* empty = bars + kCmtStages;         // [stages]: MMA commit + 256 reducer arrivals
+  uint64_t* s_full = bars + 2 * kCmtStages;    // [2]
+  uint64_t* s_empty = s_full + 2;              // [2]
+  uint64_t* a_ready = s_empty + 2;             // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xsum = reinterpret_cast<float*>(smem + kCmtStages * C::kStageBytes + 256);  // [2][128]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_rows = g.n_rows ? *g.n_rows : g.S;
+  if (n_rows > g.row_cap) n_rows = g.row_cap;
+  if (n_rows < 0) n_rows = 0;
+  const int col_tiles = (g.kc + kCmtCols - 1) / kCmtCols;
+  const int total = col_tiles * g.H;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kCmtStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1 + kCmtRowThreads);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&s_empty[b], kCmtRowThreads);
+    }
+    mbar_init(a_ready, kCmtRowThreads);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 256);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  // item -> (head, column tile); the column tiles with the most rows come first
+  auto item_head = [&](int item) { return item % g.H; };
+  auto item_tile = [&](int item) { return item / g.H; };
+  auto item_rows = [&](int item, int& a_begin) {
+    const int h = item_head(item), ct = item_tile(item);
+    const int c0 = ct * kCmtCols;
+    const int tok0 = g.cols ? __ldg(g.cols + (size_t)h * g.kc + c0) : c0;
+    a_begin = (cmt_first_row(g, n_rows, tok0) / kCmtRows) * kCmtRows;
+    return (n_rows - a_begin + kCmtRows - 1) / kCmtRows;
+  };
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ loads
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[kCmtStages];
+      for (int s2 = 0; s2 < kCmtStages; ++s2) issued[s2] = -1;
+      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
+        const int h = item_head(item);
+        int a_begin;
+        const int nt = item_rows(item, a_begin);
+        for (int t = 0; t < nt && !*abort_flag; ++t) {
+          if (!mbar_wait_sleep(&empty[stage], phase ^ 1)) {
+            set_error(g.err, kDevErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          const int a0 = a_begin + t * kCmtRows;
+          mbar_arrive_expect_tx(&full[stage], C::kQBytes + 3 * kCmtRows * 4);
+#pragma unroll
+          for (int c = 0; c < DH / 64; ++c)
+            tma_load_3d(st + c * (kCmtRows * 128), &tm_q, c * 64, a0, h, &full[stage]);
+          uint8_t* side = st + C::kQBytes;
+          bulk_g2s(side, g.m2 + (size_t)h * g.n_cap + a0, kCmtRows * 4, &full[stage]);
+          bulk_g2s(side + 256, g.rz + (size_t)h * g.n_cap + a0, kCmtRows * 4, &full[stage]);
+          bulk_g2s(side + 512, g.rtok + a0, kCmtRows * 4, &full[stage]);
+          issued[stage] = phase;
+          if (++stage == kCmtStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      for (int s2 = 0; s2 < kCmtStages; ++s2)
+        if (issued[s2] >= 0) (void)mbar_wait_sleep(&full[s2], (uint32_t)issued[s2]);
+    }
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issue
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, u = 0, item_no = 0;
+      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x, ++item_no) {
+        int a_begin;
+        const int nt = item_rows(item, a_begin);
+        if (!mbar_wait_sleep(a_ready, item_no & 1)) {
+          set_error(g.err, kDevErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        bool ok = true;
+        for (int t = 0; t < nt; ++t, ++u) {
+          if (!mbar_wait_sleep(&full[stage], phase) || (u >= 2 && !mbar_wait_sleep(&s_empty[u & 1], ((u >> 1) - 1) & 1))) {
+            set_error(g.err, kDevErrTimeout);
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = tmem + C::kColS + (u & 1) * kCmtRows;
+          const uint32_t q_addr = smem_u32(smem + stage * C::kStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            const uint32_t qd = q_addr + (ks >> 2) * (kCmtRows * 128) + (ks & 3) * 32;
+            umma_f16_ts(sb, tmem + C::kColA + ks * 8, sw128_kmajor_desc(qd), C::kIdesc, ks > 0);
+          }
+          umma_commit(&s_full[u & 1]);
+          umma_commit(&empty[stage]);
+          if (++stage == kCmtStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ reducers
+    // Thread (quarter, half): TMEM lane = column quarter*32 + lane of the
+    // item; half 0 takes rows 0..31 of each tile, half 1 rows 32..63.  A
+    // named barrier cannot time out, so after a failed wait a warp goes on
+    // through the same barriers without touching TMEM ("dead").
+    const int quarter = warp & 3, half = warp >> 2;
+    const int col = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int pair_bar = 1 + quarter;
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity) {
+      if (!dead && __any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+      if (dead) return;
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar, parity))) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        dead = true;
+        return;
+      }
+      tc_fence_after();
+    };
+    int stage = 0;
+    uint32_t phase = 0, u = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+      const int h = item_head(item), ct = item_tile(item);
+      int a_begin;
+      const int nt = item_rows(item, a_begin);
+      const int c = ct * kCmtCols + col;
+      const int ctok = c < g.kc ? (g.cols ? __ldg(g.cols + (size_t)h * g.kc + c) : c) : 0x7fffffff;
+      // this column's keys into TMEM (the MMA's A operand): half h loads
+      // elements [h*DH/2, (h+1)*DH/2)
+      if (!dead) {
+#pragma unroll 1
+        for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
+          uint32_t r[16];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            uint4 w = make_uint4(0, 0, 0, 0);
+            if (c < g.kc) w = *reinterpret_cast<const uint4*>(g.k + ((size_t)h * g.kcp + c) * DH + e0 + v * 8);
+            r[4 * v] = w.x; r[4 * v + 1] = w.y; r[4 * v + 2] = w.z; r[4 * v + 3] = w.w;
+          }
+          __syncwarp();
+          tmem_st16(tmem + lane_base + C::kColA + e0 / 2, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(a_ready);
+      }
+      float acc = 0.f;
+      for (int t = 0; t < nt; ++t, ++u) {
+        wait_or_die(&full[stage], phase);
+        wait_or_die(&s_full[u & 1], (u >> 1) & 1);
+        if (!dead) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + half * 32, r);
+          tmem_wait_ld();
+          const uint8_t* side = smem + stage * C::kStageBytes + C::kQBytes;
+          const float* sm2 = reinterpret_cast<const float*>(side) + half * 32;
+          const float* srz = reinterpret_cast<const float*>(side + 256) + half * 32;
+          const int* stok = reinterpret_cast<const int*>(side + 512) + half * 32;
+          float pa[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float v = ex2(__uint_as_float(r[e]) - sm2[e]) * srz[e];
+            pa[e & 3] += stok[e] >= ctok ? v : 0.f;
+          }
+          acc += (pa[0] + pa[1]) + (pa[2] + pa[3]);
+          tc_fence_before();
+          mbar_arrive(&s_empty[u & 1]);
+          mbar_arrive(&empty[stage]);
+        }
+        if (++stage == kCmtStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+      // the two halves' sums of each column
+      xsum[half * 128 + col] = acc;
+      named_bar_sync(pair_bar, 64);
+      if (!dead && half == 0 && c < g.kc && ctok >= 0 && ctok < g.S)
+        g.out[(size_t)h * g.S + ctok] = acc + xsum[128 + col];
+      named_bar_sync(pair_bar, 64);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 256);
+  }
+}
+
+// Rows of the column mass, per head: fp16 q, m in log2 units, 1/Z, and the
+// row tokens (-1 past the last row, up to n_cap).
+template <int DH>
+__global__ void __launch_bounds__(256)
+colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, float* rz, int32_t* rtok) {
+  int n_rows = a.n_rows ? *a.n_rows : a.S;
+  if (n_rows > a.row_cap) n_rows = a.row_cap;
+  const int lane = threadIdx.x & 31;
+  const long long items = (long long)n_cap * a.H;
+  for (long long w = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); w < items; w += (long long)gridDim.x * 8) {
+    const int h = (int)(w % a.H), r = (int)(w / a.H);
+    int tok = -1;
+    if (r < n_rows) {
+      tok = a.rows ? a.rows[r] : r;
+      if (tok < 0 || tok >= a.S) {
+        if (lane == 0) set_error(a.err, FLASHLOOP_DEVERR_INDEX);
+        tok = -1;
+      }
+    }
+    __half* qd = q16 + ((size_t)h * n_cap + r) * DH;
+    constexpr int E = DH / 32;
+    float x[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) x[e] = 0.f;
+    if (tok >= 0) {
+      const uint16_t* qs = a.q + (size_t)tok * a.H * DH + (size_t)h * DH + lane * E;
+#pragma unroll
+      for (int e = 0; e < E; ++e) x[e] = bf16_bits_to_float(qs[e]);
+    }
+#pragma unroll
+    for (int e = 0; e < E; ++e) qd[lane * E + e] = __float2half_rn(x[e]);
+    if (lane == 0) {
+      m2[(size_t)h * n_cap + r] = tok >= 0 ? a.m[(size_t)h * a.S + tok] * kAtLog2e : 0.f;
+      rz[(size_t)h * n_cap + r] = tok >= 0 ? 1.f / a.z[(size_t)h * a.S + tok] : 0.f;
+      if (h == 0) rtok[r] = tok;
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 at_encode_fn() {
@@ -555,6 +883,43 @@ static int at_sm_count() {
     cached[dev] = n;
   }
   return cached[dev];
+}
+
+// Column mass of loop `a` on the tensor cores (prep + kernel).  scratch_q
+// holds [H, n_cap, dh] fp16, scratch_rows [H, n_cap] x 2 floats + [n_cap] ints.
+int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scratch_q, void* scratch_rows,
+                      cudaStream_t stream) {
+  const int dh = p->head_dim, H = p->n_heads;
+  const int n_cap = ((a.row_cap + kCmtRows - 1) / kCmtRows) * kCmtRows;
+  __half* q16 = static_cast<__half*>(scratch_q);
+  float* m2 = static_cast<float*>(scratch_rows);
+  float* rz = m2 + (size_t)H * n_cap;
+  int32_t* rtok = reinterpret_cast<int32_t*>(rz + (size_t)H * n_cap);
+  long long items = (long long)n_cap * H;
+  int pgrid = (int)((items + 7) / 8);
+  if (pgrid > 148 * 16) pgrid = 148 * 16;
+  if (dh == 128) colmass_prep_kernel<128><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rz, rtok);
+  else colmass_prep_kernel<64><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rz, rtok);
+  int rc = launch_status();
+  if (rc != FLASHLOOP_OK) return rc;
+  CUtensorMap tq;
+  rc = make_tmap_f16_3d(&tq, q16, dh, n_cap, H, dh, (uint64_t)n_cap * dh, 64, kCmtRows);
+  if (rc != FLASHLOOP_OK) return rc;
+  CmtArgs g{};
+  g.S = a.S; g.H = H; g.kc = a.kc; g.kcp = a.kcp; g.n_cap = n_cap; g.n_rows = a.n_rows; g.row_cap = a.row_cap;
+  g.cols = a.cols; g.rtok = rtok; g.m2 = m2; g.rz = rz; g.k = a.k_new; g.out = a.out; g.err = a.err;
+  const int max_items = ((a.kc + kCmtCols - 1) / kCmtCols) * H;
+  int grid = at_sm_count();
+  if (grid > max_items) grid = max_items;
+  if (grid < 1) grid = 1;
+  if (dh == 128) {
+    FL_TRY(cudaFuncSetAttribute(colmass_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, CmtCfg<128>::kSmem));
+    colmass_tc_kernel<128><<<grid, kCmtThreads, CmtCfg<128>::kSmem, stream>>>(tq, g);
+  } else {
+    FL_TRY(cudaFuncSetAttribute(colmass_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, CmtCfg<64>::kSmem));
+    colmass_tc_kernel<64><<<grid, kCmtThreads, CmtCfg<64>::kSmem, stream>>>(tq, g);
+  }
+  return launch_status();
 }
 
 // K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.

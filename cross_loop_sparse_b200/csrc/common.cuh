@@ -56,8 +56,8 @@ struct Workspace {
   size_t ticket;    // uint32 counter of the last-block compaction (gate)
   size_t flags;     // uint8 [S] per-candidate gate decisions
   size_t keys;      // float [S] per-candidate change ratios (top-k retention)
-  size_t k_new;     // float [S, H, dh] projected keys of the active rows (compact)
-  size_t v_new;     // float [S, H, dh]
+  size_t cm_q;      // column-mass scratch: fp16 q of the rows [H, S, dh] (room for float [S, H, dh])
+  size_t cm_rows;   // column-mass scratch: row max (log2), 1/Z [H, S] each, row tokens [S]
   size_t cols_kv;   // fp16 dequantised selected columns: 4 x [H, kmax, dh] or 2 x [H, S, dh]
   size_t total;
 };
@@ -78,8 +78,11 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   w.ticket = off; off = align256(off + 16);
   w.flags = off; off = align256(off + S);
   w.keys = off; off = align256(off + S * sizeof(float));
-  w.k_new = off; off = align256(off + S * H * dh * sizeof(float));
-  w.v_new = off; off = align256(off + S * H * dh * sizeof(float));
+  const size_t S64 = (S + 63) / 64 * 64;  // the column mass pads its rows to whole 64-row tiles
+  const size_t cmq = S * H * dh * sizeof(float) > S64 * H * dh * 2 ? S * H * dh * sizeof(float) : S64 * H * dh * 2;
+  const size_t cmr = S * H * dh * sizeof(float) > S64 * (8 * H + 4) ? S * H * dh * sizeof(float) : S64 * (8 * H + 4);
+  w.cm_q = off; off = align256(off + cmq);
+  w.cm_rows = off; off = align256(off + cmr);
   size_t sel = 4 * H * (size_t)pad8(max_topk(p)) * dh;
   size_t dense = 2 * H * (size_t)pad8(p->seq) * dh;
   w.cols_kv = off; off = align256(off + (sel > dense ? sel : dense) * sizeof(__half));
