@@ -221,3 +221,78 @@ def test_loop_step_shrinking_budgets():
             assert cols[h].size == topk[r - 1] and np.all(np.diff(cols[h]) > 0)
     worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True, topk=topk)
     print("shrinking", worst)
+
+
+@pytest.mark.parametrize("seq,k", [(300, 30), (131, 14), (64, 64)])
+def test_loop_step_ragged_sizes(seq, k):
+    """Sequence lengths and budgets that cut through the 128-row, 64-column
+    and 256-column tiles of every kernel (and k = S at 64)."""
+    cfg = CONFIGS["tiny"].with_(seq=seq)
+    topk = [seq] + [k] * (cfg.n_loops - 1)
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    orc = O.OracleSequence(cfg, W, X, topk=topk).run()
+    p, st, snaps = run_gpu(cfg, W, X, topk=topk)
+    worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True, topk=topk)
+    print(seq, k, worst)
+
+
+def test_full_budget_zero_threshold_is_dense_attention():
+    """tau = 0 and k = S: every token active and every column selected, so
+    loop r's output is dense causal attention with q^(r) over Khat^(r), Vhat^(r)
+    (the identity the method is built on), here on the GPU against a dense
+    float64 evaluation of the GPU's own caches and queries."""
+    cfg = CONFIGS["tiny"].with_(seq=192, tau=0.0)
+    S, H, dh = cfg.seq, cfg.n_heads, cfg.head_dim
+    topk = [S] * cfg.n_loops
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    p = F.Params.from_config(cfg, topk=topk, tau=0.0)
+    st = F.FlashLoopState(p)
+    xs = [bf16_to_torch(x) for x in X]
+    wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
+    slots = {}
+    for r in range(1, cfg.n_loops + 1):
+        F.flashloop_loop_step(p, r, xs[r - 1], xs[r - 2] if r > 1 else None, wqkv, wo, st)
+        torch.cuda.synchronize()
+        if r >= 2:
+            assert int(st["n_active"][r - 1].item()) == S
+            slots[r] = st[f"slot{r}"].cpu().numpy()
+        og = bf16_rows(torch_to_bf16_bits(st["O"])).reshape(S, H, dh)
+        q = bf16_rows(torch_to_bf16_bits(st[f"q{st.q_slot(r)}"])).reshape(S, H, dh)
+        toks = np.arange(S)
+        Kh, _ = gpu_reconstruct(st, cfg, "k", toks, r, slots)
+        Vh, _ = gpu_reconstruct(st, cfg, "v", toks, r, slots)
+        for h in range(H):
+            s = (q[:, h, :] @ Kh[:, h, :].T) / np.sqrt(dh)
+            s = np.where(np.tril(np.ones((S, S), bool)), s, -np.inf)
+            pmat = np.exp(s - s.max(axis=1, keepdims=True))
+            ref = (pmat @ Vh[:, h, :]) / pmat.sum(axis=1, keepdims=True)
+            err = row_rel_l2(og[:, h, :], ref)
+            assert err.max() < 1e-2, (r, h, err.max())
+    assert st.error_code() == 0
+
+
+def test_empty_active_set():
+    """A loop where no token changes enough: the gate keeps nothing and the
+    kernels of that loop run on zero rows; O and Y keep the previous loop's
+    rows and the next loop finds no candidates."""
+    cfg = CONFIGS["tiny"].with_(seq=128, tau=10.0)
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    p = F.Params.from_config(cfg, tau=10.0)
+    st = F.FlashLoopState(p)
+    xs = [bf16_to_torch(x) for x in X]
+    wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
+    F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
+    torch.cuda.synchronize()
+    o1 = torch_to_bf16_bits(st["O"]).copy()
+    y1 = torch_to_bf16_bits(st["Y"]).copy()
+    for r in range(2, cfg.n_loops + 1):
+        F.flashloop_loop_step(p, r, xs[r - 1], xs[r - 2], wqkv, wo, st)
+        torch.cuda.synchronize()
+        assert int(st["n_active"][r - 1].item()) == 0
+        assert np.all(st[f"slot{r}"].cpu().numpy() == -1)
+    assert np.array_equal(torch_to_bf16_bits(st["O"]), o1)
+    assert np.array_equal(torch_to_bf16_bits(st["Y"]), y1)
+    assert st.error_code() == 0
