@@ -300,34 +300,42 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       if (!dead) {
         const uint16_t* qsrc = half == 0 ? g.q_new : g.q_old;
         const bool load_q = tok >= 0 && (half == 0 || has_old);
+        const bool load_n = !g.dense && tok >= 0;
         const uint32_t qcol = half == 0 ? C::kColQn : C::kColQo;
-#pragma unroll 1
+        // 32-byte accesses: one full sector per thread and instruction
+        uint32_t qv[DH / 16][8];
+#pragma unroll
+        for (int v = 0; v < DH / 16; ++v) {
+          if (load_q) {
+            ld_global_v8(qsrc + (size_t)tok * HD + (size_t)h * DH + v * 16, qv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[v][e] = 0u;
+          }
+        }
+#pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 32) {
           uint32_t r[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            uint4 w = make_uint4(0, 0, 0, 0);
-            if (load_q) w = *reinterpret_cast<const uint4*>(qsrc + (size_t)tok * HD + (size_t)h * DH + c0 + v * 8);
-            const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) r[4 * v + q] = bf16x2_to_half2_bits(ws[q]);
-          }
+          for (int e = 0; e < 16; ++e) r[e] = bf16x2_to_half2_bits(qv[c0 / 16 + e / 8][e % 8]);
           __syncwarp();
           tmem_st16(tmem + lane_base + qcol + c0 / 2, r);
         }
-#pragma unroll 1
+        uint32_t nv[kHalfCols / 8][8];
+#pragma unroll
+        for (int v = 0; v < kHalfCols / 8; ++v) {
+          if (load_n) {
+            ld_global_v8(g.n_in + ((size_t)h * g.S + tok) * DH + half * kHalfCols + 8 * v, nv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) nv[v][e] = 0u;
+          }
+        }
+#pragma unroll
         for (int c0 = 0; c0 < kHalfCols; c0 += 16) {
           uint32_t r[16];
 #pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (!g.dense && tok >= 0)
-              w = *reinterpret_cast<const float4*>(g.n_in + ((size_t)h * g.S + tok) * DH + half * kHalfCols + c0 + 4 * v);
-            r[4 * v + 0] = __float_as_uint(w.x);
-            r[4 * v + 1] = __float_as_uint(w.y);
-            r[4 * v + 2] = __float_as_uint(w.z);
-            r[4 * v + 3] = __float_as_uint(w.w);
-          }
+          for (int e = 0; e < 16; ++e) r[e] = nv[c0 / 8 + e / 8][e % 8];
           __syncwarp();
           tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + c0, r);
         }
@@ -477,23 +485,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         tmem_wait_ld();
         if (tok >= 0) {
           const int col = half * kHalfCols + cc;
-          float4* nd = reinterpret_cast<float4*>(g.n_out + ((size_t)h * g.S + tok) * DH + col);
-#pragma unroll
-          for (int v = 0; v < 4; ++v)
-            nd[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
-                                __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
-          uint4* od = reinterpret_cast<uint4*>(g.o + (size_t)tok * HD + (size_t)h * DH + col);
+          float* nd = g.n_out + ((size_t)h * g.S + tok) * DH + col;
+          uint32_t w[8];
 #pragma unroll
           for (int v = 0; v < 2; ++v) {
-            uint32_t w[4];
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int e = 8 * v + 2 * q;
-              w[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(r[e]) * inv) |
-                     ((uint32_t)float_to_bf16_bits(__uint_as_float(r[e + 1]) * inv) << 16);
-            }
-            od[v] = make_uint4(w[0], w[1], w[2], w[3]);
+            for (int e = 0; e < 8; ++e) w[e] = r[8 * v + e];
+            st_global_v8(nd + 8 * v, w);
           }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q]) * inv) |
+                   ((uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q + 1]) * inv) << 16);
+          st_global_v8(g.o + (size_t)tok * HD + (size_t)h * DH + col, w);
         }
       }
       if (tok >= 0 && half == 0) {
@@ -925,6 +929,10 @@ int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scr
 // K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.
 int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
+  // the row warps move q, N and O rows in 32-byte accesses
+  const void* aligned32[] = {a.q_new, a.q_old, a.n_in, a.n_out, a.o};
+  for (const void* ptr : aligned32)
+    if (reinterpret_cast<uintptr_t>(ptr) % 32 != 0) return FLASHLOOP_ERR_INVALID_ARG;
   CUtensorMap tkn, tko, tvn, tvo;
   int rc = make_tmap_f16_3d(&tkn, a.k_new, dh, a.kc, H, dh, (uint64_t)kcp * dh, 64, kAtCols);
   if (rc == FLASHLOOP_OK) rc = make_tmap_f16_3d(&tvn, a.v_new, a.kc, dh, H, kcp, (uint64_t)kcp * dh, kAtCols, dh);

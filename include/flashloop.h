@@ -16,6 +16,10 @@
  *    call is asynchronous on the given stream (a cudaStream_t passed as
  *    void*, NULL = legacy default stream).
  *  - bf16 tensors are passed as uint16_t bit patterns, fp16 scales likewise.
+ *  - Device tensors start on a 32-byte boundary (cudaMalloc and PyTorch
+ *    allocations start on 256 bytes); the attention calls return
+ *    FLASHLOOP_ERR_INVALID_ARG for a query, numerator or output tensor that
+ *    does not.
  *  - Layouts are row-major.  Hidden states X are [S, d_model]; linear weights
  *    are [out, in] (y = x W^T); head h owns columns [h*dh, (h+1)*dh).
  *  - A loop r (1-based) indexes per-loop arrays at position r-1.

@@ -296,3 +296,30 @@ def test_empty_active_set():
     assert np.array_equal(torch_to_bf16_bits(st["O"]), o1)
     assert np.array_equal(torch_to_bf16_bits(st["Y"]), y1)
     assert st.error_code() == 0
+
+
+def test_attention_rejects_unaligned_output():
+    """The attention update moves q, N and O rows in 32-byte accesses: an
+    output tensor that does not start on 32 bytes is refused before any
+    launch, and the state is left as it was."""
+    cfg = CONFIGS["tiny"]
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    p = F.Params.from_config(cfg)
+    st = F.FlashLoopState(p)
+    xs = [bf16_to_torch(x) for x in X]
+    wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
+    F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
+    torch.cuda.synchronize()
+    o_before = torch_to_bf16_bits(st["O"]).copy()
+    good = st.c.O
+    st.c.O = good + 16
+    try:
+        with pytest.raises(F.FlashLoopError) as exc:
+            F.flashloop_sparse_attn_update(p, 1, st, 0)
+        assert exc.value.status == -1  # FLASHLOOP_ERR_INVALID_ARG
+    finally:
+        st.c.O = good
+    torch.cuda.synchronize()
+    assert np.array_equal(torch_to_bf16_bits(st["O"]), o_before)
+    assert st.error_code() == 0
