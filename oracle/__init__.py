@@ -14,9 +14,11 @@ from .flashloop_oracle import (  # noqa: F401
     apply_rope,
     cache_bytes,
     dense_causal_attention,
+    dense_causal_probs,
     dense_kv_bytes,
     dequantize_groups,
     first_order_storage,
+    fixed_mass_update,
     gate,
     gate_norms,
     gate_topk,

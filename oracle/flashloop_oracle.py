@@ -39,6 +39,11 @@ supports):
      ascending.  For r >= 3 the candidates are the previous selection.
   R9 column mass at loop 1 is the dense column sum of the softmax; at r >= 2
      it is summed over active rows for the selected columns only.
+  R10 fixed-mass form (the pages' eq. 3 reading, an option): each row's
+     selected columns J keep the total probability M_i they had in the
+     previous loop's full distribution; within J the mass is shared in
+     proportion to e^(s_new).  Unselected columns keep their probabilities,
+     so every row's distribution still sums to one [FL §4.2, D.2; FZ §3].
 
 Parity unpinned: nothing in this module is without a pin; the accuracy and
 reconstruction figures the paper reports on real models are out of reach
@@ -383,6 +388,51 @@ def sparse_update(rows, T, q_old_bits, q_new_bits, K_old, K_new, V_old, V_new, m
     return m2, Z2, N2, cmass
 
 
+def dense_causal_probs(q_bits, Khat):
+    """The full causal softmax of one head as an explicit [S, S] matrix:
+    P[i, j] = e^(s_ij) / sum_{j' <= i} e^(s_ij') for j <= i, 0 above the
+    diagonal (s_ij = q_i . Khat_j / sqrt(dh))."""
+    q = bf16_vals(q_bits)
+    S, dh = q.shape
+    s = (q @ np.asarray(Khat, dtype=np.float64).T) / math.sqrt(dh)
+    s = np.where(np.tri(S, dtype=bool), s, -np.inf)
+    e = np.exp(s - s.max(axis=1, keepdims=True))
+    return e / e.sum(axis=1, keepdims=True)
+
+
+def fixed_mass_update(rows, T, q_new_bits, K_new, V_old, V_new, P, O):
+    """Loop r >= 2 of one head in the fixed-mass form (reading R10), on the
+    explicit distributions.  For every active row i with J = {j in T : j <= i}:
+
+      M_i = sum_J P[i, j]                             (cached mass of the selection)
+      P'[i, j] = M_i e^(s_new_ij) / sum_J e^(s_new)    for j in J, else P[i, j]
+      O'_i = O_i - sum_J P[i, j] Vhat_j^(r-1) + sum_J P'[i, j] Vhat_j^(r)
+
+    P [S, S] and O [S, dh] (float64) are updated in place; returns the column
+    mass sum_i P'[i, j] over the active rows for j in T."""
+    rows = np.asarray(rows, dtype=np.int64)
+    T = np.asarray(T, dtype=np.int64)
+    dh = K_new.shape[1]
+    qn = bf16_vals(q_new_bits)
+    s_new = (qn @ np.asarray(K_new, dtype=np.float64).T) / math.sqrt(dh)   # [n, k]
+    Vo = np.asarray(V_old, dtype=np.float64)
+    Vn = np.asarray(V_new, dtype=np.float64)
+    cmass = np.zeros(T.size)
+    for a, i in enumerate(rows):
+        sel = T <= i
+        if not sel.any():
+            continue
+        J = T[sel]
+        p_old = P[i, J].copy()
+        M = p_old.sum()
+        e = np.exp(s_new[a, sel] - s_new[a, sel].max())
+        p_new = M * e / e.sum()
+        O[i] = O[i] - p_old @ Vo[sel] + p_new @ Vn[sel]
+        P[i, J] = p_new
+        cmass[sel] += p_new
+    return cmass
+
+
 def out_projection(o_bits, wo_bits):
     """Y = O W_o^T for the given rows, stored as bf16 (float64 arithmetic)."""
     return to_bf16_bits(bf16_vals(o_bits) @ bf16_vals(wo_bits).T)
@@ -401,10 +451,15 @@ class OracleSequence:
     """
 
     def __init__(self, cfg, W, X, heads=None, quantize=True, topk=None, tau=None,
-                 keep_history=True, token_budgets=None):
+                 keep_history=True, token_budgets=None, fixed_mass=False):
         """``token_budgets`` (per loop, index r-1) switches the gate from the
-        tau threshold to top-k token retention with those budgets."""
+        tau threshold to top-k token retention with those budgets.
+        ``fixed_mass`` runs loops >= 2 in the fixed-mass form (reading R10)
+        on explicit [S, S] distributions per head (small S only)."""
         self.cfg = cfg
+        self.fixed_mass = fixed_mass
+        self.P = None          # fixed-mass form: head -> [S, S] probabilities
+        self.Ofm = None        # fixed-mass form: head -> [S, dh] float64 outputs
         self.token_budgets = None if token_budgets is None else list(token_budgets)
         self.W = W
         self.X = X
@@ -445,7 +500,10 @@ class OracleSequence:
 
     def _store_output(self, r, rows):
         Hs, dh = len(self.heads), self.dh
-        O = self.N[:, rows, :] / self.Z[:, rows, None]            # [Hs, n, dh]
+        if self.fixed_mass:
+            O = self.Ofm[:, rows, :]
+        else:
+            O = self.N[:, rows, :] / self.Z[:, rows, None]        # [Hs, n, dh]
         self.O[rows] = to_bf16_bits(O.transpose(1, 0, 2).reshape(rows.size, Hs * dh))
         if self.all_heads:
             self.Y[rows] = out_projection(self.O[rows], self.W["wo"])
@@ -473,6 +531,9 @@ class OracleSequence:
             self.m[a], self.Z[a], self.N[a], cm[a] = dense_causal_attention(
                 self.q[1][:, a, :], Kh[:, a, :], Vh[:, a, :])
         self.colmass[1] = cm
+        if self.fixed_mass:
+            self.P = np.stack([dense_causal_probs(self.q[1][:, a, :], Kh[:, a, :]) for a in range(Hs)])
+            self.Ofm = np.einsum('hij,jhd->hid', self.P, Vh.astype(np.float64))
         self._store_output(1, rows)
         self.loop = 1
 
@@ -509,6 +570,10 @@ class OracleSequence:
             Kn = self.Kc.reconstruct(Ta, r)[:, a, :]
             Vo = self.Vc.reconstruct(Ta, r - 1)[:, a, :]
             Vn = self.Vc.reconstruct(Ta, r)[:, a, :]
+            if self.fixed_mass:
+                cm[a, Ta] = fixed_mass_update(rows, Ta, self.q[r][rows, a, :], Kn, Vo, Vn,
+                                              self.P[a], self.Ofm[a])
+                continue
             m2, Z2, N2, c = sparse_update(
                 rows, Ta, self.q[r - 1][rows, a, :], self.q[r][rows, a, :],
                 Ko, Kn, Vo, Vn, self.m[a, rows], self.Z[a, rows], self.N[a, rows])

@@ -29,6 +29,13 @@ def read_golden(name):
 
 
 @pytest.fixture(scope="module")
+def tiny_cfg_data():
+    cfg = CONFIGS["tiny"]
+    X, _ = make_hidden_states(cfg)
+    return cfg, make_weights(cfg), X
+
+
+@pytest.fixture(scope="module")
 def tiny():
     cfg = CONFIGS["tiny"]
     W = make_weights(cfg)
@@ -485,3 +492,97 @@ def test_decode_selection_is_topk_of_loop1_probabilities():
         want = sorted(sorted(range(pr.size), key=lambda j: (-float(pr[j]), j))[:k])
         assert dec.T[h].tolist() == want
         assert abs(dec.probs[h].sum() - 1) < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# fixed-mass form of the sparse update (reading R10) [FL §4.2, D.2; FZ §3]
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("quantize", [True, False])
+def test_fixed_mass_full_budget_zero_threshold_is_dense_attention(quantize):
+    """Every column j <= i selected: the cached mass of the selection is 1,
+    so each loop's distribution is the plain softmax of that loop."""
+    cfg = CONFIGS["tiny"].with_(seq=128)
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    S, H = cfg.seq, cfg.n_heads
+    run = O.OracleSequence(cfg, W, X, quantize=quantize, tau=0.0, topk=[S] * cfg.n_loops,
+                           fixed_mass=True)
+    rows = np.arange(S)
+    run.run_loop1()
+    for r in range(1, cfg.n_loops + 1):
+        if r >= 2:
+            run.run_loop(r)
+        K = run.Kc.reconstruct(rows, r).astype(np.float64)
+        V = run.Vc.reconstruct(rows, r).astype(np.float64)
+        for h in range(H):
+            q = bf16_bits_to_f32(run.q[r][:, h, :]).astype(np.float64)
+            want, p = _textbook(q, K[:, h], V[:, h], rows)
+            assert np.allclose(run.Ofm[h], want, rtol=1e-9, atol=1e-12), (r, h)
+            assert np.allclose(run.P[h], p, rtol=1e-9, atol=1e-15), (r, h)
+
+
+def test_fixed_mass_keeps_selected_mass_and_normalisation(tiny_cfg_data):
+    """After every loop each row is a distribution over j <= i; an active row's
+    selected columns carry the mass they had before the loop; inactive rows and
+    unselected columns do not move."""
+    cfg, W, X = tiny_cfg_data
+    S, H = cfg.seq, cfg.n_heads
+    run = O.OracleSequence(cfg, W, X, fixed_mass=True)
+    run.run_loop1()
+    upper = ~np.tri(S, dtype=bool)
+    for r in range(2, cfg.n_loops + 1):
+        before = run.P.copy()
+        run.run_loop(r)
+        after = run.P
+        assert np.all(after >= 0) and np.all(after[:, upper] == 0)
+        assert np.allclose(after.sum(axis=2), 1.0, rtol=0, atol=1e-12)
+        rows = run.active[r]
+        inactive = np.setdiff1d(np.arange(S), rows)
+        assert np.array_equal(after[:, inactive], before[:, inactive])
+        for h in range(H):
+            T = run.T[r][h]
+            unsel = np.setdiff1d(np.arange(S), T)
+            assert np.array_equal(after[h][np.ix_(rows, unsel)], before[h][np.ix_(rows, unsel)])
+            for i in rows[::7]:
+                J = T[T <= i]
+                assert abs(after[h, i, J].sum() - before[h, i, J].sum()) <= 1e-12
+                if J.size > 1:
+                    # within J the shares follow e^(s_new): log-ratios are score differences
+                    K = run.Kc.reconstruct(J, r)[:, h].astype(np.float64)
+                    q = bf16_bits_to_f32(run.q[r][i, h, :]).astype(np.float64)
+                    s = K @ q / math.sqrt(cfg.head_dim)
+                    lr = np.log(after[h, i, J]) - np.log(after[h, i, J[0]])
+                    assert np.allclose(lr, s - s[0], rtol=0, atol=1e-9)
+
+
+def test_fixed_mass_output_is_distribution_times_counted_values(tiny_cfg_data):
+    """Closed form of the incremental output: O_i = sum_j P[i, j] Vhat_j of the
+    last loop that updated the pair (i, j) (loop 1, or a loop where i was
+    active and j selected)."""
+    cfg, W, X = tiny_cfg_data
+    S, H = cfg.seq, cfg.n_heads
+    run = O.OracleSequence(cfg, W, X, fixed_mass=True).run()
+    cols = np.arange(S)
+    causal = cols[None, :] <= cols[:, None]
+    for h in range(H):
+        last = np.where(causal, 1, 0)
+        for r in range(2, cfg.n_loops + 1):
+            sel = np.zeros(S, bool); sel[run.T[r][h]] = True
+            upd = np.zeros((S, S), bool)
+            upd[run.active[r]] = sel[None, :]
+            last = np.where(upd & causal, r, last)
+        want = np.zeros((S, cfg.head_dim))
+        for l in range(1, cfg.n_loops + 1):
+            V = run.Vc.reconstruct(cols, l)[:, h].astype(np.float64)
+            want += np.where(last == l, run.P[h], 0.0) @ V
+        assert np.allclose(run.Ofm[h], want, rtol=1e-9, atol=1e-12), h
+
+
+def test_fixed_mass_unchanged_inputs_leave_output_unchanged():
+    cfg = CONFIGS["tiny"].with_(seq=128)
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    Xs = [X[0]] * cfg.n_loops
+    run = O.OracleSequence(cfg, W, Xs, tau=0.0, quantize=False, fixed_mass=True).run()
+    for r in range(2, cfg.n_loops + 1):
+        assert np.array_equal(run.O_hist[r], run.O_hist[1])
