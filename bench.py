@@ -146,7 +146,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     xs = [to_dev(x) for x in X]
     wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
-    p = F.Params.from_config(cfg)
+    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass)
     st = F.FlashLoopState(p, device=dev)
     S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
@@ -180,7 +180,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
                 e1.record(stream)
                 attn_events.append((r, e0, e1))
             F.flashloop_out_proj(p, st["O"], act, n_act, p.capacity[r - 1], wo, st["Y"])
-            n += 3
+            n += 4 if p.fixed_mass else 3  # the fixed-mass form runs a statistics and an update pass
         launches_per_step = n
 
     def barrier():
@@ -231,8 +231,10 @@ def run_cuda(args, cfg, rank, world, local_rank):
     achieved = flop2 / (ms2 * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
-                "kernel": "attn_tc_kernel<128>, loop-2 launch (sparse attention update, tcgen05)",
+                "traffic": None if args.fixed_mass else ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
+                "kernel": ("attn_tc_kernel<128> statistics + update passes, loop 2 (fixed-mass form, tcgen05)"
+                           if args.fixed_mass else
+                           "attn_tc_kernel<128>, loop-2 launch (sparse attention update, tcgen05)"),
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
                 "per_loop": {f"loop{r}": {"ms": round(statistics.mean(v), 4),
@@ -310,7 +312,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded workload generator; random-init weights of the stated shape)",
-        "config": {"workload": workload_desc(cfg),
+        "config": {"workload": workload_desc(cfg) + (", fixed-mass form of the update" if args.fixed_mass else ""),
                    "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
                    "parallelism": f"one sequence per GPU, {world} GPU(s), no exchange",
                    "active_tokens": {f"loop{r}": int(st['n_active'][r - 1].item()) for r in range(2, R + 1)},
@@ -621,6 +623,9 @@ def main():
     ap.add_argument("--impl", choices=["cuda", "reference"], default="cuda")
     ap.add_argument("--config", default="prefill_32k", choices=list(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--fixed-mass", action="store_true",
+                    help="prefill workloads: the fixed-mass form of the sparse update (no CPU baseline: its "
+                         "oracle keeps explicit S x S distributions)")
     ap.add_argument("--batch", type=int, default=None,
                     help="decode workloads: sequences per GPU (a smaller case for profiler captures)")
     args = ap.parse_args()
@@ -629,6 +634,8 @@ def main():
         if not cfg.decode:
             ap.error("--batch applies to decode workloads only")
         cfg = cfg.with_(batch=args.batch)
+    if args.fixed_mass and (cfg.decode or args.impl != "cuda"):
+        ap.error("--fixed-mass applies to the CUDA arm on prefill workloads only")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -647,7 +654,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     out = (run_decode_cuda if cfg.decode else run_cuda)(args, cfg, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fixed_mass:
         if cfg.decode:
             t_est, sample = DecodeOracleSample(cfg).step()
             value = round(cfg.batch / t_est, 4)

@@ -254,6 +254,9 @@ static int check_state(const flashloop_params* p, const flashloop_state* st, int
   for (int i = 0; i < 3; ++i)
     if (!st->q[i] || !st->m[i] || !st->Z[i] || !st->N[i]) return FLASHLOOP_ERR_INVALID_ARG;
   if (!st->colmass[0] || !st->k.base_codes || !st->v.base_codes) return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->fixed_mass)
+    for (int i = 0; i < 3; ++i)
+      if (!st->G[i]) return FLASHLOOP_ERR_INVALID_ARG;
   for (int r = 2; r <= loop; ++r)
     if (!st->active[r - 1] || !st->slot[r - 1]) return FLASHLOOP_ERR_INVALID_ARG;
   for (int r = 2; r <= loop; ++r)
@@ -328,6 +331,17 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
   a.o = st->O;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->head_dim);
   a.err = st->err_word;
+  if (p->fixed_mass && !dense) {
+    // fixed-mass form: a statistics pass (frame m' and factor g per row), then the update
+    a.g_in = st->G[prev];
+    a.g_out = st->G[cur];
+    a.mode = 1;
+    rc = launch_attn_tc(p, a, b.kcp, s);
+    if (rc != FLASHLOOP_OK) return rc;
+    a.mode = 2;
+  } else if (p->fixed_mass) {
+    a.g_out = st->G[cur];  // the dense loop's distribution: g = 1
+  }
   rc = launch_attn_tc(p, a, b.kcp, s);
   if (rc != FLASHLOOP_OK) return rc;
   if (dense || want_colmass) {
@@ -338,6 +352,7 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
     c.out = dense ? st->colmass[0] : st->colmass[1];
     c.scale_log2 = 1.0f;  // the rebuilt keys already carry log2(e)/sqrt(dh)
     c.err = st->err_word;
+    c.g = p->fixed_mass ? st->G[cur] : nullptr;
     const Workspace w = workspace_layout(p);
     rc = launch_colmass_tc(p, c, ws_ptr<void>(st->workspace, w.cm_q), ws_ptr<void>(st->workspace, w.cm_rows), s);
   }
@@ -456,6 +471,7 @@ static int check_decode_params(const flashloop_params* p) {
   int rc = check_params(p);
   if (rc != FLASHLOOP_OK) return rc;
   if (p->batch < 1 || p->batch > 64) return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->fixed_mass) return FLASHLOOP_ERR_UNSUPPORTED;  // decode keeps the running (m, N, Z) form
   const int hd = p->n_heads * p->head_dim, hg = hd / 32;
   if (hd % 256 != 0 || 256 % hg != 0 || hg % 8 != 0) return FLASHLOOP_ERR_UNSUPPORTED;
   if (p->n_loops >= 2 && p->topk[1] > p->seq + 1) return FLASHLOOP_ERR_INVALID_ARG;

@@ -27,6 +27,9 @@ struct AttnArgs {
   uint16_t* o;                  // bf16 [S, H*DH]
   float scale_log2;             // log2(e) / sqrt(dh)
   int32_t* err;
+  int mode;                     // 0 running state, 1 / 2 fixed-mass statistics / update pass
+  const float* g_in;            // [H, S] selected-column factor of loop r-1 (fixed-mass passes)
+  float* g_out;                 // [H, S] (statistics pass; the dense loop writes 1 when set)
 };
 
 struct ColmassArgs {
@@ -42,6 +45,7 @@ struct ColmassArgs {
   float* out;              // [H, S], written at the column tokens
   float scale_log2;
   int32_t* err;
+  const float* g;          // [H, S] selected-column factor of the rows (NULL: 1)
 };
 
 }  // namespace fl

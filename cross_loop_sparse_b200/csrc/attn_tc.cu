@@ -23,6 +23,17 @@
 // maximum exceeds it by 8 (log2 units), which keeps every exponential
 // <= 2^8 and represents the same (m, N, Z) state (N and Z are defined up to
 // the common factor e^m).  All waits are bounded.
+//
+// Fixed-mass form [FlashLoop §4.2 "rescales selected-column probabilities by
+// their cached full-attention mass"]: the selected columns J of row i keep
+// the probability mass M_i they had after loop r-1 and share it in
+// proportion to e^(s_new).  With a per-row factor g (the weight of the
+// selected columns relative to e^(s - m) / Z; g = 1 after the dense loop)
+// that is N' = a N - g_prev sum_J e^(s_old - m') V_old + g sum_J e^(s_new - m') V_new,
+// Z' = a Z, g = g_prev sum_J e^(s_old - m') / sum_J e^(s_new - m').  Two
+// launches: a statistics pass (mode 1: S tiles and exponential sums only,
+// no V, no N) fixes m' and g; the update pass (mode 2) then adds the
+// contributions in that fixed frame, with no running maximum.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -43,7 +54,7 @@ struct AtCfg {
   static constexpr int kKBytes = kAtCols * DH * 2;  // K tile: 64 rows x DH (DH/64 swizzle chunks)
   static constexpr int kVBytes = DH * kAtCols * 2;  // V^T tile: DH rows x 64
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kVBytes;
-  static constexpr int kSmem = 1024 + kAtStages * kStageBytes + 512 + 6 * 128 * 4;
+  static constexpr int kSmem = 1024 + kAtStages * kStageBytes + 512 + 8 * 128 * 4;
   static constexpr uint32_t kColQn = 0;
   static constexpr uint32_t kColQo = DH / 2;
   static constexpr uint32_t kColN = DH;
@@ -52,8 +63,12 @@ struct AtCfg {
   static constexpr uint32_t kIdescPV = f16_idesc(128, DH, 0);
 };
 
+enum AtMode { kAtRunning = 0, kAtFixedMassStats = 1, kAtFixedMassUpdate = 2 };
+
 struct AtArgs {
   int S, H, kc, dense;
+  const float* g_in;     // [H, S] selected-column factor of loop r-1 (fixed-mass modes)
+  float* g_out;          // [H, S] written by mode 1 (and set to 1 by the dense loop)
   const int32_t* rows;
   const int32_t* n_rows;
   int row_cap;
@@ -91,7 +106,7 @@ __device__ __forceinline__ int at_tiles(const AtArgs& g, int h, int rt, int n_ro
   return (nc + kAtCols - 1) / kAtCols;
 }
 
-template <int DH>
+template <int DH, int MODE>
 __global__ void __launch_bounds__(kAtThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
                const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_vo, AtArgs g) {
@@ -144,7 +159,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
     if (lane == 0) {
       int stage = 0;
       uint32_t phase = 0;
-      const uint32_t bytes = has_old ? C::kStageBytes : (C::kKBytes + C::kVBytes);
+      constexpr bool load_v = MODE != kAtFixedMassStats;
+      const uint32_t bytes = (has_old ? 2 : 1) * (C::kKBytes + (load_v ? C::kVBytes : 0));
       int issued[kAtStages];
       for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
       for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
@@ -161,12 +177,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 #pragma unroll
           for (int c = 0; c < DH / 64; ++c)
             tma_load_3d(st + c * (kAtCols * 128), &tm_kn, c * 64, t * kAtCols, h, &kv_full[stage]);
-          tma_load_3d(st + 2 * C::kKBytes, &tm_vn, t * kAtCols, 0, h, &kv_full[stage]);
+          if (load_v) tma_load_3d(st + 2 * C::kKBytes, &tm_vn, t * kAtCols, 0, h, &kv_full[stage]);
           if (has_old) {
 #pragma unroll
             for (int c = 0; c < DH / 64; ++c)
               tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), &tm_ko, c * 64, t * kAtCols, h, &kv_full[stage]);
-            tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, &tm_vo, t * kAtCols, 0, h, &kv_full[stage]);
+            if (load_v) tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, &tm_vo, t * kAtCols, 0, h, &kv_full[stage]);
           }
           issued[stage] = phase;
           if (++stage == kAtStages) {
@@ -229,16 +245,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
               break;
             }
             tc_fence_after();
-            const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
-            const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKBytes);
-#pragma unroll
-            for (int ks = 0; ks < kAtCols / 16; ++ks)
-              umma_f16_ts(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
-            if (has_old) {
+            if (MODE != kAtFixedMassStats) {  // the statistics pass has no P.V
+              const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
+              const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKBytes);
 #pragma unroll
               for (int ks = 0; ks < kAtCols / 16; ++ks)
-                umma_f16_ts(tmem + C::kColN, pcol + 32 + ks * 8, sw128_kmajor_desc(v_addr + C::kVBytes + ks * 32),
-                            C::kIdescPV, 1u);
+                umma_f16_ts(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
+              if (has_old) {
+#pragma unroll
+                for (int ks = 0; ks < kAtCols / 16; ++ks)
+                  umma_f16_ts(tmem + C::kColN, pcol + 32 + ks * 8, sw128_kmajor_desc(v_addr + C::kVBytes + ks * 32),
+                              C::kIdescPV, 1u);
+              }
             }
             umma_commit(&kv_empty[prev_stage]);
             umma_commit(&pv_done[up & 1]);
@@ -267,7 +285,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
     const int row = quarter * 32 + lane;
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const int pair_bar = 1 + quarter;
-    float* xchg = reinterpret_cast<float*>(tmem_slot + 4);  // [2 parities][2 halves][128] maxima, then [2][128] sums
+    float* xchg = reinterpret_cast<float*>(tmem_slot + 4);  // [2 parities][2 halves][128] maxima, [2][128] sums, [2][128] old sums
+    constexpr bool stats = MODE == kAtFixedMassStats;     // fixed-mass statistics pass
+    constexpr bool fixed = MODE == kAtFixedMassUpdate;    // fixed-mass update pass
     const int HD = g.H * DH;
     constexpr int kHalfCols = DH / 2;
     bool dead = false;
@@ -295,12 +315,38 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           tok = -1;
         }
       }
+      // Per-row frame.  Running state (mode 0) and statistics pass: the
+      // reference starts at the previous maximum and is raised lazily.  Update
+      // pass: the frame is the statistics pass's reference, lifted by log2 of
+      // the larger g so that the scaled exponentials stay <= 2^8; N_in and Z_in
+      // are brought into it by a = 2^(m_in - m_ref).
+      float m_ref = 0.f, z = 0.f, z_old = 0.f, alpha = 1.f, g_prev = 1.f;
+      float off_new = 0.f, off_old = 0.f;  // update pass: exponent offsets m_ref - log2 g
+      if (tok >= 0) {
+        const size_t hi = (size_t)h * g.S + tok;
+        m_ref = g.dense ? -INFINITY : g.m_in[hi] * kAtLog2e;
+        if (MODE == kAtRunning) {
+          if (!g.dense && half == 0) z = g.z_in[hi];
+        } else {
+          g_prev = g.g_in[hi];
+          if (fixed) {
+            const float g_new = g.g_out[hi];
+            const float lift = fmaxf(0.f, log2f(fmaxf(g_prev, g_new)));
+            const float m_in = m_ref;
+            m_ref = g.m_out[hi] * kAtLog2e + lift;
+            alpha = ex2(m_in - m_ref);
+            off_new = m_ref - log2f(g_new);   // g = 0 gives +inf: exponentials of 0
+            off_old = m_ref - log2f(g_prev);
+            if (half == 0) z = alpha * g.z_in[hi];
+          }
+        }
+      }
       // Q (fp16 pairs, exact from bf16) and this half of N into TMEM.  The
       // rebuilt keys carry the factor log2(e)/sqrt(dh), so S is in log2 units.
       if (!dead) {
         const uint16_t* qsrc = half == 0 ? g.q_new : g.q_old;
         const bool load_q = tok >= 0 && (half == 0 || has_old);
-        const bool load_n = !g.dense && tok >= 0;
+        const bool load_n = !g.dense && tok >= 0 && !stats;
         const uint32_t qcol = half == 0 ? C::kColQn : C::kColQo;
         // 32-byte accesses: one full sector per thread and instruction
         uint32_t qv[DH / 16][8];
@@ -335,18 +381,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         for (int c0 = 0; c0 < kHalfCols; c0 += 16) {
           uint32_t r[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = nv[c0 / 8 + e / 8][e % 8];
+          for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(nv[c0 / 8 + e / 8][e % 8]) * alpha);
           __syncwarp();
           tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + c0, r);
         }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(q_ready);
-      }
-      float m_ref = 0.f, z = 0.f;
-      if (tok >= 0) {
-        m_ref = g.dense ? -INFINITY : g.m_in[(size_t)h * g.S + tok] * kAtLog2e;
-        if (!g.dense && half == 0) z = g.z_in[(size_t)h * g.S + tok];
       }
 
       const int32_t* hcols = g.cols ? g.cols + (size_t)h * g.kc : nullptr;
@@ -394,73 +435,89 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
               }
             }
           }
-          // tree reduction: 5 dependent steps instead of a 32-long chain
-          float t16[16];
+          if (!fixed) {
+            // tree reduction: 5 dependent steps instead of a 32-long chain
+            float t16[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) t16[e] = fmaxf(__uint_as_float(rn[e]), __uint_as_float(rn[e + 16]));
+            for (int e = 0; e < 16; ++e) t16[e] = fmaxf(__uint_as_float(rn[e]), __uint_as_float(rn[e + 16]));
 #pragma unroll
-          for (int w = 8; w > 0; w >>= 1)
+            for (int w = 8; w > 0; w >>= 1)
 #pragma unroll
-            for (int e = 0; e < w; ++e) t16[e] = fmaxf(t16[e], t16[e + w]);
-          mx = t16[0];
+              for (int e = 0; e < w; ++e) t16[e] = fmaxf(t16[e], t16[e + w]);
+            mx = t16[0];
+          }
         }
-        float* xm = xchg + (b * 2) * 128;  // [half][128] of this parity
-        xm[half * 128 + row] = mx;
-        named_bar_sync(pair_bar, 64);
-        mx = fmaxf(mx, xm[(1 - half) * 128 + row]);
+        if (!fixed) {  // the update pass has a fixed frame: no maxima to exchange
+          float* xm = xchg + (b * 2) * 128;  // [half][128] of this parity
+          xm[half * 128 + row] = mx;
+          named_bar_sync(pair_bar, 64);
+          mx = fmaxf(mx, xm[(1 - half) * 128 + row]);
+        }
         if (dead) continue;
-        const bool need = mx > m_ref + kRescaleThreshold;
+        const bool need = !fixed && mx > m_ref + kRescaleThreshold;
         if (__any_sync(0xffffffffu, need)) {
           // raise the reference of this warp's rows: N and Z scale by 2^(m_ref - mx)
           const float new_ref = need ? mx : m_ref;
           const float f = need ? ex2(m_ref - new_ref) : 1.f;
-          if (t > 0) {
-            const uint32_t up = u - 1;
-            wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
-            if (dead) continue;
-          }
+          if (!stats) {  // the statistics pass keeps no N
+            if (t > 0) {
+              const uint32_t up = u - 1;
+              wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+              if (dead) continue;
+            }
 #pragma unroll 1
-          for (int cc = 0; cc < kHalfCols; cc += 16) {
-            uint32_t r[16];
-            __syncwarp();
-            tmem_ld16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
-            tmem_wait_ld();
+            for (int cc = 0; cc < kHalfCols; cc += 16) {
+              uint32_t r[16];
+              __syncwarp();
+              tmem_ld16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
+              tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
-            __syncwarp();
-            tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
+              for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+              __syncwarp();
+              tmem_st16(tmem + lane_base + C::kColN + half * kHalfCols + cc, r);
+            }
+            tmem_wait_st();
           }
-          tmem_wait_st();
           z *= f;
+          z_old *= f;
           m_ref = new_ref;
         }
         uint32_t pk[16];
+        const float o_new = fixed ? off_new : m_ref;
+        const float o_old = fixed ? off_old : m_ref;
         // four independent partial sums per matrix (short dependency chains)
         float za[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int e2 = 0; e2 < 16; ++e2) {
-          const float p0 = ex2(__uint_as_float(rn[2 * e2]) - m_ref);
-          const float p1 = ex2(__uint_as_float(rn[2 * e2 + 1]) - m_ref);
+          const float p0 = ex2(__uint_as_float(rn[2 * e2]) - o_new);
+          const float p1 = ex2(__uint_as_float(rn[2 * e2 + 1]) - o_new);
           za[e2 & 3] += p0 + p1;
           pk[e2] = pack_half2(p0, p1);
         }
-        __syncwarp();
-        tmem_st16(sbase + half * 16, pk);
+        if (!stats) {
+          __syncwarp();
+          tmem_st16(sbase + half * 16, pk);
+        }
+        float zb[4] = {0.f, 0.f, 0.f, 0.f};
         if (has_old) {
-          float zb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
-            const float p0 = ex2(__uint_as_float(ro[2 * e2]) - m_ref);
-            const float p1 = ex2(__uint_as_float(ro[2 * e2 + 1]) - m_ref);
+            const float p0 = ex2(__uint_as_float(ro[2 * e2]) - o_old);
+            const float p1 = ex2(__uint_as_float(ro[2 * e2 + 1]) - o_old);
             zb[e2 & 3] += p0 + p1;
             pk[e2] = pack_half2(-p0, -p1);
           }
-          __syncwarp();
-          tmem_st16(sbase + 32 + half * 16, pk);
-#pragma unroll
-          for (int i = 0; i < 4; ++i) za[i] -= zb[i];
+          if (!stats) {
+            __syncwarp();
+            tmem_st16(sbase + 32 + half * 16, pk);
+          }
         }
-        z += (za[0] + za[1]) + (za[2] + za[3]);
+        if (MODE == kAtRunning) {
+          z += ((za[0] + za[1]) + (za[2] + za[3])) - ((zb[0] + zb[1]) + (zb[2] + zb[3]));
+        } else if (stats) {
+          z += (za[0] + za[1]) + (za[2] + za[3]);
+          z_old += (zb[0] + zb[1]) + (zb[2] + zb[3]);
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
@@ -471,11 +528,24 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       }
       // combine the two halves' sums
       float* xz = xchg + 4 * 128;
+      float* xzo = xchg + 6 * 128;
       xz[half * 128 + row] = z;
+      xzo[half * 128 + row] = z_old;
       named_bar_sync(pair_bar, 64);
       const float z_row = xz[row] + xz[128 + row];
+      const float z_old_row = xzo[row] + xzo[128 + row];
       named_bar_sync(pair_bar, 64);
       if (dead) continue;
+      if (stats) {
+        // the frame and the selected-column factor for the update pass:
+        // g = g_prev sum_J e^(s_old - m') / sum_J e^(s_new - m'), kept when J is empty
+        if (tok >= 0 && half == 0) {
+          const size_t hi = (size_t)h * g.S + tok;
+          g.m_out[hi] = m_ref / kAtLog2e;
+          g.g_out[hi] = z_row > 0.f ? g_prev * (z_old_row / z_row) : g_prev;
+        }
+        continue;
+      }
       const float inv = 1.f / z_row;
 #pragma unroll 1
       for (int cc = 0; cc < kHalfCols; cc += 16) {
@@ -503,6 +573,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       if (tok >= 0 && half == 0) {
         g.m_out[(size_t)h * g.S + tok] = m_ref / kAtLog2e;
         g.z_out[(size_t)h * g.S + tok] = z_row;
+        if (g.dense && g.g_out) g.g_out[(size_t)h * g.S + tok] = 1.f;
       }
       tc_fence_before();
     }
@@ -837,7 +908,8 @@ colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, floa
     for (int e = 0; e < E; ++e) qd[lane * E + e] = __float2half_rn(x[e]);
     if (lane == 0) {
       m2[(size_t)h * n_cap + r] = tok >= 0 ? a.m[(size_t)h * a.S + tok] * kAtLog2e : 0.f;
-      rz[(size_t)h * n_cap + r] = tok >= 0 ? 1.f / a.z[(size_t)h * a.S + tok] : 0.f;
+      rz[(size_t)h * n_cap + r] =
+          tok >= 0 ? (a.g ? a.g[(size_t)h * a.S + tok] : 1.f) / a.z[(size_t)h * a.S + tok] : 0.f;
       if (h == 0) rtok[r] = tok;
     }
   }
@@ -949,17 +1021,27 @@ int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaSt
   g.row_cap = a.row_cap; g.cols = a.cols; g.q_new = a.q_new; g.q_old = a.q_old; g.m_in = a.m_in;
   g.z_in = a.z_in; g.n_in = a.n_in; g.m_out = a.m_out; g.z_out = a.z_out; g.n_out = a.n_out; g.o = a.o;
   g.scale_log2 = a.scale_log2; g.err = a.err;
+  g.g_in = a.g_in; g.g_out = a.g_out;
   const int max_items = ((a.row_cap + kAtRows - 1) / kAtRows) * H;
   int grid = at_sm_count();
   if (grid > max_items) grid = max_items;
   if (grid < 1) grid = 1;
+  if (a.mode != kAtRunning && (a.dense || !a.g_in || !a.g_out)) return FLASHLOOP_ERR_INVALID_ARG;
+  auto launch = [&](auto kernel, int smem) -> int {
+    FL_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    kernel<<<grid, kAtThreads, smem, stream>>>(tkn, tko, tvn, tvo, g);
+    return FLASHLOOP_OK;
+  };
   if (dh == 128) {
-    FL_TRY(cudaFuncSetAttribute(attn_tc_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtCfg<128>::kSmem));
-    attn_tc_kernel<128><<<grid, kAtThreads, AtCfg<128>::kSmem, stream>>>(tkn, tko, tvn, tvo, g);
+    if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<128, kAtFixedMassStats>, AtCfg<128>::kSmem);
+    else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<128, kAtFixedMassUpdate>, AtCfg<128>::kSmem);
+    else rc = launch(attn_tc_kernel<128, kAtRunning>, AtCfg<128>::kSmem);
   } else {
-    FL_TRY(cudaFuncSetAttribute(attn_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, AtCfg<64>::kSmem));
-    attn_tc_kernel<64><<<grid, kAtThreads, AtCfg<64>::kSmem, stream>>>(tkn, tko, tvn, tvo, g);
+    if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<64, kAtFixedMassStats>, AtCfg<64>::kSmem);
+    else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<64, kAtFixedMassUpdate>, AtCfg<64>::kSmem);
+    else rc = launch(attn_tc_kernel<64, kAtRunning>, AtCfg<64>::kSmem);
   }
+  if (rc != FLASHLOOP_OK) return rc;
   return launch_status();
 }
 

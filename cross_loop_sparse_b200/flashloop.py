@@ -40,13 +40,16 @@ class Params(ctypes.Structure):
     _fields_ = [("seq", c_int32), ("d_model", c_int32), ("n_heads", c_int32), ("head_dim", c_int32),
                 ("n_loops", c_int32), ("batch", c_int32), ("tau", c_float), ("rope_theta", c_float),
                 ("topk", c_int32 * MAX_LOOPS), ("bits", c_int32 * MAX_LOOPS),
-                ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32)]
+                ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32), ("fixed_mass", c_int32)]
 
     @classmethod
-    def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None):
+    def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None,
+                    fixed_mass=False):
         """Params of a workload.Config; capacities default to S (no overflow possible).
-        token_budgets (per loop) selects top-k token retention with those budgets."""
+        token_budgets (per loop) selects top-k token retention with those budgets;
+        fixed_mass selects the fixed-mass form of the sparse update."""
         p = cls()
+        p.fixed_mass = 1 if fixed_mass else 0
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
         p.n_loops, p.batch = cfg.n_loops, (cfg.batch if cfg.decode else 1)
@@ -74,7 +77,7 @@ class StateC(ctypes.Structure):
                 ("n_active", c_void_p), ("q", c_void_p * 3), ("m", c_void_p * 3), ("Z", c_void_p * 3),
                 ("N", c_void_p * 3), ("colmass", c_void_p * 2), ("cols", c_void_p * MAX_LOOPS),
                 ("O", c_void_p), ("Y", c_void_p), ("rope_cs", c_void_p), ("err_word", c_void_p),
-                ("workspace", c_void_p), ("workspace_bytes", c_size_t)]
+                ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("G", c_void_p * 3)]
 
 
 class DecodeStateC(ctypes.Structure):
@@ -358,6 +361,9 @@ class FlashLoopState:
             self.t[f"N{i}"] = z((H, S, dh), torch.float32)
             c.q[i], c.m[i] = self.t[f"q{i}"].data_ptr(), self.t[f"m{i}"].data_ptr()
             c.Z[i], c.N[i] = self.t[f"Z{i}"].data_ptr(), self.t[f"N{i}"].data_ptr()
+            if params.fixed_mass:
+                self.t[f"G{i}"] = z((H, S), torch.float32)
+                c.G[i] = self.t[f"G{i}"].data_ptr()
         for i in range(2):
             self.t[f"colmass{i}"] = z((H, S), torch.float32)
             c.colmass[i] = self.t[f"colmass{i}"].data_ptr()

@@ -74,6 +74,7 @@ typedef struct flashloop_params {
   int32_t bits[FLASHLOOP_MAX_LOOPS];     /* code width per loop: bits[0] = 8 (base); 8, 4 or 2 after */
   int32_t capacity[FLASHLOOP_MAX_LOOPS]; /* rows allocated for loop r's active list and residual stream */
   int32_t gate_topk; /* 0: the tau threshold gate; else top-k token retention keeping capacity[r-1] tokens */
+  int32_t fixed_mass; /* 0: running (m, N, Z) update; else the fixed-mass form (see flashloop_sparse_attn_update) */
 } flashloop_params;
 
 /* One quantised cache (K or V) of a sequence: the loop-1 base over every
@@ -112,6 +113,8 @@ typedef struct flashloop_state {
   int32_t* err_word;                    /* device error word, 0 = no error */
   void* workspace;                      /* scratch, zero-filled once before first use */
   size_t workspace_bytes;               /* >= flashloop_workspace_bytes(params) */
+  float* G[3];                          /* [H, S] selected-column factor g, one per m/Z/N slot
+                                           (params.fixed_mass only; NULL otherwise) */
 } flashloop_state;
 
 /* ---------------------------------------------------------------- sizing */
@@ -249,7 +252,20 @@ int flashloop_selcol_dequant(const flashloop_params* p, int32_t loop, flashloop_
  * state slot sel(r) and the rows of O.  With want_colmass != 0 also writes
  * colmass[1][h, j] = sum_i e^(s_new - m') / Z' for the selected j.
  * loop == 1 runs the dense loop-1 attention (every j <= i, no removal, the
- * state starts empty) and always writes colmass[0]. */
+ * state starts empty) and always writes colmass[0].
+ *
+ * With params.fixed_mass [FlashLoop §4.2: selected-column probabilities are
+ * rescaled by their cached full-attention mass]: the selected columns J of
+ * row i keep the total probability they had after loop r-1 and share it in
+ * proportion to e^(s_new); unselected columns keep theirs.  The state gains
+ * g (G[slot], [H, S]), the weight of the selected columns relative to
+ * e^(s - m) / Z (the dense loop writes g = 1):
+ *   g' = g sum_J e^(s_old - m') / sum_J e^(s_new - m')   (g' = g when J is empty),
+ *   Z' = a Z_i,
+ *   N' = a N_i - g sum_J e^(s_old - m') Vhat_j^(r-1) + g' sum_J e^(s_new - m') Vhat_j^(r),
+ * with m' any common frame (the call picks one that keeps the scaled
+ * exponentials in fp16 range).  It runs as two launches, a statistics pass
+ * and the update; colmass[1] then sums g' e^(s_new - m') / Z'. */
 int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashloop_state* st,
                                  int32_t want_colmass, void* stream);
 

@@ -18,8 +18,8 @@ from gpu_helpers import bf16_rows, bf16_to_torch, row_rel_l2, torch_to_bf16_bits
 TOL = 1e-2
 
 
-def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None):
-    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets)
+def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None, fixed_mass=False, tau=None):
+    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets, fixed_mass=fixed_mass, tau=tau)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
@@ -322,4 +322,50 @@ def test_attention_rejects_unaligned_output():
         st.c.O = good
     torch.cuda.synchronize()
     assert np.array_equal(torch_to_bf16_bits(st["O"]), o_before)
+    assert st.error_code() == 0
+
+
+@pytest.mark.parametrize("case", ["tiny", "tiny_shrinking", "tiny_dense", "ouro_heads"])
+def test_loop_step_fixed_mass_matches_oracle(case):
+    """The fixed-mass form (selected columns keep their cached mass) against
+    the oracle's explicit per-row distributions: the tiny workload, shrinking
+    budgets (loops 3 and 4 rank the fixed-mass column mass), tau = 0 with
+    k = S (every loop is then dense attention), and the 1.4B-like shape on
+    two heads."""
+    cfg = CONFIGS["ouro14_4k"].with_(seq=1024) if case == "ouro_heads" else CONFIGS["tiny"]
+    topk, tau, heads = None, None, list(range(cfg.n_heads))
+    if case == "tiny_shrinking":
+        topk = [cfg.seq, 40, 26, 13]
+    elif case == "tiny_dense":
+        cfg = cfg.with_(seq=192, tau=0.0)
+        topk, tau = [cfg.seq] * cfg.n_loops, 0.0
+    elif case == "ouro_heads":
+        heads = [0, 9]
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    orc = O.OracleSequence(cfg, W, X, heads=heads, topk=topk, tau=tau, fixed_mass=True).run()
+    p, st, snaps = run_gpu(cfg, W, X, topk=topk, fixed_mass=True, tau=tau)
+    assert p.fixed_mass == 1
+    worst = compare(cfg, orc, snaps, st, heads, len(heads) == cfg.n_heads, topk=topk)
+    print(case, worst)
+    # the GPU's factor g reproduces the cached mass: for an active row of the last
+    # loop, the selected columns' probabilities sum to the oracle's M_i
+    R = cfg.n_loops
+    slot = st.q_slot(R)
+    G = st[f"G{slot}"].cpu().numpy()
+    m = st[f"m{slot}"].cpu().numpy()
+    Z = st[f"Z{slot}"].cpu().numpy()
+    assert np.all(np.isfinite(G)) and np.all(G[:, orc.active[R]] >= 0)
+    for a, h in enumerate(heads):
+        T = orc.T[F.flashloop_selection_loop(p, R)][a]
+        for i in orc.active[R][::17]:
+            J = T[T <= i]
+            if J.size == 0:
+                continue
+            want = orc.P[a, i, J].sum()
+            q = bf16_rows(torch_to_bf16_bits(st[f"q{slot}"])[i:i + 1]).reshape(cfg.n_heads, -1)[h]
+            Kj = orc.Kc.reconstruct(J, R)[:, a].astype(np.float64)
+            s_new = Kj @ q / np.sqrt(cfg.head_dim)
+            got = G[h, i] * np.exp(s_new - m[h, i]).sum() / Z[h, i]
+            assert abs(got - want) <= 2e-2 * want + 1e-6, (h, int(i), got, want)
     assert st.error_code() == 0
