@@ -24,8 +24,8 @@
 // <= 2^8 and represents the same (m, N, Z) state (N and Z are defined up to
 // the common factor e^m).  All waits are bounded.
 //
-// Fixed-mass form [FlashLoop §4.2 "rescales selected-column probabilities by
-// their cached full-attention mass"]: the selected columns J of row i keep
+// Fixed-mass form [FlashLoop §4.2: the selection's probabilities are scaled to
+// the mass the previous loop gave those columns]: the selected columns J of row i keep
 // the probability mass M_i they had after loop r-1 and share it in
 // proportion to e^(s_new).  With a per-row factor g (the weight of the
 // selected columns relative to e^(s - m) / Z; g = 1 after the dense loop)

@@ -134,7 +134,7 @@ int flashloop_rope_table(const flashloop_params* p, int32_t n_pos, float* cs, vo
 
 /* ---------------------------------------------------------------- the path */
 
-/* (a1, top-k retention) [FlashLoop §4.1 "top-k tokens retained", App. D.1]:
+/* (a1, top-k retention) [FlashLoop §4.1 and App. D.1: a budget of tokens kept per loop]:
  * instead of the tau threshold, keep the `budget` candidates of largest
  * normalised change ||x_cur - x_prev||^2 / ||x_prev||^2 (float32 sums, IEEE
  * division; a zero previous row counts as +inf if it changed, 0 if not),
@@ -254,8 +254,8 @@ int flashloop_selcol_dequant(const flashloop_params* p, int32_t loop, flashloop_
  * loop == 1 runs the dense loop-1 attention (every j <= i, no removal, the
  * state starts empty) and always writes colmass[0].
  *
- * With params.fixed_mass [FlashLoop §4.2: selected-column probabilities are
- * rescaled by their cached full-attention mass]: the selected columns J of
+ * With params.fixed_mass [FlashLoop §4.2: the selection's probabilities are
+ * scaled to the mass the previous loop gave those columns]: the selected columns J of
  * row i keep the total probability they had after loop r-1 and share it in
  * proportion to e^(s_new); unselected columns keep theirs.  The state gains
  * g (G[slot], [H, S]), the weight of the selected columns relative to

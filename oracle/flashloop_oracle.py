@@ -515,7 +515,7 @@ class OracleSequence:
 
     def run_loop1(self):
         """Dense loop: every token, INT8 base, dense causal attention on the
-        reconstructed base, column mass c^(1) [FL App. D.1 "dense early loops"]."""
+        reconstructed base, column mass c^(1) [FL App. D.1: the early loops run dense]."""
         S, dh = self.S, self.dh
         rows = np.arange(S)
         self.active[1] = rows
@@ -593,7 +593,7 @@ class OracleSequence:
 
 
 # --------------------------------------------------------------------------
-# decode: one new token per sequence  [FL App. G "fused sparse decode selection"]
+# decode: one new token per sequence  [FL App. G: the decode selection is fused with the decode pass]
 # --------------------------------------------------------------------------
 class OracleDecode:
     """One decode token at position p = S_ctx against a context whose KV path
