@@ -146,7 +146,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     xs = [to_dev(x) for x in X]
     wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
-    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass)
+    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass, attn_pairs=args.sm_pairs)
     st = F.FlashLoopState(p, device=dev)
     S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
@@ -231,9 +231,11 @@ def run_cuda(args, cfg, rank, world, local_rank):
     achieved = flop2 / (ms2 * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": None if args.fixed_mass else ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
+                "traffic": None if (args.fixed_mass or args.sm_pairs) else ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
                 "kernel": ("attn_tc_kernel<128> statistics + update passes, loop 2 (fixed-mass form, tcgen05)"
                            if args.fixed_mass else
+                           "attn_pair_kernel<128>, loop-2 launch (sparse attention update, tcgen05 on SM pairs)"
+                           if args.sm_pairs else
                            "attn_tc_kernel<128>, loop-2 launch (sparse attention update, tcgen05)"),
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
@@ -312,7 +314,8 @@ def run_cuda(args, cfg, rank, world, local_rank):
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded workload generator; random-init weights of the stated shape)",
-        "config": {"workload": workload_desc(cfg) + (", fixed-mass form of the update" if args.fixed_mass else ""),
+        "config": {"workload": workload_desc(cfg) + (", fixed-mass form of the update" if args.fixed_mass else "")
+                   + (", attention on SM pairs" if args.sm_pairs else ""),
                    "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
                    "parallelism": f"one sequence per GPU, {world} GPU(s), no exchange",
                    "active_tokens": {f"loop{r}": int(st['n_active'][r - 1].item()) for r in range(2, R + 1)},
@@ -626,6 +629,8 @@ def main():
     ap.add_argument("--fixed-mass", action="store_true",
                     help="prefill workloads: the fixed-mass form of the sparse update (no CPU baseline: its "
                          "oracle keeps explicit S x S distributions)")
+    ap.add_argument("--sm-pairs", action="store_true",
+                    help="prefill workloads: the running update on SM pairs (cta_group::2)")
     ap.add_argument("--batch", type=int, default=None,
                     help="decode workloads: sequences per GPU (a smaller case for profiler captures)")
     args = ap.parse_args()

@@ -933,8 +933,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 at_encode_fn() {
 // 3-D fp16 tensor map: dims (innermost first) d0 x d1 x d2, row pitch p1 and
 // plane pitch p2 in elements, box b0 x b1 x 1, 128-byte swizzle.  Coordinates
 // past d1 read as zero.
-static int make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
-                            uint64_t p1, uint64_t p2, uint32_t b0, uint32_t b1) {
+int make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uint64_t d1, uint64_t d2,
+                     uint64_t p1, uint64_t p2, uint32_t b0, uint32_t b1) {
   auto fn = at_encode_fn();
   if (fn == nullptr) return FLASHLOOP_ERR_CUDA;
   if ((reinterpret_cast<uintptr_t>(base) & 15) != 0 || (p1 * 2) % 16 != 0 || (p2 * 2) % 16 != 0)
@@ -949,7 +949,7 @@ static int make_tmap_f16_3d(CUtensorMap* map, const void* base, uint64_t d0, uin
   return r == CUDA_SUCCESS ? FLASHLOOP_OK : FLASHLOOP_ERR_CUDA;
 }
 
-static int at_sm_count() {
+int at_sm_count() {
   static int cached[128];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
@@ -999,8 +999,16 @@ int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scr
 }
 
 // K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.
+int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream);
+
 int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
+  if (a.mode == kAtRunning && p->attn_pairs) {
+    // the running update on SM pairs (half of every K / V tile per SM), where
+    // the device can co-schedule them
+    const int rc = launch_attn_pair(p, a, kcp, stream);
+    if (rc != FLASHLOOP_ERR_UNSUPPORTED) return rc;
+  }
   // the row warps move q, N and O rows in 32-byte accesses
   const void* aligned32[] = {a.q_new, a.q_old, a.n_in, a.n_out, a.o};
   for (const void* ptr : aligned32)

@@ -40,16 +40,19 @@ class Params(ctypes.Structure):
     _fields_ = [("seq", c_int32), ("d_model", c_int32), ("n_heads", c_int32), ("head_dim", c_int32),
                 ("n_loops", c_int32), ("batch", c_int32), ("tau", c_float), ("rope_theta", c_float),
                 ("topk", c_int32 * MAX_LOOPS), ("bits", c_int32 * MAX_LOOPS),
-                ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32), ("fixed_mass", c_int32)]
+                ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32), ("fixed_mass", c_int32),
+                ("attn_pairs", c_int32)]
 
     @classmethod
     def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None,
-                    fixed_mass=False):
+                    fixed_mass=False, attn_pairs=False):
         """Params of a workload.Config; capacities default to S (no overflow possible).
         token_budgets (per loop) selects top-k token retention with those budgets;
-        fixed_mass selects the fixed-mass form of the sparse update."""
+        fixed_mass selects the fixed-mass form of the sparse update; attn_pairs runs
+        the running update on SM pairs."""
         p = cls()
         p.fixed_mass = 1 if fixed_mass else 0
+        p.attn_pairs = 1 if attn_pairs else 0
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
         p.n_loops, p.batch = cfg.n_loops, (cfg.batch if cfg.decode else 1)

@@ -18,8 +18,9 @@ from gpu_helpers import bf16_rows, bf16_to_torch, row_rel_l2, torch_to_bf16_bits
 TOL = 1e-2
 
 
-def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None, fixed_mass=False, tau=None):
-    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets, fixed_mass=fixed_mass, tau=tau)
+def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None, fixed_mass=False, tau=None, attn_pairs=False):
+    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets, fixed_mass=fixed_mass, tau=tau,
+                             attn_pairs=attn_pairs)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
@@ -369,3 +370,17 @@ def test_loop_step_fixed_mass_matches_oracle(case):
             got = G[h, i] * np.exp(s_new - m[h, i]).sum() / Z[h, i]
             assert abs(got - want) <= 2e-2 * want + 1e-6, (h, int(i), got, want)
     assert st.error_code() == 0
+
+
+@pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
+def test_loop_step_on_sm_pairs_matches_oracle(name):
+    """The running update on SM pairs (two CTAs share every K / V tile, each
+    loading half; cta_group::2 MMAs over 256 rows), loop 1 included."""
+    cfg = CONFIGS[name]
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    orc = O.OracleSequence(cfg, W, X).run()
+    p, st, snaps = run_gpu(cfg, W, X, attn_pairs=True)
+    assert p.attn_pairs == 1
+    worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True)
+    print(name, "pairs", worst)
