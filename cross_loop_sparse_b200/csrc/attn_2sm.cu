@@ -12,8 +12,8 @@
 // thread of CTA 0 issues M = 256 MMAs that read A (Q, then P) from both CTAs'
 // TMEM and B from both CTAs' shared memory and write both CTAs' TMEM.
 // Loads land in the loading CTA's shared memory and count on CTA 0's
-// barrier (cta_group::2 bulk tensor loads, no multicast); tcgen05.commit
-// signals the barrier of both CTAs.  Row warps of CTA 1 report to CTA 0
+// barrier (cta_group::2 bulk tensor loads, no multicast); a tcgen05.commit
+// to each CTA's barrier signals both.  Row warps of CTA 1 report to CTA 0
 // with remote mbarrier arrivals.  All waits are bounded.
 #include <cuda.h>
 #include <cudaTypedefs.h>
@@ -86,12 +86,13 @@ __device__ __forceinline__ void umma_f16_ts_pair(uint32_t d_tmem, uint32_t a_tme
       ::"r"(d_tmem), "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(0u), "r"(0u), "r"(0u), "r"(0u),
       "r"(0u), "r"(0u), "r"(0u), "r"(0u));
 }
-// Arrive on the barrier at this offset in both CTAs once the issued MMAs complete.
+// Arrive on the barrier at this offset in both CTAs once the issued MMAs
+// complete: one commit per CTA, the second addressed to the peer's copy.
 __device__ __forceinline__ void umma_commit_pair(uint64_t* bar) {
-  asm volatile(
-      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;\n"
-      ::"r"(smem_u32(bar)), "h"((uint16_t)3)
-      : "memory");
+  const uint32_t own = smem_u32(bar);
+  const uint32_t peer = mapa_shared(own, 1);
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(own) : "memory");
+  asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];\n" ::"r"(peer) : "memory");
 }
 // 3-D tile load into this CTA's shared memory, bytes counted on `bar_cluster`
 // (a barrier of either CTA of the pair).
