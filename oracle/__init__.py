@@ -11,6 +11,9 @@ from .flashloop_oracle import (  # noqa: F401
     KVStream,
     OracleDecode,
     OracleSequence,
+    PAPER_GROUP,
+    PAPER_TAIL,
+    PaperKVStream,
     apply_rope,
     cache_bytes,
     dense_causal_attention,
@@ -23,8 +26,11 @@ from .flashloop_oracle import (  # noqa: F401
     gate_norms,
     gate_topk,
     out_projection,
+    paper_cache_bytes,
     pack_codes,
     project_qkv,
+    quantize_asym,
+    dequantize_asym,
     quantize_groups,
     rope_angles,
     sparse_update,

@@ -44,6 +44,11 @@ supports):
      previous loop's full distribution; within J the mass is shared in
      proportion to e^(s_new).  Unselected columns keep their probabilities,
      so every row's distribution still sums to one [FL §4.2, D.2; FZ §3].
+  R11 the pages' own cache setting (an option): INT4 asymmetric groups of
+     64 with an fp16 scale and an fp16 minimum, keys grouped per channel over
+     64 tokens (residual keys over 64 entries of the loop's active list),
+     values per token over 64 channels, the last 64 tokens in bf16 at every
+     loop [FL App. E; FZ §3].
 
 Parity unpinned: nothing in this module is without a pin; the accuracy and
 reconstruction figures the paper reports on real models are out of reach
@@ -294,6 +299,174 @@ class KVStream:
 
 
 # --------------------------------------------------------------------------
+# (f2) the pages' own cache setting  [FL App. E "Quantization Setting"; FZ §3]
+# --------------------------------------------------------------------------
+PAPER_GROUP = 64
+PAPER_TAIL = 64
+PAPER_LEVELS = 15          # INT4 asymmetric: codes 0..15
+
+
+def quantize_asym(g32):
+    """Asymmetric INT4 quantisation of float32 groups along the last axis
+    (reading R11).  Per group: lo = fp16(min), s = fp16((max - min) / 15),
+    code = clamp(rint((x - lo) / s), 0, 15) in float32 with IEEE division and
+    round-half-even; s = 0 gives code 0.  Returns (codes uint8, s fp16, lo fp16)."""
+    g32 = np.asarray(g32, dtype=np.float32)
+    mn = np.min(g32, axis=-1)
+    mx = np.max(g32, axis=-1)
+    with np.errstate(over="ignore"):
+        lo16 = mn.astype(np.float16)
+        s16 = ((mx - mn) / np.float32(PAPER_LEVELS)).astype(np.float16)
+    s32 = s16.astype(np.float32)[..., None]
+    q = np.zeros_like(g32)
+    np.divide(g32 - lo16.astype(np.float32)[..., None], s32, out=q, where=np.broadcast_to(s32 > 0, g32.shape))
+    codes = np.clip(np.rint(q), 0, PAPER_LEVELS).astype(np.uint8)
+    return codes, s16, lo16
+
+
+def dequantize_asym(codes, s16, lo16):
+    """code * s + lo in float32."""
+    return (np.asarray(codes).astype(np.float32) * s16.astype(np.float32)[..., None]
+            + lo16.astype(np.float32)[..., None])
+
+
+class PaperKVStream:
+    """One of K or V in the pages' own setting (reading R11): an INT4
+    asymmetric base over the tokens before the last 64, groups of 64 along
+    the token axis per channel for keys and along the channels per token for
+    values, residuals of later loops in the same format for the active
+    tokens (key groups run over 64 consecutive entries of the loop's active
+    list), and the last 64 tokens kept in bf16 at every loop they are active.
+    Same interface as KVStream."""
+
+    def __init__(self, tokens, heads, head_dim, kind, tail=PAPER_TAIL, group=PAPER_GROUP):
+        assert kind in ("k", "v") and head_dim % group == 0
+        self.T, self.H, self.dh = tokens, heads, head_dim
+        self.kind, self.tail, self.group = kind, min(tail, tokens), group
+        self.body = tokens - self.tail       # tokens [0, body) are quantised
+        self.base = None                     # (codes, s, lo) of the body
+        self.res = {}                        # loop -> (codes, s, lo, n) of the active body tokens
+        self.tail_vals = {}                  # loop -> (tokens, bf16 bits [n, H, dh]) of the active tail tokens
+        self.slot = {}                       # loop -> int64 [tokens], -1 when absent (body tokens only)
+        self.active = {}                     # loop -> ascending active tokens
+
+    # -- group layout ---------------------------------------------------------
+    def _quant(self, x):
+        """x float32 [n, H, dh] -> quantised groups (codes, s, lo, n)."""
+        n = x.shape[0]
+        G = self.group
+        if self.kind == "v":                       # per token: groups of G channels
+            g = x.reshape(n, self.H, self.dh // G, G)
+            return quantize_asym(g) + (n,)
+        pad = (-n) % G                              # per channel: groups of G rows
+        xp = np.concatenate([x, np.repeat(x[-1:], pad, axis=0)]) if pad and n else x
+        g = xp.reshape(-1, G, self.H, self.dh).transpose(0, 2, 3, 1)   # [groups, H, dh, G]
+        codes, s16, lo16 = quantize_asym(g)
+        return codes, s16, lo16, n
+
+    def _deq(self, item, rows):
+        codes, s16, lo16, n = item
+        rows = np.asarray(rows, dtype=np.int64)
+        if self.kind == "v":
+            return dequantize_asym(codes[rows], s16[rows], lo16[rows]).reshape(rows.size, self.H, self.dh)
+        G = self.group
+        grp, off = rows // G, rows % G
+        full = dequantize_asym(codes[grp], s16[grp], lo16[grp])          # [r, H, dh, G]
+        return np.take_along_axis(full, off[:, None, None, None], axis=3)[..., 0]
+
+    # -- loop 1 ---------------------------------------------------------------
+    def write_base(self, x):
+        x = np.asarray(x)
+        self.base = self._quant(x[: self.body].astype(np.float32))
+        toks = np.arange(self.body, self.T)
+        self.tail_vals[1] = (toks, to_bf16_bits(x[self.body:]))
+        self.active[1] = np.arange(self.T)
+
+    def _tail_value(self, tok, loop):
+        for l in range(loop, 0, -1):
+            if l in self.tail_vals:
+                toks, bits = self.tail_vals[l]
+                i = np.searchsorted(toks, tok)
+                if i < toks.size and toks[i] == tok:
+                    return bf16_vals(bits[i])
+        raise KeyError(tok)
+
+    # -- reconstruction -------------------------------------------------------
+    def reconstruct(self, tokens, loop):
+        """Xhat^(loop): for body tokens the base plus every residual of loops
+        2..loop where the token was active (float32, loop order); for tail
+        tokens the bf16 value of the latest loop <= `loop` that stored one."""
+        tokens = np.asarray(tokens, dtype=np.int64)
+        out = np.zeros((tokens.size, self.H, self.dh), dtype=np.float64)
+        body = tokens < self.body
+        if np.any(body):
+            bt = tokens[body]
+            acc = self._deq(self.base, bt)
+            for l in range(2, loop + 1):
+                if l not in self.slot:
+                    continue
+                sl = self.slot[l][bt]
+                have = sl >= 0
+                if np.any(have):
+                    add = np.zeros_like(acc)
+                    add[have] = self._deq(self.res[l], sl[have])
+                    acc = acc + add
+            out[body] = acc
+        for i in np.nonzero(~body)[0]:
+            out[i] = self._tail_value(int(tokens[i]), loop)
+        return out
+
+    # -- loops r >= 2 ---------------------------------------------------------
+    def write_residual(self, loop, tokens, x):
+        """Body tokens store the quantised x - Xhat^(loop-1); tail tokens store
+        x in bf16.  ``tokens`` ascending, x [n, H, dh]."""
+        tokens = np.asarray(tokens, dtype=np.int64)
+        x = np.asarray(x)
+        body = tokens < self.body
+        bt = tokens[body]
+        rho = x[body].astype(np.float32) - self.reconstruct(bt, loop - 1).astype(np.float32)
+        self.res[loop] = self._quant(rho)
+        slot = np.full(self.T, -1, dtype=np.int64)
+        slot[bt] = np.arange(bt.size)
+        self.slot[loop] = slot
+        self.tail_vals[loop] = (tokens[~body], to_bf16_bits(x[~body]))
+        self.active[loop] = tokens
+
+    def stored_bytes(self):
+        """Bytes of everything stored: 4-bit codes, an fp16 scale and an fp16
+        minimum per group, bf16 tail values."""
+        def q_bytes(item):
+            codes, s16, lo16, n = item
+            if self.kind == "v":
+                elems = n * self.H * self.dh
+            else:   # the padding rows of a partial key group store no codes
+                elems = n * self.H * self.dh
+            return elems // 2 + 2 * s16.size + 2 * lo16.size
+        total = q_bytes(self.base)
+        for item in self.res.values():
+            total += q_bytes(item)
+        for toks, _ in self.tail_vals.values():
+            total += toks.size * self.H * self.dh * 2
+        return total
+
+
+def paper_cache_bytes(S, n_heads, head_dim, body_active, tail_active, tail=PAPER_TAIL, group=PAPER_GROUP):
+    """Bytes of K and V in the pages' own setting (reading R11), by formula:
+    the body's 4-bit codes plus 4 bytes (fp16 scale and minimum) per group of
+    64, and 2 bytes per element of the bf16 tail at every loop it is stored.
+    ``body_active[l]`` / ``tail_active[l]`` = active body / tail tokens of loop
+    l+1 (index 0: loop 1, every token)."""
+    E = n_heads * head_dim
+    total = 0
+    for l, (nb, nt) in enumerate(zip(body_active, tail_active)):
+        codes = 2 * nb * E // 2
+        v_groups = nb * E // group
+        k_groups = -(-nb // group) * E
+        total += codes + 4 * (v_groups + k_groups) + 2 * nt * E * 2
+    return total
+
+
+# --------------------------------------------------------------------------
 # (a4) column selection  [FL §3.2, §4.2, App. D.2; FZ §3; reading R8]
 # --------------------------------------------------------------------------
 def topk_columns(mass32, candidates, k):
@@ -451,11 +624,13 @@ class OracleSequence:
     """
 
     def __init__(self, cfg, W, X, heads=None, quantize=True, topk=None, tau=None,
-                 keep_history=True, token_budgets=None, fixed_mass=False):
+                 keep_history=True, token_budgets=None, fixed_mass=False, kv_scheme="spec"):
         """``token_budgets`` (per loop, index r-1) switches the gate from the
         tau threshold to top-k token retention with those budgets.
         ``fixed_mass`` runs loops >= 2 in the fixed-mass form (reading R10)
-        on explicit [S, S] distributions per head (small S only)."""
+        on explicit [S, S] distributions per head (small S only).
+        ``kv_scheme="paper"`` stores K and V in the pages' own setting
+        (reading R11) instead of the INT8 + INT4/INT2 symmetric streams."""
         self.cfg = cfg
         self.fixed_mass = fixed_mass
         self.P = None          # fixed-mass form: head -> [S, S] probabilities
@@ -471,8 +646,12 @@ class OracleSequence:
         self.kbud = list(cfg.k_per_loop() if topk is None else topk)
         self.keep = keep_history
         Hs = len(self.heads)
-        self.Kc = KVStream(self.S, Hs, self.dh, cfg.bits, quantize)
-        self.Vc = KVStream(self.S, Hs, self.dh, cfg.bits, quantize)
+        if kv_scheme == "paper":
+            self.Kc = PaperKVStream(self.S, Hs, self.dh, "k")
+            self.Vc = PaperKVStream(self.S, Hs, self.dh, "v")
+        else:
+            self.Kc = KVStream(self.S, Hs, self.dh, cfg.bits, quantize)
+            self.Vc = KVStream(self.S, Hs, self.dh, cfg.bits, quantize)
         self.active = {}
         self.q = {}            # loop -> bf16 bits [S, Hs, dh] (rows active at that loop set)
         self.k_exact = {}      # loop -> float64 [n, Hs, dh] of the active rows

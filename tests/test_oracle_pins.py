@@ -586,3 +586,149 @@ def test_fixed_mass_unchanged_inputs_leave_output_unchanged():
     run = O.OracleSequence(cfg, W, Xs, tau=0.0, quantize=False, fixed_mass=True).run()
     for r in range(2, cfg.n_loops + 1):
         assert np.array_equal(run.O_hist[r], run.O_hist[1])
+
+
+# ---------------------------------------------------------------------------
+# the pages' own cache setting (reading R11) [FL App. E; FZ §3]
+# ---------------------------------------------------------------------------
+def _asym_bound(g):
+    """Per-element error bound of quantize_asym on float32 groups g [..., G]:
+    half a step inside the grid, plus what the fp16 rounding of the minimum
+    and of the step moves the grid's ends."""
+    g = np.asarray(g, dtype=np.float32)
+    mn = g.min(axis=-1).astype(np.float64)
+    mx = g.max(axis=-1).astype(np.float64)
+    s_exact = (mx - mn) / 15.0
+    lo16 = mn.astype(np.float16).astype(np.float64)
+    s16 = ((g.max(axis=-1) - g.min(axis=-1)) / np.float32(15)).astype(np.float16).astype(np.float64)
+    return (s16 / 2 + np.abs(lo16 - mn) + 15 * np.abs(s16 - s_exact))[..., None] * (1 + 1e-6) + 1e-30
+
+
+def test_asym_quantiser_round_trip_bound_and_grid():
+    rng = np.random.default_rng(11)
+    g = (rng.standard_normal((512, 64)) * np.exp(rng.uniform(-6, 4, (512, 1)))
+         + rng.uniform(-5, 5, (512, 1))).astype(np.float32)
+    codes, s16, lo16 = O.quantize_asym(g)
+    assert codes.dtype == np.uint8 and codes.max() <= 15
+    err = np.abs(O.dequantize_asym(codes, s16, lo16).astype(np.float64) - g.astype(np.float64))
+    assert np.all(err <= _asym_bound(g))
+    # values on an fp16-exact grid come back exactly, the ends included
+    lo, st = np.float16(-1.25), np.float16(0.1875)
+    c = rng.integers(0, 16, size=(64, 64))
+    c[:, 0], c[:, 1] = 0, 15
+    x = (c * np.float32(st) + np.float32(lo)).astype(np.float32)
+    codes, s16, lo16 = O.quantize_asym(x)
+    assert np.all(s16 == st) and np.all(lo16 == lo)
+    assert np.array_equal(codes, c.astype(np.uint8))
+    assert np.array_equal(O.dequantize_asym(codes, s16, lo16), x)
+    # an exact half step rounds to the even code; a constant group has step 0
+    h = np.array([[0.0, 1.5, 2.5, 15.0]], np.float32)
+    codes, s16, _ = O.quantize_asym(h)
+    assert s16[0] == 1 and list(codes[0]) == [0, 2, 2, 15]
+    codes, s16, lo16 = O.quantize_asym(np.full((1, 64), 3.3, np.float32))
+    assert s16[0] == 0 and not codes.any() and lo16[0] == np.float16(3.3)
+
+
+def test_paper_stream_group_layout_and_tail():
+    """Keys are grouped per channel over 64 tokens, values per token over 64
+    channels; the last 64 tokens come back as their bf16 values."""
+    rng = np.random.default_rng(3)
+    S, H, dh = 256, 2, 128
+    scale = np.arange(1, dh + 1, dtype=np.float64)            # channel d spans ~(d+1)
+    x = rng.uniform(-1, 1, (S, H, dh)) * scale
+    K = O.PaperKVStream(S, H, dh, "k")
+    V = O.PaperKVStream(S, H, dh, "v")
+    K.write_base(x)
+    V.write_base(x)
+    _, ks, _, kn = K.base
+    _, vs, _, vn = V.base
+    assert kn == vn == S - O.PAPER_TAIL
+    assert ks.shape == ((S - 64) // 64, H, dh) and vs.shape == (S - 64, H, dh // 64)
+    # a key group's step follows its own channel's range, not the token's
+    ratio = ks.astype(np.float64)[..., -1] / ks.astype(np.float64)[..., 0]
+    assert np.all(ratio > 20)
+    toks = np.arange(S - 64, S)
+    for st in (K, V):
+        got = st.reconstruct(toks, 1)
+        assert np.array_equal(got, O.flashloop_oracle.bf16_vals(O.flashloop_oracle.to_bf16_bits(x[S - 64:])))
+        body = np.arange(S - 64)
+        _, s16, _, _ = st.base
+        err = np.abs(st.reconstruct(body, 1) - x[: S - 64].astype(np.float32))
+        assert err.max() <= s16.astype(np.float64).max() * 0.51 + 1e-6
+
+
+def test_paper_stream_residuals_telescope_and_bytes():
+    """A residual re-encodes x - Xhat^(r-1): the loop-r reconstruction of an
+    active body token is within the loop-r quantiser's error of x, inactive
+    tokens keep theirs, and the bytes stored equal the closed form."""
+    cfg = CONFIGS["tiny"]
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    run = O.OracleSequence(cfg, W, X, kv_scheme="paper").run()
+    S, H, dh = cfg.seq, cfg.n_heads, cfg.head_dim
+    body_n, tail_n = [S - 64], [64]
+    for r in range(2, cfg.n_loops + 1):
+        act = run.active[r]
+        body, tail = act[act < S - 64], act[act >= S - 64]
+        body_n.append(body.size)
+        tail_n.append(tail.size)
+        for st, exact in ((run.Kc, run.k_exact[r]), (run.Vc, run.v_exact[r])):
+            x32 = exact.astype(np.float32)
+            rec = st.reconstruct(act, r)
+            inb = act < S - 64
+            _, s16, lo16, _ = st.res[r]
+            err = np.abs(rec[inb] - x32[inb])
+            assert err.max() <= s16.astype(np.float64).max() * 0.51 + 1e-5, (r, st.kind)
+            # tail tokens: exactly the bf16 value of this loop
+            tb = O.flashloop_oracle.bf16_vals(O.flashloop_oracle.to_bf16_bits(exact[~inb]))
+            assert np.array_equal(rec[~inb], tb)
+        # a token not active at r keeps its loop r-1 reconstruction
+        gone = np.setdiff1d(run.active[r - 1], act)
+        if gone.size:
+            assert np.array_equal(run.Kc.reconstruct(gone, r), run.Kc.reconstruct(gone, r - 1))
+    stored = run.Kc.stored_bytes() + run.Vc.stored_bytes()
+    assert stored == O.paper_cache_bytes(S, H, dh, body_n, tail_n)
+
+
+def test_paper_setting_bytes_against_page_cell3_model():
+    """Against the first-order model of [FZ §3, Cell 3] (codes only, no group
+    metadata, the tail counted once) at the pages' 32K schedule: the fp16
+    scale and minimum of every 64-element group add one eighth of the code
+    bytes (a little more where a residual key list ends in a partial group),
+    and the bf16 tail costs what it does per loop it is stored."""
+    S, H, dh = 32768, 16, 128
+    fracs = [0.2, 0.08]          # two dense loops, then 20% and 8% of the tokens
+    E = 2 * H * dh               # K and V elements per token and loop
+    body = [S - 64, S - 64] + [round(f * (S - 64)) for f in fracs]
+    tail = [64, 64] + [round(f * 64) for f in fracs]
+    stored = O.paper_cache_bytes(S, H, dh, body, tail)
+    codes = sum(b * E // 2 for b in body)
+    tails = sum(t * E * 2 for t in tail)
+    meta = stored - codes - tails
+    assert codes / 8 <= meta <= codes / 8 * 1.01
+    base, res, tl = O.first_order_storage(S, E, 4, 4, [1.0] + fracs, 64)
+    model = base + res + tl
+    # the model's codes span all S tokens of each loop (fractional counts);
+    # ours stop before the tail (whole tokens: at most one token apart per loop)
+    assert abs(base + res - codes - sum(t * E // 2 for t in tail)) <= len(fracs) * E // 2
+    assert 1.12 < stored / model < 1.16
+
+
+def test_paper_setting_full_budget_zero_threshold_is_dense_attention():
+    """The update's algebra does not depend on the cache format: with tau = 0
+    and k = S each loop's output is dense attention over the loop's
+    reconstructed keys and values in the pages' setting too."""
+    cfg = CONFIGS["tiny"].with_(seq=192)
+    W = make_weights(cfg)
+    X, _ = make_hidden_states(cfg)
+    S, H = cfg.seq, cfg.n_heads
+    run = O.OracleSequence(cfg, W, X, tau=0.0, topk=[S] * cfg.n_loops, kv_scheme="paper").run()
+    rows = np.arange(S)
+    for r in range(1, cfg.n_loops + 1):
+        K = run.Kc.reconstruct(rows, r)
+        V = run.Vc.reconstruct(rows, r)
+        m, Z, N = run.hist[r]
+        for h in range(H):
+            q = bf16_bits_to_f32(run.q[r][:, h, :]).astype(np.float64)
+            want, _ = _textbook(q, K[:, h], V[:, h], rows)
+            assert np.allclose(N[h] / Z[h][:, None], want, rtol=1e-9, atol=1e-12), (r, h)
