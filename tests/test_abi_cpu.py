@@ -40,6 +40,8 @@ int main(void) {
          offsetof(flashloop_state, workspace_bytes));
   printf("%zu %zu %zu\n", offsetof(flashloop_state, cols), offsetof(flashloop_state, rope_cs),
          offsetof(flashloop_state, colmass));
+  printf("%zu %zu %zu %zu\n", offsetof(flashloop_params, gate_topk), offsetof(flashloop_params, fixed_mass),
+         offsetof(flashloop_params, attn_pairs), offsetof(flashloop_state, G));
   return 0;
 }
 '''
@@ -53,7 +55,9 @@ int main(void) {
     want = [ctypes.sizeof(F.Params), ctypes.sizeof(F.KV), ctypes.sizeof(F.StateC),
             F.Params.tau.offset, F.Params.topk.offset, F.Params.capacity.offset,
             F.StateC.n_active.offset, F.StateC.workspace_bytes.offset,
-            F.StateC.cols.offset, F.StateC.rope_cs.offset, F.StateC.colmass.offset]
+            F.StateC.cols.offset, F.StateC.rope_cs.offset, F.StateC.colmass.offset,
+            F.Params.gate_topk.offset, F.Params.fixed_mass.offset, F.Params.attn_pairs.offset,
+            F.StateC.G.offset]
     assert got == want
 
 
@@ -106,3 +110,13 @@ def test_host_checks_reject_bad_params():
     p = F.Params.from_config(cfg); p.n_loops = 17
     assert _status(p) == -1
     assert F.flashloop_status_string(-2).startswith("unsupported")
+
+
+def test_decode_refuses_the_fixed_mass_form():
+    """Decode keeps the running (m, N, Z) form: its sizing helper reports the
+    fixed-mass parameters as unsupported (0 bytes) before any device query."""
+    cfg = CONFIGS["decode_32k"]
+    p = F.Params.from_config(cfg)
+    assert F._lib.flashloop_decode_workspace_bytes(ctypes.byref(p)) > 0
+    p = F.Params.from_config(cfg, fixed_mass=True)
+    assert F._lib.flashloop_decode_workspace_bytes(ctypes.byref(p)) == 0
