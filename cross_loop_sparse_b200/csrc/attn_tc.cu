@@ -15,18 +15,19 @@
 // TMEM (512 columns): Q_new | Q_old (fp16 pairs), N (f32, DH columns), two
 // score buffers {S_new 64 | S_old 64}; P = [e_new | -e_old] (fp16 pairs) is
 // written over the S_new half of its buffer and fed to the P.V MMA from TMEM.
-// Roles: warps 0-3 own one row each (TMEM lane) and do the masking,
-// exponentials, running max and sums, the Q / N set-up and the write-back;
-// warp 4 allocates TMEM and streams K (64 x DH) and V^T (DH x 64) tiles by TMA;
-// warp 5 issues S(t+1) while the rows process S(t), then P(t).V.
+// Roles: warps 0-7 hold two threads per row (TMEM lane), one per half of a
+// tile, and do the masking, exponentials, running max and sums, the Q / N
+// set-up and the write-back; warp 8 allocates TMEM and streams K (64 x DH)
+// and V^T (DH x 64) tiles, new and old, by TMA into a ring of three stages;
+// warp 9 issues S(t+1) while the rows process S(t), then P(t).V.
 // The running maximum is a per-row reference raised only when a tile's
 // maximum exceeds it by 8 (log2 units), which keeps every exponential
 // <= 2^8 and represents the same (m, N, Z) state (N and Z are defined up to
 // the common factor e^m).  All waits are bounded.
 //
-// Fixed-mass form [FlashLoop §4.2: the selection's probabilities are scaled to
-// the mass the previous loop gave those columns]: the selected columns J of row i keep
-// the probability mass M_i they had after loop r-1 and share it in
+// Fixed-mass form [FlashLoop §4.2: the selection's probabilities are scaled
+// to the mass the previous loop gave those columns]: the selected columns J of
+// row i keep the probability mass M_i they had after loop r-1 and share it in
 // proportion to e^(s_new).  With a per-row factor g (the weight of the
 // selected columns relative to e^(s - m) / Z; g = 1 after the dense loop)
 // that is N' = a N - g_prev sum_J e^(s_old - m') V_old + g sum_J e^(s_new - m') V_new,
