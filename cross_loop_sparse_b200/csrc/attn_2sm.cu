@@ -580,6 +580,454 @@ attn_pair_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constan
   }
 }
 
+
+constexpr int k4Threads = 576, k4TmaWarp = 16, k4MmaWarp = 17;  // 16 row warps (four threads per row)
+template <int DH>
+constexpr int a4_smem() { return 1024 + k2Stages * A2Cfg<DH>::kStageBytes + 512 + 12 * 128 * 4; }
+
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};\n"
+               ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
+}
+
+template <int DH>
+__global__ void __launch_bounds__(k4Threads, 1)
+attn_pair4_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
+                 const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_vo, A2Args g) {
+  using C = A2Cfg<DH>;
+  constexpr int kSmemXchg = 512;  // offset of the row exchange after the barriers
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + k2Stages * C::kStageBytes);
+  uint64_t* kv_full = bars;                    // [stages] (CTA 0's count both CTAs' bytes)
+  uint64_t* kv_empty = bars + k2Stages;        // [stages]
+  uint64_t* s_full = bars + 2 * k2Stages;      // [2]
+  uint64_t* p_full = s_full + 2;               // [2]  (CTA 0: one arrival per row warp of the pair)
+  uint64_t* pv_done = p_full + 2;              // [2]
+  uint64_t* q_ready = pv_done + 2;             // [1]  (CTA 0: one arrival per row warp of the pair)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xchg = reinterpret_cast<float*>(smem + k2Stages * C::kStageBytes + kSmemXchg);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool has_old = !g.dense;
+  int n_rows = g.n_rows ? *g.n_rows : g.S;
+  if (n_rows > g.row_cap) n_rows = g.row_cap;
+  if (n_rows < 0) n_rows = 0;
+  const int row_tiles = (n_rows + k2Rows - 1) / k2Rows;
+  const int pairs = (row_tiles + 1) / 2;
+  const int total = pairs * g.H;
+  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < k2Stages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], 32);
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(q_ready, 32);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == k4TmaWarp) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync_all();  // barriers of both CTAs exist before any remote arrival or load
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == k4TmaWarp) {
+    // ------------------------------------------------------------ TMA loads (both CTAs)
+    if (lane == 0) {
+      const uint32_t half_bytes = (has_old ? 2 : 1) * (C::kKHalf + C::kVHalf);
+      const uint32_t full_bar0 = mapa_shared(smem_u32(kv_full), 0);
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued[k2Stages];
+      for (int s2 = 0; s2 < k2Stages; ++s2) issued[s2] = -1;
+      for (int item = cluster; item < total && !*abort_flag; item += n_clusters) {
+        const int h = item / pairs, rp = item % pairs;
+        const int nt = a2_tiles(g, h, rp, n_rows);
+        for (int t = 0; t < nt && !*abort_flag; ++t) {
+          if (!mbar_wait_sleep(&kv_empty[stage], phase ^ 1)) {
+            set_error(g.err, kDevErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          uint8_t* st = smem + stage * C::kStageBytes;
+          const uint32_t bar = full_bar0 + stage * 8;  // CTA 0's kv_full[stage]
+          if (rank == 0) mbar_arrive_expect_tx(&kv_full[stage], 2 * half_bytes);
+          const int key0 = t * k2Cols + (int)rank * (k2Cols / 2);
+#pragma unroll
+          for (int c = 0; c < DH / 64; ++c)
+            tma_load_3d_pair(st + c * C::kKChunk, &tm_kn, c * 64, key0, h, bar);
+          tma_load_3d_pair(st + 2 * C::kKHalf, &tm_vn, t * k2Cols, (int)rank * (DH / 2), h, bar);
+          if (has_old) {
+#pragma unroll
+            for (int c = 0; c < DH / 64; ++c)
+              tma_load_3d_pair(st + C::kKHalf + c * C::kKChunk, &tm_ko, c * 64, key0, h, bar);
+            tma_load_3d_pair(st + 2 * C::kKHalf + C::kVHalf, &tm_vo, t * k2Cols, (int)rank * (DH / 2), h, bar);
+          }
+          issued[stage] = (int)phase;
+          if (++stage == k2Stages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      // CTA 0's barriers count both CTAs' bytes: never leave with a copy in flight
+      if (rank == 0)
+        for (int s2 = 0; s2 < k2Stages; ++s2)
+          if (issued[s2] >= 0) (void)mbar_wait(&kv_full[s2], (uint32_t)issued[s2]);
+    }
+  } else if (warp == k4MmaWarp) {
+    // ------------------------------------------------------------ MMA issue (CTA 0)
+    if (lane == 0 && rank == 0) {
+      int stage = 0, prev_stage = 0;
+      uint32_t phase = 0;
+      uint32_t u = 0;
+      uint32_t item_no = 0;
+      bool ok = true;
+      for (int item = cluster; item < total && ok && !*abort_flag; item += n_clusters, ++item_no) {
+        const int h = item / pairs, rp = item % pairs;
+        const int nt = a2_tiles(g, h, rp, n_rows);
+        if (!mbar_wait_sleep(q_ready, item_no & 1)) {
+          set_error(g.err, kDevErrTimeout);
+          *abort_flag = 1;
+          break;
+        }
+        tc_fence_after();
+        for (int t = 0; t <= nt && ok; ++t) {
+          if (t < nt) {
+            // S(t) into buffer u & 1 of both CTAs
+            if (!mbar_wait_sleep(&kv_full[stage], phase)) {
+              set_error(g.err, kDevErrTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t sb = tmem + C::kColS + (u & 1) * 128;
+            const uint32_t k_addr = smem_u32(smem + stage * C::kStageBytes);
+#pragma unroll
+            for (int ks = 0; ks < DH / 16; ++ks) {
+              const uint32_t kd = k_addr + (ks >> 2) * C::kKChunk + (ks & 3) * 32;
+              umma_f16_ts_pair(sb, tmem + C::kColQn + ks * 8, sw128_kmajor_desc(kd), C::kIdescS, ks > 0);
+              if (has_old)
+                umma_f16_ts_pair(sb + 64, tmem + C::kColQo + ks * 8, sw128_kmajor_desc(kd + C::kKHalf), C::kIdescS,
+                                 ks > 0);
+            }
+            umma_commit_pair(&s_full[u & 1]);
+          }
+          if (t > 0) {
+            // P(t-1).V into N of both CTAs
+            const uint32_t up = u - 1;
+            if (!mbar_wait_sleep(&p_full[up & 1], (up >> 1) & 1)) {
+              set_error(g.err, kDevErrTimeout);
+              *abort_flag = 1;
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
+            const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKHalf);
+#pragma unroll
+            for (int ks = 0; ks < k2Cols / 16; ++ks)
+              umma_f16_ts_pair(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
+            if (has_old) {
+#pragma unroll
+              for (int ks = 0; ks < k2Cols / 16; ++ks)
+                umma_f16_ts_pair(tmem + C::kColN, pcol + 32 + ks * 8,
+                                 sw128_kmajor_desc(v_addr + C::kVHalf + ks * 32), C::kIdescPV, 1u);
+            }
+            umma_commit_pair(&kv_empty[prev_stage]);
+            umma_commit_pair(&pv_done[up & 1]);
+          }
+          if (t < nt) {
+            prev_stage = stage;
+            if (++stage == k2Stages) {
+              stage = 0;
+              phase ^= 1;
+            }
+            ++u;
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ rows (both CTAs)
+    // Four threads per row: part p (warps 4p..4p+3) takes columns
+    // [16 p, 16 p + 16) of S_new and S_old of each tile, a quarter of Q
+    // (parts 0-1 Q_new, 2-3 Q_old) and N columns [p DH/4, (p + 1) DH/4).
+    // The four warps of a lane quarter exchange tile maxima and sums through
+    // shared memory at a named barrier of 128 threads; dead mode as in
+    // attn_tc.cu.  Each warp reports with one arrival on CTA 0's barrier.
+    const int quarter = warp & 3, part = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int quad_bar = 1 + quarter;
+    const int HD = g.H * DH;
+    constexpr int kPartCols = DH / 4;   // N columns of a part
+    constexpr int kQElems = DH / 2;     // Q elements of a part (half of one matrix)
+    const uint32_t p_full0 = mapa_shared(smem_u32(p_full), 0);
+    const uint32_t q_ready0 = mapa_shared(smem_u32(q_ready), 0);
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity) {
+      if (!dead && __any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+      if (dead) return;
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar, parity))) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        dead = true;
+        return;
+      }
+      tc_fence_after();
+    };
+    auto warp_arrive = [&](uint32_t bar0) {
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(bar0);
+    };
+    uint32_t u = 0;
+    for (int item = cluster; item < total; item += n_clusters) {
+      const int h = item / pairs, rp = item % pairs;
+      const int nt = a2_tiles(g, h, rp, n_rows);
+      const int a = (rp * 2 + (int)rank) * k2Rows + row;
+      int tok = -1;
+      if (a < n_rows) {
+        tok = g.rows ? __ldg(g.rows + a) : a;
+        if (tok < 0 || tok >= g.S) {
+          if (part == 0) set_error(g.err, FLASHLOOP_DEVERR_INDEX);
+          tok = -1;
+        }
+      }
+      if (!dead) {
+        const bool old_q = part >= 2;
+        const uint16_t* qsrc = old_q ? g.q_old : g.q_new;
+        const bool load_q = tok >= 0 && (!old_q || has_old);
+        const bool load_n = !g.dense && tok >= 0;
+        const uint32_t qcol = (old_q ? C::kColQo : C::kColQn) + (part & 1) * (kQElems / 2);
+        const int q0 = (part & 1) * kQElems;   // first Q element of this part
+        uint32_t qv[kQElems / 16][8];
+#pragma unroll
+        for (int v = 0; v < kQElems / 16; ++v) {
+          if (load_q) {
+            ld_global_v8(qsrc + (size_t)tok * HD + (size_t)h * DH + q0 + v * 16, qv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[v][e] = 0u;
+          }
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kQElems; c0 += 32) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = bf16x2_to_half2_bits(qv[c0 / 16 + e / 8][e % 8]);
+          __syncwarp();
+          tmem_st16(tmem + lane_base + qcol + c0 / 2, r);
+        }
+        uint32_t nv[kPartCols / 8][8];
+#pragma unroll
+        for (int v = 0; v < kPartCols / 8; ++v) {
+          if (load_n) {
+            ld_global_v8(g.n_in + ((size_t)h * g.S + tok) * DH + part * kPartCols + 8 * v, nv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) nv[v][e] = 0u;
+          }
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kPartCols; c0 += 16) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = nv[c0 / 8 + e / 8][e % 8];
+          __syncwarp();
+          tmem_st16(tmem + lane_base + C::kColN + part * kPartCols + c0, r);
+        }
+        warp_arrive(q_ready0);
+      }
+      float m_ref = 0.f, z = 0.f;
+      if (tok >= 0) {
+        m_ref = g.dense ? -INFINITY : g.m_in[(size_t)h * g.S + tok] * k2Log2e;
+        if (!g.dense && part == 0) z = g.z_in[(size_t)h * g.S + tok];
+      }
+      const int32_t* hcols = g.cols ? g.cols + (size_t)h * g.kc : nullptr;
+      int wmin = tok < 0 ? 0x7fffffff : tok;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) wmin = min(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+      auto tile_last = [&](int tt) -> int {
+        const int ce = min((tt + 1) * k2Cols, g.kc);
+        return hcols ? __ldg(hcols + ce - 1) : ce - 1;
+      };
+      int next_last = nt > 0 ? tile_last(0) : 0;
+      for (int t = 0; t < nt; ++t, ++u) {
+        const uint32_t b = u & 1;
+        const int c0 = t * k2Cols;
+        const int c_end = min(c0 + k2Cols, g.kc);
+        const int last_tok = next_last;
+        if (t + 1 < nt) next_last = tile_last(t + 1);
+        const bool need_mask = (c0 + k2Cols > g.kc) || (last_tok > wmin);
+        int nvalid = k2Cols;
+        if (need_mask) {
+          if (tok < 0) {
+            nvalid = 0;
+          } else {
+            int lo = c0, hi = c_end;
+            while (lo < hi) {
+              const int mid = (lo + hi) >> 1;
+              const int ct = hcols ? __ldg(hcols + mid) : mid;
+              if (ct <= tok) lo = mid + 1;
+              else hi = mid;
+            }
+            nvalid = lo - c0;
+          }
+        }
+        const int first = part * 16;
+        wait_or_die(&s_full[b], (u >> 1) & 1);
+        uint32_t rn[16], ro[16];
+        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
+        float mx = -INFINITY;
+        if (!dead) {
+          __syncwarp();
+          tmem_ld16(sbase + first, rn);
+          if (has_old) tmem_ld16(sbase + 64 + first, ro);
+          tmem_wait_ld();
+          if (nvalid < first + 16) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              if (first + e >= nvalid) {
+                rn[e] = 0xff800000u;
+                ro[e] = 0xff800000u;
+              }
+            }
+          }
+          float t8[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) t8[e] = fmaxf(__uint_as_float(rn[e]), __uint_as_float(rn[e + 8]));
+#pragma unroll
+          for (int w = 4; w > 0; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e) t8[e] = fmaxf(t8[e], t8[e + w]);
+          mx = t8[0];
+        }
+        float* xm = xchg + b * 4 * 128;  // [part][128] of this parity
+        xm[part * 128 + row] = mx;
+        named_bar_sync(quad_bar, 128);
+        mx = fmaxf(fmaxf(xm[row], xm[128 + row]), fmaxf(xm[256 + row], xm[384 + row]));
+        if (dead) continue;
+        const bool need = mx > m_ref + k2RescaleThreshold;
+        if (__any_sync(0xffffffffu, need)) {
+          const float new_ref = need ? mx : m_ref;
+          const float f = need ? ex2(m_ref - new_ref) : 1.f;
+          if (t > 0) {
+            const uint32_t up = u - 1;
+            wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+            if (dead) continue;
+          }
+#pragma unroll 1
+          for (int cc = 0; cc < kPartCols; cc += 16) {
+            uint32_t r[16];
+            __syncwarp();
+            tmem_ld16(tmem + lane_base + C::kColN + part * kPartCols + cc, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+            __syncwarp();
+            tmem_st16(tmem + lane_base + C::kColN + part * kPartCols + cc, r);
+          }
+          tmem_wait_st();
+          z *= f;
+          m_ref = new_ref;
+        }
+        uint32_t pk[8];
+        float za[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int e2 = 0; e2 < 8; ++e2) {
+          const float p0 = ex2(__uint_as_float(rn[2 * e2]) - m_ref);
+          const float p1 = ex2(__uint_as_float(rn[2 * e2 + 1]) - m_ref);
+          za[e2 & 3] += p0 + p1;
+          pk[e2] = pack_half2(p0, p1);
+        }
+        __syncwarp();
+        tmem_st8(sbase + part * 8, pk);
+        if (has_old) {
+          float zb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e2 = 0; e2 < 8; ++e2) {
+            const float p0 = ex2(__uint_as_float(ro[2 * e2]) - m_ref);
+            const float p1 = ex2(__uint_as_float(ro[2 * e2 + 1]) - m_ref);
+            zb[e2 & 3] += p0 + p1;
+            pk[e2] = pack_half2(-p0, -p1);
+          }
+          __syncwarp();
+          tmem_st8(sbase + 32 + part * 8, pk);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) za[i] -= zb[i];
+        }
+        z += (za[0] + za[1]) + (za[2] + za[3]);
+        warp_arrive(p_full0 + b * 8);
+      }
+      if (nt > 0) {
+        const uint32_t up = u - 1;
+        wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+      }
+      float* xz = xchg + 8 * 128;   // [part][128]
+      xz[part * 128 + row] = z;
+      named_bar_sync(quad_bar, 128);
+      const float z_row = (xz[row] + xz[128 + row]) + (xz[256 + row] + xz[384 + row]);
+      named_bar_sync(quad_bar, 128);
+      if (dead) continue;
+      const float inv = 1.f / z_row;
+#pragma unroll 1
+      for (int cc = 0; cc < kPartCols; cc += 16) {
+        uint32_t r[16];
+        __syncwarp();
+        tmem_ld16(tmem + lane_base + C::kColN + part * kPartCols + cc, r);
+        tmem_wait_ld();
+        if (tok >= 0) {
+          const int col = part * kPartCols + cc;
+          float* nd = g.n_out + ((size_t)h * g.S + tok) * DH + col;
+          uint32_t w[8];
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = r[8 * v + e];
+            st_global_v8(nd + 8 * v, w);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q]) * inv) |
+                   ((uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q + 1]) * inv) << 16);
+          st_global_v8(g.o + (size_t)tok * HD + (size_t)h * DH + col, w);
+        }
+      }
+      if (tok >= 0 && part == 0) {
+        g.m_out[(size_t)h * g.S + tok] = m_ref / k2Log2e;
+        g.z_out[(size_t)h * g.S + tok] = z_row;
+        if (g.dense && g.g_out) g.g_out[(size_t)h * g.S + tok] = 1.f;
+      }
+      tc_fence_before();
+    }
+  }
+  // neither CTA leaves (or frees TMEM) while the pair's MMAs, loads or
+  // arrivals may still touch it
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == k4TmaWarp) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -587,17 +1035,16 @@ int make_tmap_f16_3d(CUtensorMap* m, const void* base, uint64_t d0, uint64_t d1,
                      uint64_t s2_elems, uint32_t b0, uint32_t b1);
 int at_sm_count();
 
-// Pairs of SMs the device can run at once for this kernel (clusters of 2).
-template <int DH>
-static int a2_max_pairs() {
-  static int cached[64] = {0};
+// Pairs of SMs the device can run at once for a kernel (clusters of 2).
+static int a2_max_pairs(const void* kernel, int threads, int smem, int slot) {
+  static int cached[4][64] = {{0}};
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 0;
-  if (cached[dev] != 0) return cached[dev];
+  if (cached[slot][dev] != 0) return cached[slot][dev];
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * 74, 1, 1);
-  cfg.blockDim = dim3(k2Threads, 1, 1);
-  cfg.dynamicSmemBytes = A2Cfg<DH>::kSmem;
+  cfg.blockDim = dim3(threads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -606,26 +1053,30 @@ static int a2_max_pairs() {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, attn_pair_kernel<DH>, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
     (void)cudaGetLastError();
     n = -1;
   }
-  cached[dev] = n;
+  cached[slot][dev] = n;
   return n;
 }
 
-// The running update on SM pairs; returns FLASHLOOP_ERR_UNSUPPORTED when the
-// device cannot co-schedule pairs (the caller then uses one SM per tile).
+// The running update on SM pairs (params.attn_pairs: 1 two threads per row,
+// 2 four threads per row); returns FLASHLOOP_ERR_UNSUPPORTED when the device
+// cannot co-schedule pairs (the caller then uses one SM per tile).
 int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
   if (dh != 128 && dh != 64) return FLASHLOOP_ERR_UNSUPPORTED;
   const void* aligned32[] = {a.q_new, a.q_old, a.n_in, a.n_out, a.o};
   for (const void* ptr : aligned32)
     if (reinterpret_cast<uintptr_t>(ptr) % 32 != 0) return FLASHLOOP_ERR_INVALID_ARG;
-  const int smem = dh == 128 ? A2Cfg<128>::kSmem : A2Cfg<64>::kSmem;
-  if (dh == 128) FL_TRY(cudaFuncSetAttribute(attn_pair_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  else FL_TRY(cudaFuncSetAttribute(attn_pair_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
-  const int max_pairs = dh == 128 ? a2_max_pairs<128>() : a2_max_pairs<64>();
+  const bool four = p->attn_pairs == 2;
+  const void* kernel = four ? (dh == 128 ? (const void*)attn_pair4_kernel<128> : (const void*)attn_pair4_kernel<64>)
+                            : (dh == 128 ? (const void*)attn_pair_kernel<128> : (const void*)attn_pair_kernel<64>);
+  const int threads = four ? k4Threads : k2Threads;
+  const int smem = four ? (dh == 128 ? a4_smem<128>() : a4_smem<64>()) : (dh == 128 ? A2Cfg<128>::kSmem : A2Cfg<64>::kSmem);
+  FL_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+  const int max_pairs = a2_max_pairs(kernel, threads, smem, (four ? 2 : 0) + (dh == 128 ? 1 : 0));
   if (max_pairs <= 0) return FLASHLOOP_ERR_UNSUPPORTED;
   // K halves: 32 keys x 64 head-dim elements per box; V^T halves: 64 keys x DH/2 rows
   CUtensorMap tkn, tko, tvn, tvo;
@@ -652,7 +1103,7 @@ int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cuda
   if (n_pairs < 1) n_pairs = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * n_pairs, 1, 1);
-  cfg.blockDim = dim3(k2Threads, 1, 1);
+  cfg.blockDim = dim3(threads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -662,8 +1113,13 @@ int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cuda
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (dh == 128) FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair_kernel<128>, tkn, tko, tvn, tvo, g));
-  else FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair_kernel<64>, tkn, tko, tvn, tvo, g));
+  if (four) {
+    if (dh == 128) FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair4_kernel<128>, tkn, tko, tvn, tvo, g));
+    else FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair4_kernel<64>, tkn, tko, tvn, tvo, g));
+  } else {
+    if (dh == 128) FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair_kernel<128>, tkn, tko, tvn, tvo, g));
+    else FL_TRY(cudaLaunchKernelEx(&cfg, attn_pair_kernel<64>, tkn, tko, tvn, tvo, g));
+  }
   return launch_status();
 }
 

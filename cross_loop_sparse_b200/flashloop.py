@@ -52,7 +52,7 @@ class Params(ctypes.Structure):
         the running update on SM pairs."""
         p = cls()
         p.fixed_mass = 1 if fixed_mass else 0
-        p.attn_pairs = 1 if attn_pairs else 0
+        p.attn_pairs = int(attn_pairs)
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
         p.n_loops, p.batch = cfg.n_loops, (cfg.batch if cfg.decode else 1)

@@ -75,7 +75,8 @@ typedef struct flashloop_params {
   int32_t capacity[FLASHLOOP_MAX_LOOPS]; /* rows allocated for loop r's active list and residual stream */
   int32_t gate_topk; /* 0: the tau threshold gate; else top-k token retention keeping capacity[r-1] tokens */
   int32_t fixed_mass; /* 0: running (m, N, Z) update; else the fixed-mass form (see flashloop_sparse_attn_update) */
-  int32_t attn_pairs; /* running update: 0 one SM per 128-row tile; else SM pairs sharing each K/V tile (cta_group::2) */
+  int32_t attn_pairs; /* running update: 0 one SM per 128-row tile; 1 / 2 SM pairs sharing each K/V tile
+                         (cta_group::2) with two / four row threads per row */
 } flashloop_params;
 
 /* One quantised cache (K or V) of a sequence: the loop-1 base over every

@@ -372,15 +372,17 @@ def test_loop_step_fixed_mass_matches_oracle(case):
     assert st.error_code() == 0
 
 
+@pytest.mark.parametrize("pairs", [1, 2])
 @pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
-def test_loop_step_on_sm_pairs_matches_oracle(name):
+def test_loop_step_on_sm_pairs_matches_oracle(name, pairs):
     """The running update on SM pairs (two CTAs share every K / V tile, each
-    loading half; cta_group::2 MMAs over 256 rows), loop 1 included."""
+    loading half; cta_group::2 MMAs over 256 rows), loop 1 included, with two
+    (pairs = 1) or four (pairs = 2) threads per row."""
     cfg = CONFIGS[name]
     W = make_weights(cfg)
     X, _ = make_hidden_states(cfg)
     orc = O.OracleSequence(cfg, W, X).run()
-    p, st, snaps = run_gpu(cfg, W, X, attn_pairs=True)
-    assert p.attn_pairs == 1
+    p, st, snaps = run_gpu(cfg, W, X, attn_pairs=pairs)
+    assert p.attn_pairs == pairs
     worst = compare(cfg, orc, snaps, st, list(range(cfg.n_heads)), True)
     print(name, "pairs", worst)
