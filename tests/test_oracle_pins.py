@@ -184,6 +184,131 @@ def test_rope_closed_forms():
     assert abs(d1 - d2) < 1e-10
 
 
+# ---------------------------------------------------------------- projections
+def _rope_elem(x, d, pos, theta):
+    """Element d of rotate-half RoPE of the head vector x at position pos,
+    written out: pair (i, i + dh/2) turns by pos * theta^(-2i/dh)."""
+    dh = x.shape[0]
+    half = dh // 2
+    i = d % half
+    ang = pos * theta ** (-(2.0 * i) / dh)
+    if d < half:
+        return x[d] * math.cos(ang) - x[d + half] * math.sin(ang)
+    return x[d] * math.cos(ang) + x[d - half] * math.sin(ang)
+
+
+def _bf16_close(got_bits, want):
+    """bf16 values within one bf16 step (2^-7 relative) of float64 values."""
+    got = bf16_bits_to_f32(got_bits).astype(np.float64)
+    want = np.asarray(want, dtype=np.float64)
+    return np.all(np.abs(got - want) <= 2.0 ** -7 * np.maximum(np.abs(got), np.abs(want)) + 1e-30)
+
+
+def test_projection_selector_weights_give_rope_of_chosen_inputs():
+    """Weights with one non-zero entry per output row pick one input element:
+    q = RoPE(x[c_q]), k = RoPE(2 x[c_k]), v = -x[c_v], each from its own
+    matrix (W_q, W_k, W_v take different columns) and its own head block."""
+    rng = np.random.default_rng(11)
+    H, dh, d, theta = 3, 8, 24, 1e4
+    n = 5
+    x = f32_to_bf16_bits(rng.standard_normal((n, d)).astype(np.float32))
+    xv = bf16_bits_to_f32(x).astype(np.float64)
+    pos = np.array([0, 3, 17, 1000, 32767])
+    picks = {name: rng.permutation(d) for name in ("wq", "wk", "wv")}
+    gains = {"wq": 1.0, "wk": 2.0, "wv": -1.0}
+    W = {}
+    for name in ("wq", "wk", "wv"):
+        w = np.zeros((d, d), np.float32)
+        w[np.arange(d), picks[name]] = gains[name]
+        W[name] = f32_to_bf16_bits(w)
+    assert not np.array_equal(picks["wq"], picks["wk"])
+    heads = [2, 0]
+    q, k, v = O.project_qkv(x, pos, W, heads, dh, theta)
+    assert q.shape == (n, 2, dh) and k.shape == (n, 2, dh) and v.shape == (n, 2, dh)
+    for t in range(n):
+        for a, h in enumerate(heads):
+            rows = np.arange(h * dh, (h + 1) * dh)
+            pre = {name: gains[name] * xv[t, picks[name][rows]] for name in ("wq", "wk", "wv")}
+            q_want = [_rope_elem(pre["wq"], e, pos[t], theta) for e in range(dh)]
+            k_want = [_rope_elem(pre["wk"], e, pos[t], theta) for e in range(dh)]
+            assert _bf16_close(q[t, a], q_want), (t, h)
+            assert np.allclose(k[t, a], k_want, rtol=1e-12, atol=1e-12), (t, h)
+            assert np.array_equal(v[t, a], pre["wv"]), (t, h)
+
+
+def test_oracle_queries_match_projection_written_out(tiny):
+    """run.q of every loop: for active rows, x_r . (row of W_q) followed by the
+    written-out RoPE at the token position, rounded to bf16; for inactive
+    rows, the previous loop's query unchanged."""
+    cfg, W, X, _, run = tiny
+    H, dh = cfg.n_heads, cfg.head_dim
+    wq = bf16_bits_to_f32(W["wq"]).astype(np.float64)
+    rng = np.random.default_rng(12)
+    for r in range(1, cfg.n_loops + 1):
+        act = run.active[r]
+        x = bf16_bits_to_f32(X[r - 1]).astype(np.float64)
+        for t in rng.choice(act, size=min(12, act.size), replace=False):
+            for h in range(H):
+                pre = np.array([np.dot(x[t], wq[h * dh + e]) for e in range(dh)])
+                want = [_rope_elem(pre, e, int(t), cfg.rope_theta) for e in range(dh)]
+                assert _bf16_close(run.q[r][t, h], want), (r, t, h)
+        if r >= 2:
+            inactive = np.setdiff1d(np.arange(cfg.seq), act)
+            assert np.array_equal(run.q[r][inactive], run.q[r - 1][inactive])
+
+
+def _y_brute(o_bits, wo_bits):
+    """Y[i, c] = bf16(sum_e O[i, e] W_o[c, e]), one exactly rounded sum per element."""
+    o = bf16_bits_to_f32(o_bits).astype(np.float64)
+    w = bf16_bits_to_f32(wo_bits).astype(np.float64)
+    y = np.empty((o.shape[0], w.shape[0]))
+    for i in range(o.shape[0]):
+        for c in range(w.shape[0]):
+            y[i, c] = math.fsum(o[i] * w[c])
+    return f32_to_bf16_bits(y.astype(np.float32))
+
+
+def test_out_projection_hand_case_identity_and_permutation():
+    """Y = O W_o^T: a 1 x 4 case by hand, W_o = I returns O, and permuting
+    W_o's rows permutes Y's columns (a W_o used untransposed fails all three)."""
+    o = f32_to_bf16_bits(np.array([[1.0, 2.0, 3.0, 4.0]], np.float32))
+    wo = f32_to_bf16_bits(np.array([[1, 0, 0, 0], [0, 0, 0, 2], [1, 1, 0, 0], [0, 0, 0.5, 0]], np.float32))
+    y = bf16_bits_to_f32(O.out_projection(o, wo))
+    assert y.tolist() == [[1.0, 8.0, 3.0, 1.5]]
+    rng = np.random.default_rng(13)
+    d = 16
+    o = f32_to_bf16_bits(rng.standard_normal((7, d)).astype(np.float32))
+    eye = f32_to_bf16_bits(np.eye(d, dtype=np.float32))
+    assert np.array_equal(O.out_projection(o, eye), o)
+    wo = f32_to_bf16_bits((rng.standard_normal((d, d)) / 4).astype(np.float32))
+    perm = rng.permutation(d)
+    assert np.array_equal(O.out_projection(o, wo[perm]), O.out_projection(o, wo)[:, perm])
+
+
+def test_out_projection_brute_force():
+    """Every element against an exactly rounded per-element sum (bf16 products
+    and short sums are exact in float64, so the bits agree)."""
+    rng = np.random.default_rng(14)
+    o = f32_to_bf16_bits(rng.standard_normal((6, 32)).astype(np.float32))
+    wo = f32_to_bf16_bits((rng.standard_normal((24, 32)) / 6).astype(np.float32))
+    assert np.array_equal(O.out_projection(o, wo), _y_brute(o, wo))
+
+
+def test_sequence_output_projection_active_rows_and_kept_rows(tiny):
+    """In a run: Y of loop r's active rows is the brute-force projection of that
+    loop's O rows; every other row keeps the previous loop's Y."""
+    cfg, W, X, _, run = tiny
+    rng = np.random.default_rng(15)
+    for r in range(1, cfg.n_loops + 1):
+        act = run.active[r]
+        some = np.sort(rng.choice(act, size=min(6, act.size), replace=False))
+        assert np.array_equal(run.Y_hist[r][some], _y_brute(run.O_hist[r][some], W["wo"]))
+        if r >= 2:
+            inactive = np.setdiff1d(np.arange(cfg.seq), act)
+            assert np.array_equal(run.Y_hist[r][inactive], run.Y_hist[r - 1][inactive])
+            assert np.array_equal(run.O_hist[r][inactive], run.O_hist[r - 1][inactive])
+
+
 # ---------------------------------------------------------------- gate
 def test_gate_threshold_is_inclusive_and_squared():
     d = 256
