@@ -6,6 +6,8 @@
 #include <math.h>
 #include <stdio.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace fl {
@@ -45,18 +47,20 @@ int launch_colmass_tc(const flashloop_params*, const ColmassArgs&, void*, void*,
 // checks
 // ---------------------------------------------------------------------------
 static int check_arch() {
-  static int cached[64];  // 0 = unknown, 1 = sm_100, -1 = other
+  static std::atomic<int> cached[64];  // 0 = unknown, 1 = sm_100, -1 = other
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return FLASHLOOP_ERR_CUDA;
   if (dev < 0 || dev >= 64) return FLASHLOOP_ERR_CUDA;
-  if (cached[dev] == 0) {
+  int c = cached[dev].load(std::memory_order_relaxed);
+  if (c == 0) {
     int major = 0, minor = 0;
     if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return FLASHLOOP_ERR_CUDA;
-    cached[dev] = (major == 10 && minor == 0) ? 1 : -1;
+    c = (major == 10 && minor == 0) ? 1 : -1;
+    cached[dev].store(c, std::memory_order_relaxed);
   }
-  return cached[dev] == 1 ? FLASHLOOP_OK : FLASHLOOP_ERR_ARCH;
+  return c == 1 ? FLASHLOOP_OK : FLASHLOOP_ERR_ARCH;
 }
 
 static int check_params(const flashloop_params* p) {
@@ -84,6 +88,11 @@ static int check_common(const flashloop_params* p) {
   if (rc != FLASHLOOP_OK) return rc;
   return check_arch();
 }
+
+// The parameter and architecture checks of every entry point, for the entry
+// points defined in other files.
+int check_params_and_arch(const flashloop_params* p) { return check_common(p); }
+int check_device_arch() { return check_arch(); }
 
 static inline cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

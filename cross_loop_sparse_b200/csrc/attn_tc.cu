@@ -360,14 +360,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
             for (int e = 0; e < 8; ++e) qv[v][e] = 0u;
           }
         }
+        bool q_ok = true;  // q must fit fp16, the MMA operand type
 #pragma unroll
         for (int c0 = 0; c0 < DH; c0 += 32) {
           uint32_t r[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) r[e] = bf16x2_to_half2_bits(qv[c0 / 16 + e / 8][e % 8]);
+          for (int e = 0; e < 16; ++e) {
+            const float2 f = bf16x2_to_float2(qv[c0 / 16 + e / 8][e % 8]);
+            q_ok = q_ok && half_range_ok(f.x) && half_range_ok(f.y);
+            r[e] = bf16x2_to_half2_bits(qv[c0 / 16 + e / 8][e % 8]);
+          }
           __syncwarp();
           tmem_st16(tmem + lane_base + qcol + c0 / 2, r);
         }
+        if (!q_ok) set_error(g.err, FLASHLOOP_DEVERR_RANGE);
         uint32_t nv[kHalfCols / 8][8];
 #pragma unroll
         for (int v = 0; v < kHalfCols / 8; ++v) {
@@ -919,15 +925,17 @@ colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, floa
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+// The driver's cuTensorMapEncodeTiled, looked up once (a function-local
+// static: its initialisation is thread-safe).
 static PFN_cuTensorMapEncodeTiled_v12000 at_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (fn == nullptr) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* p = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    return nullptr;
+  }();
   return fn;
 }
 

@@ -42,6 +42,12 @@ __device__ __forceinline__ uint16_t float_to_bf16_bits(float f) {
   return __bfloat16_as_ushort(__float2bfloat16_rn(f));
 }
 
+// Largest finite fp16: the range of every tensor-core operand of the library.
+constexpr float kHalfMax = 65504.f;
+
+// |x| <= 65504 (false for NaN): x converts to fp16 without overflow.
+__device__ __forceinline__ bool half_range_ok(float x) { return fabsf(x) <= kHalfMax; }
+
 // bf16 pair -> fp16 pair (exact for |x| in fp16's normal range).
 __device__ __forceinline__ uint32_t bf16x2_to_half2_bits(uint32_t w) {
   float2 f = bf16x2_to_float2(w);

@@ -250,6 +250,14 @@ selcol_dequant_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, 
 #pragma unroll
         for (int e = 0; e < E; ++e) acc[e] = oldv[e] = 0.f;
       }
+      {
+        // the attention MMAs take fp16 operands: flag a value that does not fit
+        const float sc = which == 0 ? kscale : 1.f;
+        bool ok = true;
+#pragma unroll
+        for (int e = 0; e < E; ++e) ok = ok && half_range_ok(acc[e] * sc) && half_range_ok(oldv[e] * sc);
+        if (!ok) set_error(err, FLASHLOOP_DEVERR_RANGE);
+      }
       if (which == 0) {
         if (col < kcp) {
           const size_t off = ((size_t)h * kcp + col) * DH + lane * E;

@@ -121,6 +121,7 @@ _SIG = {
     "flashloop_decode_out": (_I, [_P, _V, _D, _V]),
     "flashloop_selection_loop": (_I, [_P, _I]),
     "flashloop_check_error_word": (_I, [_V, POINTER(c_int32), _V]),
+    "flashloop_selftest_bounded_wait": (_I, [_I, _V, _V]),
     "flashloop_status_string": (ctypes.c_char_p, [_I]),
 }
 for _name, (_res, _args) in _SIG.items():
@@ -295,6 +296,11 @@ def flashloop_decode_step(params, loop, x_tok, w_qkv, w_o, ctx, dstate, stream=N
     return _check("flashloop_decode_step", _lib.flashloop_decode_step(
         ctypes.byref(params), loop, _ptr(x_tok), _ptr(w_qkv), _ptr(w_o), ctypes.byref(ctx.c),
         ctypes.byref(dstate.c), _stream(stream)))
+
+
+def flashloop_selftest_bounded_wait(kind, err_word, stream=None):
+    return _check("flashloop_selftest_bounded_wait", _lib.flashloop_selftest_bounded_wait(
+        int(kind), _ptr(err_word), _stream(stream)))
 
 
 def flashloop_check_error_word(err_word, stream=None):

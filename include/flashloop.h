@@ -59,6 +59,10 @@ typedef enum flashloop_status {
 /* Codes a kernel may leave in *err_word. */
 #define FLASHLOOP_DEVERR_CAPACITY 1 /* more active tokens than the loop's capacity */
 #define FLASHLOOP_DEVERR_INDEX 2    /* a token or column index outside [0, S) */
+#define FLASHLOOP_DEVERR_TIMEOUT 3  /* a bounded wait inside a pipelined kernel gave up */
+#define FLASHLOOP_DEVERR_RANGE 4    /* an attention operand (q, or a rebuilt key or value, keys
+                                       times log2(e)/sqrt(dh)) is NaN or beyond the largest fp16
+                                       (65504): the tensor-core operands are fp16 */
 
 /* Problem description.  Plain values, read on the host only. */
 typedef struct flashloop_params {
@@ -175,8 +179,13 @@ int flashloop_gate(const flashloop_params* p, const uint16_t* x_cur, const uint1
  *  - Candidates (prev_capacity, or S when prev_active is NULL) above
  *    FLASHLOOP_NOALLOC_MAX_CANDIDATES return FLASHLOOP_ERR_UNSUPPORTED.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress) and caches it; make that first call before any
- *    stream capture.
+ *    (cudaGetSymbolAddress) and caches it with the current context; make
+ *    that first call before any stream capture.  A call made in another
+ *    context of that device (after cudaDeviceReset, or a new context) looks
+ *    the address up again: the first call after such a change is again a
+ *    set-up call and belongs before any capture.
+ *  - Parameters, architecture and arguments are checked exactly as
+ *    flashloop_gate checks them, with the same status codes.
  *  - Nothing is allocated or freed; each call zeroes the ticket with
  *    cudaMemsetAsync on `stream`, then launches the gate kernel.
  *  - Every call shares the one array, which keeps the previous call's
@@ -389,6 +398,16 @@ int32_t flashloop_selection_loop(const flashloop_params* p, int32_t loop);
 /* Copy *err_word to the host (synchronising the stream) and map it to a
  * status: FLASHLOOP_OK, or FLASHLOOP_ERR_DEVICE with the code in *code. */
 int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* stream);
+
+/* Self-test of the bounded waits that every pipelined kernel of the library
+ * uses (diagnostics; the paper has no counterpart).  One thread initialises a
+ * shared-memory barrier that nothing ever completes and waits on it with the
+ * library's spinning wait (kind 0, about 2^22 polls with back-off) or its
+ * sleeping wait (kind 1, about 2^16 tries of up to 20 us); when the wait gives
+ * up the kernel writes FLASHLOOP_DEVERR_TIMEOUT to *err_word and returns, so
+ * the stream and the context stay usable.  Takes about a second on the GPU.
+ * Returns FLASHLOOP_ERR_INVALID_ARG for another kind or a NULL err_word. */
+int flashloop_selftest_bounded_wait(int32_t kind, int32_t* err_word, void* stream);
 
 /* Static description of a status code. */
 const char* flashloop_status_string(int status);

@@ -120,3 +120,31 @@ def test_decode_refuses_the_fixed_mass_form():
     assert F._lib.flashloop_decode_workspace_bytes(ctypes.byref(p)) > 0
     p = F.Params.from_config(cfg, fixed_mass=True)
     assert F._lib.flashloop_decode_workspace_bytes(ctypes.byref(p)) == 0
+
+
+def test_noalloc_gate_refuses_what_the_workspace_gate_refuses():
+    """flashloop_gate_noalloc runs flashloop_gate's parameter checks first, so
+    bad parameters get the same status from both, before any device query."""
+    cfg = CONFIGS["tiny"]
+    dummy = ctypes.c_void_p(16)
+
+    def both(p):
+        g = F._lib.flashloop_gate(ctypes.byref(p), dummy, dummy, None, None, cfg.seq, dummy, dummy,
+                                  dummy, cfg.seq, dummy, dummy, None)
+        n = F._lib.flashloop_gate_noalloc(ctypes.byref(p), dummy, dummy, None, None, cfg.seq, dummy,
+                                          dummy, dummy, cfg.seq, dummy, None)
+        return g, n
+
+    cases = []
+    p = F.Params.from_config(cfg); p.head_dim = 96; p.d_model = 96 * 4
+    cases.append((p, -2))
+    p = F.Params.from_config(cfg); p.d_model = 200
+    cases.append((p, -1))
+    p = F.Params.from_config(cfg); p.bits[2] = 3
+    cases.append((p, -2))
+    p = F.Params.from_config(cfg); p.n_heads = 0
+    cases.append((p, -1))
+    p = F.Params.from_config(cfg); p.tau = -1.0
+    cases.append((p, -1))
+    for p, want in cases:
+        assert both(p) == (want, want)

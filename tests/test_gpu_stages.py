@@ -128,6 +128,72 @@ def test_topk_ties_candidates_and_edges():
     assert np.array_equal(out.cpu().numpy(), np.tile(np.arange(S), (H, 1)))
 
 
+def test_gate_bit_exact_at_32k():
+    """The gate of loops 2..4 on the 32K workload's hidden states, each loop
+    given the oracle's previous active set: sets, slot maps and counts
+    bit-exact."""
+    cfg = CONFIGS["prefill_32k"]
+    X, _ = make_hidden_states(cfg)
+    p = F.Params.from_config(cfg)
+    st = F.FlashLoopState(p, kv_only=True)
+    xs = [bf16_to_torch(x) for x in X]
+    S = cfg.seq
+    prev = np.arange(S)
+    for r in range(2, cfg.n_loops + 1):
+        want = O.gate(X[r - 1], X[r - 2], prev, cfg.tau)
+        D, P = O.gate_norms(X[r - 1], X[r - 2], prev)
+        assert np.min(np.abs(np.sqrt(D / P) - cfg.tau)) > 1e-3 * cfg.tau   # no row on the threshold
+        act = torch.zeros(S, dtype=torch.int32, device="cuda")
+        slot = torch.full((S,), 7, dtype=torch.int32, device="cuda")
+        n = torch.zeros(1, dtype=torch.int32, device="cuda")
+        F.flashloop_gate(p, xs[r - 1], xs[r - 2], None if r == 2 else i32(prev),
+                         None if r == 2 else i32([prev.size]), S, act, slot, n, S, st["workspace"], st["err"])
+        torch.cuda.synchronize()
+        assert int(n.item()) == want.size, r
+        assert np.array_equal(act[: want.size].cpu().numpy(), want), r
+        ws = np.full(S, -1, np.int32)
+        ws[want] = np.arange(want.size)
+        assert np.array_equal(slot.cpu().numpy(), ws), r
+        prev = want
+    assert st.error_code() == 0
+
+
+@pytest.mark.parametrize("with_candidates", [False, True])
+def test_topk_bit_exact_at_32k_all_heads(with_candidates):
+    """Top-k of S = 32768 columns on all 16 heads (one radix select over 32K
+    keys per head), k = 3277: a column mass shaped like the workload's
+    (about ln(S/j) with noise), exact ties planted at each head's k-th value
+    and zeros of both signs; and the shrinking-budget form, k = 1638 among a
+    head's 3277 previous columns.  Identical sets to the oracle's top-k."""
+    cfg = CONFIGS["prefill_32k"]
+    p = F.Params.from_config(cfg)
+    H, S, k = cfg.n_heads, cfg.seq, cfg.k
+    rng = np.random.default_rng(21)
+    j = np.arange(S, dtype=np.float64)
+    mass = (np.log(S / (j + 1.0))[None, :] * (1.0 + 0.05 * rng.standard_normal((H, S)))).astype(np.float32)
+    for h in range(H):
+        kth = np.sort(mass[h])[::-1][k - 1]
+        mass[h, rng.choice(S, 40, replace=False)] = kth
+        z = rng.choice(S, 20, replace=False)
+        mass[h, z] = np.where(rng.random(20) < 0.5, np.float32(0.0), np.float32(-0.0))
+    if with_candidates:
+        cand = np.stack([O.topk_columns(mass[h], np.arange(S), k) for h in range(H)]).astype(np.int32)
+        kk = (k + 1) // 2
+        for h in range(H):   # ties at the new k-th value inside the candidates
+            vals = mass[h, cand[h]]
+            kth = np.sort(vals)[::-1][kk - 1]
+            mass[h, cand[h][rng.choice(k, 12, replace=False)]] = kth
+        want = np.stack([O.topk_columns(mass[h], cand[h], kk) for h in range(H)])
+        out = torch.zeros((H, kk), dtype=torch.int32, device="cuda")
+        F.flashloop_topk_columns(p, f32(mass), i32(cand), k, kk, out)
+    else:
+        want = np.stack([O.topk_columns(mass[h], np.arange(S), k) for h in range(H)])
+        out = torch.zeros((H, k), dtype=torch.int32, device="cuda")
+        F.flashloop_topk_columns(p, f32(mass), None, 0, k, out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), want)
+
+
 @pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
 def test_gathered_qkv_projection(name):
     cfg, W, X, planted, orc = oracle_run(name)

@@ -9,6 +9,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from workload import CONFIGS, make_hidden_states
 
 pytestmark = pytest.mark.gpu
@@ -41,9 +42,13 @@ def test_noalloc_gate_matches_workspace_gate_on_consecutive_calls(name):
     xs = [_dev(x) for x in X]
     ws = torch.zeros(F.flashloop_workspace_bytes(p), dtype=torch.uint8, device="cuda")
     prev, n_prev = None, None
+    cand = np.arange(S)
     for r in range(2, cfg.n_loops + 1):
         want = _outputs(F.flashloop_gate, p, xs[r - 1], xs[r - 2], prev, n_prev, S,
                         lambda err: (ws, err))
+        # the workspace gate itself is the oracle's gate, bit for bit
+        cand = O.gate(X[r - 1], X[r - 2], cand, cfg.tau)
+        assert np.array_equal(want[1], cand), r
         for call in range(2):          # two calls in a row share the static scratch
             got = _outputs(F.flashloop_gate_noalloc, p, xs[r - 1], xs[r - 2], prev, n_prev, S,
                            lambda err: (err,))
