@@ -35,6 +35,7 @@ int launch_qkv_quant_gemm(const flashloop_params*, int, const uint16_t*, const i
 
 namespace fl {
 int launch_attn_tc(const flashloop_params*, const AttnArgs&, int, cudaStream_t);
+int launch_attn_row_counts(const AttnArgs&, int32_t*, cudaStream_t);
 DecodeLayout decode_layout(const flashloop_params*);
 int launch_decode_attn(const flashloop_params*, int, const flashloop_state*, flashloop_decode_state*, cudaStream_t);
 int launch_decode_select(const flashloop_params*, flashloop_decode_state*, cudaStream_t);
@@ -340,6 +341,13 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
   a.o = st->O;
   a.scale_log2 = 1.4426950408889634f / sqrtf((float)p->head_dim);
   a.err = st->err_word;
+  if (!dense) {
+    // each active row's causal prefix of the selection, per head
+    int32_t* cnt = ws_ptr<int32_t>(st->workspace, workspace_layout(p).row_cnt);
+    rc = launch_attn_row_counts(a, cnt, s);
+    if (rc != FLASHLOOP_OK) return rc;
+    a.row_cnt = cnt;
+  }
   if (p->fixed_mass && !dense) {
     // fixed-mass form: a statistics pass (frame m' and factor g per row), then the update
     a.g_in = st->G[prev];

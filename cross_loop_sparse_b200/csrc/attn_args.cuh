@@ -30,6 +30,7 @@ struct AttnArgs {
   int mode;                     // 0 running state, 1 / 2 fixed-mass statistics / update pass
   const float* g_in;            // [H, S] selected-column factor of loop r-1 (fixed-mass passes)
   float* g_out;                 // [H, S] (statistics pass; the dense loop writes 1 when set)
+  const int32_t* row_cnt;       // [H, row_cap]: selected columns <= the row's token (required with cols)
 };
 
 struct ColmassArgs {

@@ -85,16 +85,18 @@ struct AtArgs {
   uint16_t* o;
   float scale_log2;
   int32_t* err;
+  const int32_t* row_cnt;  // [H, row_cap] selected columns <= the row's token (with cols; NULL when dense)
 };
 
-__device__ __forceinline__ int at_count_le(const int32_t* cols, int n, int tok) {
-  int lo = 0, hi = n;
-  while (lo < hi) {
-    const int mid = (lo + hi) >> 1;
-    if (__ldg(cols + mid) <= tok) lo = mid + 1;
-    else hi = mid;
-  }
-  return lo;
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
+}
+
+// Selected columns at or before active row a's token, for head h: from the
+// precomputed counts, or the identity selection (dense).
+__device__ __forceinline__ int at_row_count(const AtArgs& g, int h, int a, int tok) {
+  if (g.row_cnt) return __ldg(g.row_cnt + (size_t)h * g.row_cap + a);
+  return min(tok + 1, g.kc);
 }
 
 // Number of column tiles work item (h, rt) needs: columns up to its last row token.
@@ -103,8 +105,7 @@ __device__ __forceinline__ int at_tiles(const AtArgs& g, int h, int rt, int n_ro
   int tok = g.rows ? __ldg(g.rows + last) : last;
   if (tok < 0) return 0;
   if (tok >= g.S) tok = g.S - 1;
-  const int nc = g.cols ? at_count_le(g.cols + (size_t)h * g.kc, g.kc, tok) : min(tok + 1, g.kc);
-  return (nc + kAtCols - 1) / kAtCols;
+  return (at_row_count(g, h, last, tok) + kAtCols - 1) / kAtCols;
 }
 
 template <int DH, int MODE>
@@ -395,34 +396,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(q_ready);
+        // bring the next item's rows (this thread's q and half of N) into L2
+        // while this item runs: they are the item switch's loads
+        const int item_next = item + gridDim.x;
+        if (item_next < total) {
+          const int hn = item_next / row_tiles, an = (item_next % row_tiles) * kAtRows + row;
+          const int tn = an < n_rows ? (g.rows ? __ldg(g.rows + an) : an) : -1;
+          if (tn >= 0 && tn < g.S) {
+            if (half == 0 || has_old) {
+              const uint16_t* qn = (half == 0 ? g.q_new : g.q_old) + (size_t)tn * HD + (size_t)hn * DH;
+#pragma unroll
+              for (int c = 0; c < DH * 2; c += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(qn) + c);
+            }
+            if (!g.dense && !stats) {
+              const float* nn = g.n_in + ((size_t)hn * g.S + tn) * DH + half * kHalfCols;
+#pragma unroll
+              for (int c = 0; c < kHalfCols * 4; c += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(nn) + c);
+            }
+          }
+        }
       }
 
-      const int32_t* hcols = g.cols ? g.cols + (size_t)h * g.kc : nullptr;
-      int wmin = tok < 0 ? 0x7fffffff : tok;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) wmin = min(wmin, __shfl_xor_sync(0xffffffffu, wmin, o));
+      // the row's causal prefix of the selection (columns ascend, so the
+      // valid columns of every tile form a prefix of it)
+      const int nc_row = tok < 0 ? 0 : at_row_count(g, h, a, tok);
       for (int t = 0; t < nt; ++t, ++u) {
         const uint32_t b = u & 1;
         const int c0 = t * kAtCols;
-        const int c_end = min(c0 + kAtCols, g.kc);
-        const int last_tok = hcols ? __ldg(hcols + c_end - 1) : c_end - 1;
-        const bool need_mask = (c0 + kAtCols > g.kc) || (last_tok > wmin);
-        // the valid columns of this tile for this row form a prefix (columns ascend)
-        int nvalid = kAtCols;
-        if (need_mask) {
-          if (tok < 0) {
-            nvalid = 0;
-          } else {
-            int lo = c0, hi = c_end;
-            while (lo < hi) {
-              const int mid = (lo + hi) >> 1;
-              const int ct = hcols ? __ldg(hcols + mid) : mid;
-              if (ct <= tok) lo = mid + 1;
-              else hi = mid;
-            }
-            nvalid = lo - c0;
-          }
-        }
+        const int nvalid = min(max(nc_row - c0, 0), kAtCols);
         const int first = half * 32;  // this thread's first column in the tile
         wait_or_die(&s_full[b], (u >> 1) & 1);
         uint32_t rn[32], ro[32];
@@ -922,6 +923,45 @@ colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, floa
   }
 }
 
+// Per head and active row: how many of the head's selected columns lie at or
+// before the row's token - the row's causal prefix of the ascending
+// selection.  The attention kernels take their tile counts and masks from it
+// instead of searching the selection at every work item.  An index outside
+// [0, S) counts 0 (the attention kernels report it).
+__global__ void __launch_bounds__(256)
+attn_row_counts_kernel(const int32_t* __restrict__ rows, const int32_t* __restrict__ n_rows_ptr, int row_cap, int S,
+                       int H, const int32_t* __restrict__ cols, int kc, int32_t* __restrict__ out) {
+  int n_rows = n_rows_ptr ? *n_rows_ptr : S;
+  if (n_rows > row_cap) n_rows = row_cap;
+  if (n_rows < 0) n_rows = 0;
+  const long long total = (long long)H * n_rows;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < total;
+       i += (long long)gridDim.x * blockDim.x) {
+    const int h = (int)(i / n_rows), a = (int)(i % n_rows);
+    const int tok = rows ? __ldg(rows + a) : a;
+    int lo = 0;
+    if (tok >= 0 && tok < S) {
+      const int32_t* c = cols + (size_t)h * kc;
+      int hi = kc;
+      while (lo < hi) {
+        const int mid = (lo + hi) >> 1;
+        if (__ldg(c + mid) <= tok) lo = mid + 1;
+        else hi = mid;
+      }
+    }
+    out[(size_t)h * row_cap + a] = lo;
+  }
+}
+
+int launch_attn_row_counts(const AttnArgs& a, int32_t* out, cudaStream_t stream) {
+  const long long total = (long long)a.H * a.row_cap;
+  int grid = (int)((total + 255) / 256);
+  if (grid > 148 * 8) grid = 148 * 8;
+  if (grid < 1) grid = 1;
+  attn_row_counts_kernel<<<grid, 256, 0, stream>>>(a.rows, a.n_rows, a.row_cap, a.S, a.H, a.cols, a.kc, out);
+  return launch_status();
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1009,6 +1049,7 @@ int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scr
 
 // K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.
 int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream);
+int launch_attn_dual(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream);
 
 int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
@@ -1018,6 +1059,9 @@ int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaSt
     const int rc = launch_attn_pair(p, a, kcp, stream);
     if (rc != FLASHLOOP_ERR_UNSUPPORTED) return rc;
   }
+  // the dense loop: two row tiles per CTA sharing every K / V tile (attn_dual.cu)
+  if (a.mode == kAtRunning && a.dense) return launch_attn_dual(p, a, kcp, stream);
+  if (a.cols != nullptr && a.row_cnt == nullptr) return FLASHLOOP_ERR_INVALID_ARG;
   // the row warps move q, N and O rows in 32-byte accesses
   const void* aligned32[] = {a.q_new, a.q_old, a.n_in, a.n_out, a.o};
   for (const void* ptr : aligned32)
@@ -1038,7 +1082,7 @@ int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaSt
   g.row_cap = a.row_cap; g.cols = a.cols; g.q_new = a.q_new; g.q_old = a.q_old; g.m_in = a.m_in;
   g.z_in = a.z_in; g.n_in = a.n_in; g.m_out = a.m_out; g.z_out = a.z_out; g.n_out = a.n_out; g.o = a.o;
   g.scale_log2 = a.scale_log2; g.err = a.err;
-  g.g_in = a.g_in; g.g_out = a.g_out;
+  g.g_in = a.g_in; g.g_out = a.g_out; g.row_cnt = a.row_cnt;
   const int max_items = ((a.row_cap + kAtRows - 1) / kAtRows) * H;
   int grid = at_sm_count();
   if (grid > max_items) grid = max_items;

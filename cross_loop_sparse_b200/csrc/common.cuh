@@ -65,6 +65,7 @@ struct Workspace {
   size_t cm_q;      // column-mass scratch: fp16 q of the rows [H, S, dh] (room for float [S, H, dh])
   size_t cm_rows;   // column-mass scratch: row max (log2), 1/Z [H, S] each, row tokens [S]
   size_t cols_kv;   // fp16 dequantised selected columns: 4 x [H, kmax, dh] or 2 x [H, S, dh]
+  size_t row_cnt;   // int32 [H, S]: per head and active row, the selected columns at or before its token
   size_t total;
 };
 
@@ -92,6 +93,7 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   size_t sel = 4 * H * (size_t)pad8(max_topk(p)) * dh;
   size_t dense = 2 * H * (size_t)pad8(p->seq) * dh;
   w.cols_kv = off; off = align256(off + (sel > dense ? sel : dense) * sizeof(__half));
+  w.row_cnt = off; off = align256(off + H * S * sizeof(int32_t));
   w.total = off;
   return w;
 }
