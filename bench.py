@@ -33,9 +33,9 @@ METRIC = "loop-step tokens/s at S=32K,R=4; HBM GB/s and tensor-pipe % of B200 pe
 DECODE_METRIC = "decode tokens/s (B sequences x 1 token x R loops) at S_ctx=32K,R=4; HBM GB/s of B200 peak"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures summarised
-# under profiles/; None once the kernel changes until it is re-captured (the 737.8 MB capture
-# predates the kernel's fixed-mass template modes).
-ATTN_LOOP2_TRAFFIC = {"attn_tc_kernel<128>": None}
+# under profiles/; None once the kernel changes until it is re-captured.
+ATTN_LOOP2_TRAFFIC = {"attn_dual_kernel<128>": None}
+ATTN_KERNEL = "attn_dual_kernel<128>"
 # captured on 2 sequences and scaled by 4 (traffic in proportion to the columns read)
 DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": 1169.5e6}
 
@@ -58,6 +58,16 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return PEAKS_FALLBACK, "fallback"
+
+
+def run_config(cfg, world, active_tokens, pairs):
+    """The config object of both arms' lines (identical keys and values for
+    the same workload, so the two lines compare)."""
+    return {"workload": workload_desc(cfg),
+            "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
+            "parallelism": f"one sequence per rank, {world} rank(s), no exchange",
+            "active_tokens": {f"loop{r}": int(n) for r, n in sorted(active_tokens.items())},
+            "attention_pairs": {f"loop{r}": int(v) for r, v in sorted(pairs.items())}}
 
 
 def workload_desc(cfg):
@@ -232,12 +242,13 @@ def run_cuda(args, cfg, rank, world, local_rank):
     achieved = flop2 / (ms2 * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": None if (args.fixed_mass or args.sm_pairs) else ATTN_LOOP2_TRAFFIC.get("attn_tc_kernel<128>"),
+                "traffic": None if (args.fixed_mass or args.sm_pairs) else ATTN_LOOP2_TRAFFIC.get(ATTN_KERNEL),
                 "kernel": ("attn_tc_kernel<128> statistics + update passes, loop 2 (fixed-mass form, tcgen05)"
                            if args.fixed_mass else
                            "attn_pair_kernel<128>, loop-2 launch (sparse attention update, tcgen05 on SM pairs)"
                            if args.sm_pairs else
-                           "attn_tc_kernel<128>, loop-2 launch (sparse attention update, tcgen05)"),
+                           f"{ATTN_KERNEL}, loop-2 launch (sparse attention update, tcgen05, two row tiles "
+                           "per CTA)"),
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
                 "per_loop": {f"loop{r}": {"ms": round(statistics.mean(v), 4),
@@ -310,24 +321,38 @@ def run_cuda(args, cfg, rank, world, local_rank):
 
     tokens = S * (R - 1) * world
     ms_step = ms / args.steps
+    # Whole step against the tensor roofline: attention 8*dh FLOP per causal-valid
+    # pair plus the gathered projections 8*d^2 FLOP per active row (QKV 6, W_o 2).
+    n_act = {r: int(st["n_active"][r - 1].item()) for r in range(2, R + 1)}
+    attn_flop = sum(8 * cfg.head_dim * pairs[r] for r in range(2, R + 1))
+    gemm_flop = sum(8 * d * d * n_act[r] for r in range(2, R + 1))
+    step_tflops = (attn_flop + gemm_flop) / (ms / args.steps * 1e-3) / 1e12
+    step_roofline = {"bound": "tensor", "flop": int(attn_flop + gemm_flop), "attention_flop": int(attn_flop),
+                     "projection_flop": int(gemm_flop), "achieved": round(step_tflops, 2),
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(step_tflops / peaks["bf16_tflops"], 4),
+                     "roofline_ms": round((attn_flop + gemm_flop) / (peaks["bf16_tflops"] * 1e12) * 1e3, 4)}
+    if args.fixed_mass or args.sm_pairs:
+        # a variant of the update: the config says so (the reference arm has no such line)
+        variant = "fixed-mass form of the update" if args.fixed_mass else "attention on SM pairs"
+    else:
+        variant = None
     out = {
         "metric": METRIC, "value": round(tokens / (ms_step * 1e-3), 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded workload generator; random-init weights of the stated shape)",
-        "config": {"workload": workload_desc(cfg) + (", fixed-mass form of the update" if args.fixed_mass else "")
-                   + (", attention on SM pairs" if args.sm_pairs else ""),
-                   "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
-                   "parallelism": f"one sequence per GPU, {world} GPU(s), no exchange",
-                   "active_tokens": {f"loop{r}": int(st['n_active'][r - 1].item()) for r in range(2, R + 1)},
-                   "attention_pairs": {f"loop{r}": pairs[r] for r in range(2, R + 1)}},
+        "config": run_config(cfg, world, {r: int(st['n_active'][r - 1].item()) for r in range(2, R + 1)}, pairs),
         "roofline": roofline,
+        "step_roofline": step_roofline,
         "e2e": {"value": round(tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": (R - 1) * S * d * 2, "d2h_bytes_per_step": S * d * 2,
                 "steps": e2e_steps},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clk,
     }
+    if variant:
+        out["config"]["workload"] += ", " + variant
     return out
 
 
@@ -579,8 +604,36 @@ class OracleSample:
             return os.cpu_count()
 
 
+class OracleFullStep:
+    """The CPU oracle over the whole workload: loops 2..R of one sequence on
+    every head, gate and output projection included, from a loop-1 state
+    computed once (untimed set-up)."""
+
+    def __init__(self, cfg):
+        import oracle as O
+        self.O, self.cfg = O, cfg
+        self.W = make_weights(cfg)
+        self.X, _ = make_hidden_states(cfg)
+        t = time.perf_counter()
+        self.base = O.OracleSequence(cfg, self.W, self.X, keep_history=False)
+        self.base.run_loop1()
+        self.setup_s = time.perf_counter() - t
+
+    def step(self):
+        import copy
+        orc = copy.deepcopy(self.base)
+        t = time.perf_counter()
+        for r in range(2, self.cfg.n_loops + 1):
+            orc.run_loop(r)
+        dt = time.perf_counter() - t
+        pairs = {r: attention_pairs(orc.active[r], orc.T[r]) for r in range(2, self.cfg.n_loops + 1)}
+        active = {r: orc.active[r].size for r in range(2, self.cfg.n_loops + 1)}
+        return dt, active, pairs
+
+
 def run_reference(args, cfg):
-    """The reference arm: the CPU oracle as it stands, on a bounded sample per step."""
+    """The reference arm: the CPU oracle as it stands.  Prefill: one full
+    step (every head), timed once; decode: a bounded sample per step."""
     if cfg.decode:
         smp = DecodeOracleSample(cfg)
         times, sample = [], ""
@@ -599,20 +652,23 @@ def run_reference(args, cfg):
                              "kind": "oracle", "sample": sample},
             "e2e": {"value": round(val, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         }
-    smp = OracleSample(cfg)
-    times, sample = [], ""
-    for i in range(args.warmup + args.steps):
-        t_est, sample = smp.step()
-        if i >= args.warmup:
-            times.append(t_est)
-    ms = statistics.mean(times) * 1e3
+    # A full step of the oracle takes about a minute on 16 cores (and its
+    # loop-1 set-up a few), so it is timed once, with no warm-up: the line
+    # reports the steps it timed, not the ones requested.
+    full = OracleFullStep(cfg)
+    dt, active, pairs = full.step()
+    ms = dt * 1e3
     tokens = cfg.seq * (cfg.n_loops - 1)
-    val = tokens / (ms * 1e-3)
+    val = tokens / dt
+    sample = (f"one full step: oracle loops 2..{cfg.n_loops} of one {cfg.seq}-token sequence on all "
+              f"{cfg.n_heads} heads (gate, projections, quantisation, selection, attention, W_o), "
+              f"{dt:.1f} s; loop-1 set-up {full.setup_s:.1f} s untimed")
     return {
         "impl": "reference", "metric": METRIC, "value": round(val, 2), "unit": "tokens/s", "n_gpus": 1,
-        "steps": len(times), "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+        "steps": 1, "warmup": 0, "requested": {"steps": args.steps, "warmup": args.warmup},
+        "ms_per_step": round(ms, 1), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": workload_desc(cfg), "parallelism": "CPU oracle, host cores"},
+        "config": run_config(cfg, 1, active, pairs),
         "cpu_baseline": {"value": round(val, 2), "unit": "tokens/s", "cores": OracleSample.cores(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(val, 2), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
