@@ -34,8 +34,8 @@ DECODE_METRIC = "decode tokens/s (B sequences x 1 token x R loops) at S_ctx=32K,
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures summarised
 # under profiles/; None once the kernel changes until it is re-captured.
-ATTN_LOOP2_TRAFFIC = {"attn_dual_kernel<128>": None}
-ATTN_KERNEL = "attn_dual_kernel<128>"
+ATTN_LOOP2_TRAFFIC = {"attn_tc_kernel<128>": None}
+ATTN_KERNEL = "attn_tc_kernel<128>"
 # captured on 2 sequences and scaled by 4 (traffic in proportion to the columns read)
 DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": 1169.5e6}
 
@@ -163,6 +163,30 @@ def run_cuda(args, cfg, rank, world, local_rank):
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
     torch.cuda.synchronize()
 
+    # Loop 1 (the dense producer of the base cache, the state and the column
+    # mass), timed on its own: it runs once per sequence, before the loop steps.
+    # Re-running it rewrites slot 0 with the same bytes.
+    def loop1(events):
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        ev[0].record(stream)
+        F.flashloop_qkv_quant(p, 1, xs[0], None, None, wqkv, st, st["q0"])
+        ev[1].record(stream)
+        F.flashloop_selcol_dequant(p, 1, st)
+        ev[2].record(stream)
+        F.flashloop_sparse_attn_update(p, 1, st, 1)
+        ev[3].record(stream)
+        F.flashloop_out_proj(p, st["O"], None, None, S, wo, st["Y"])
+        ev[4].record(stream)
+        events.append(ev)
+
+    l1_events = []
+    for i in range(4):
+        loop1(l1_events if i > 0 else [])
+    torch.cuda.synchronize()
+    l1 = {k: statistics.mean(e[a].elapsed_time(e[b]) for e in l1_events)
+          for k, a, b in (("ms", 0, 4), ("qkv_quant", 0, 1), ("rebuild", 1, 2), ("attention_colmass", 2, 3),
+                          ("out_proj", 3, 4))}
+
     launches_per_step = 0
     attn_events = []
 
@@ -247,8 +271,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
                            if args.fixed_mass else
                            "attn_pair_kernel<128>, loop-2 launch (sparse attention update, tcgen05 on SM pairs)"
                            if args.sm_pairs else
-                           f"{ATTN_KERNEL}, loop-2 launch (sparse attention update, tcgen05, two row tiles "
-                           "per CTA)"),
+                           f"{ATTN_KERNEL}, loop-2 launch (sparse attention update, tcgen05)"),
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
                 "per_loop": {f"loop{r}": {"ms": round(statistics.mean(v), 4),
@@ -332,6 +355,16 @@ def run_cuda(args, cfg, rank, world, local_rank):
                      "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                      "frac": round(step_tflops / peaks["bf16_tflops"], 4),
                      "roofline_ms": round((attn_flop + gemm_flop) / (peaks["bf16_tflops"] * 1e12) * 1e3, 4)}
+    # loop 1: projections 8*d^2 per token, dense causal attention 4*dh per pair and
+    # head, the column mass's score recomputation 2*dh per pair and head
+    pairs1 = S * (S + 1) // 2 * cfg.n_heads
+    l1_flop = 8 * d * d * S + 6 * cfg.head_dim * pairs1
+    loop1_line = {"ms": round(l1["ms"], 4), "tokens_per_s": round(S / (l1["ms"] * 1e-3), 1),
+                  "kernels_ms": {k: round(v, 4) for k, v in l1.items() if k != "ms"},
+                  "flop": int(l1_flop), "achieved": round(l1_flop / (l1["ms"] * 1e-3) / 1e12, 2),
+                  "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                  "frac": round(l1_flop / (l1["ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
+                  "roofline_ms": round(l1_flop / (peaks["bf16_tflops"] * 1e12) * 1e3, 4)}
     if args.fixed_mass or args.sm_pairs:
         # a variant of the update: the config says so (the reference arm has no such line)
         variant = "fixed-mass form of the update" if args.fixed_mass else "attention on SM pairs"
@@ -345,6 +378,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
         "config": run_config(cfg, world, {r: int(st['n_active'][r - 1].item()) for r in range(2, R + 1)}, pairs),
         "roofline": roofline,
         "step_roofline": step_roofline,
+        "loop1": loop1_line,
         "e2e": {"value": round(tokens / (e2e_ms / e2e_steps * 1e-3), 1), "unit": "tokens/s",
                 "h2d_bytes_per_step": (R - 1) * S * d * 2, "d2h_bytes_per_step": S * d * 2,
                 "steps": e2e_steps},

@@ -145,6 +145,34 @@ __device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits
   *scale = sbits;
 }
 
+__device__ __forceinline__ void prefetch_l2(const void* p) {
+  asm volatile("prefetch.global.L2 [%0];\n" ::"l"(p));
+}
+
+// The cache lines the fused quantiser will read for one row of a K or V tile
+// (the previous loops' reconstruction of the heads in this thread's half:
+// base codes and scales, then each earlier residual row present and its
+// scales), requested into L2 while the thread waits for the tile's
+// accumulator, so that the epilogue's loads need not go to DRAM.
+template <int DH>
+__device__ __forceinline__ void prefetch_recon_row(const TcGemmArgs& g, const KVStreams& kv, int t, int h0,
+                                                   int heads) {
+  const int H = g.d_model / DH;
+  for (int k = 0; k < heads; ++k) {
+    const size_t th = (size_t)t * H + h0 + k;
+#pragma unroll
+    for (int c = 0; c < DH; c += 128) prefetch_l2(kv.base_codes + th * DH + c);
+  }
+  prefetch_l2(kv.base_scales + ((size_t)t * H + h0) * (DH / 32));
+  for (int l = 2; l < g.loop; ++l) {
+    const int sl = g.lt.slot[l - 1][t];
+    if (sl < 0) continue;
+    const int rb = DH * g.lt.bits[l - 1] / 8;
+    for (int k = 0; k < heads; ++k) prefetch_l2(kv.res_codes[l - 1] + ((size_t)sl * H + h0 + k) * rb);
+    prefetch_l2(kv.res_scales[l - 1] + ((size_t)sl * H + h0) * (DH / 32));
+  }
+}
+
 template <int DH>
 __device__ __forceinline__ void epilogue_tile(const TcGemmArgs& g, int mode, int m0, int n0, int row,
                                               int n_rows, uint32_t tbase, int half) {
@@ -429,6 +457,23 @@ tc_gemm_kernel(const __grid_constant__ CUtensorMap tmap_b, TcGemmArgs g, int mod
     for (int tile = blockIdx.x; tile < total && !*abort_flag; tile += gridDim.x, ++it) {
       const int buf = it & 1;
       const uint32_t acc_phase = (it >> 1) & 1;
+      if (mode == kTcQkvQuant && g.loop >= 2) {
+        // while the accumulator is computed: this row's earlier codes into L2
+        const int n0p = (tile % n_tiles) * kTcBN, section = n0p / g.d_model;
+        const int a = (tile / n_tiles) * kTcBM + row;
+        if (section >= 1 && a < n_rows) {
+          const int t = g.rows ? g.rows[a] : a;
+          if (t >= 0 && t < g.S) {
+            prefetch_recon_row<DH>(g, section == 1 ? g.Ks : g.Vs, t,
+                                   (n0p - section * g.d_model + half * 128) / DH, 128 / DH);
+            if (section == 1) {  // the row's RoPE table entries (keys are rotated)
+              const float* cs = g.rope_cs + (size_t)t * DH;
+#pragma unroll
+              for (int c = 0; c < DH; c += 32) prefetch_l2(cs + c);
+            }
+          }
+        }
+      }
       if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[buf], acc_phase))) {
         set_error(g.err, kDevErrTimeout);
         *abort_flag = 1;
