@@ -157,11 +157,27 @@ def run_cuda(args, cfg, rank, world, local_rank):
     to_dev = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).to(dev)  # noqa: E731
     xs = [to_dev(x) for x in X]
     wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
-    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass, attn_pairs=args.sm_pairs)
+    paper = args.kv_scheme == "paper"
+    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass, attn_pairs=args.sm_pairs, kv_scheme=args.kv_scheme)
     st = F.FlashLoopState(p, device=dev)
     S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
     torch.cuda.synchronize()
+    if paper:
+        kf = torch.empty((S, d), dtype=torch.float32, device=dev)
+        vf = torch.empty_like(kf)
+
+    def project_quant(r, x, act, n_act, cap, q_out):
+        """Projection of the loop's active rows with its K/V quantisation:
+        fused into the GEMM epilogue (INT8 + INT4/INT2 streams), or the
+        gathered projection then the asymmetric INT4 quantiser (the pages'
+        setting).  Returns the launches made."""
+        if not paper:
+            F.flashloop_qkv_quant(p, r, x, act, n_act, wqkv, st, q_out)
+            return 1
+        F.flashloop_qkv_gathered(p, x, act, n_act, cap, wqkv, st["rope_cs"], q_out, kf, vf)
+        F.flashloop_paper_kv_quant(p, r, kf, vf, act, n_act, st)
+        return 4
 
     # Loop 1 (the dense producer of the base cache, the state and the column
     # mass), timed on its own: it runs once per sequence, before the loop steps.
@@ -169,7 +185,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
     def loop1(events):
         ev = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
         ev[0].record(stream)
-        F.flashloop_qkv_quant(p, 1, xs[0], None, None, wqkv, st, st["q0"])
+        project_quant(1, xs[0], None, None, S, st["q0"])
         ev[1].record(stream)
         F.flashloop_selcol_dequant(p, 1, st)
         ev[2].record(stream)
@@ -199,8 +215,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
             n_prev = None if r == 2 else st["n_active"][r - 2:]
             F.flashloop_gate(p, xs[r - 1], xs[r - 2], prev, n_prev, p.capacity[r - 2] if r > 2 else S,
                              act, st[f"slot{r}"], n_act, p.capacity[r - 1], st["workspace"], st["err"])
-            F.flashloop_qkv_quant(p, r, xs[r - 1], act, n_act, wqkv, st, st[f"q{st.q_slot(r)}"])
-            n += 2
+            n += 1 + project_quant(r, xs[r - 1], act, n_act, p.capacity[r - 1], st[f"q{st.q_slot(r)}"])
             if F.flashloop_selection_loop(p, r) == r:
                 src = st["colmass0"] if r == 2 else st["colmass1"]
                 F.flashloop_topk_columns(p, src, None, 0, p.topk[r - 1], st[f"cols{r}"])
@@ -365,11 +380,15 @@ def run_cuda(args, cfg, rank, world, local_rank):
                   "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
                   "frac": round(l1_flop / (l1["ms"] * 1e-3) / 1e12 / peaks["bf16_tflops"], 4),
                   "roofline_ms": round(l1_flop / (peaks["bf16_tflops"] * 1e12) * 1e3, 4)}
-    if args.fixed_mass or args.sm_pairs:
-        # a variant of the update: the config says so (the reference arm has no such line)
-        variant = "fixed-mass form of the update" if args.fixed_mass else "attention on SM pairs"
-    else:
-        variant = None
+    variants = []
+    # a variant of the path: the config says so (the reference arm has no such line)
+    if args.fixed_mass:
+        variants.append("fixed-mass form of the update")
+    if args.sm_pairs:
+        variants.append("attention on SM pairs")
+    if paper:
+        variants.append("the pages' cache setting (INT4 asymmetric groups of 64, 64-token bf16 tail)")
+    variant = ", ".join(variants) or None
     out = {
         "metric": METRIC, "value": round(tokens / (ms_step * 1e-3), 1), "unit": "tokens/s",
         "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -387,7 +406,28 @@ def run_cuda(args, cfg, rank, world, local_rank):
     }
     if variant:
         out["config"]["workload"] += ", " + variant
+    out["config"]["kv_cache_bytes"] = kv_cache_bytes(cfg, st, paper)
     return out
+
+
+def kv_cache_bytes(cfg, st, paper):
+    """Bytes of the K and V streams after loops 1..R (codes, fp16 scales and
+    minima, bf16 tail values), from the active lists."""
+    S, H, dh, R = cfg.seq, cfg.n_heads, cfg.head_dim, cfg.n_loops
+    E = H * dh
+    n = [S] + [int(st["n_active"][r - 1].item()) for r in range(2, R + 1)]
+    if not paper:   # INT8 base, INT4 / INT2 residuals, an fp16 scale per group of 32
+        return int(sum(2 * (nr * E * cfg.bits[i] // 8 + nr * E // 32 * 2) for i, nr in enumerate(n)))
+    tail = min(64, S)
+    body = S - tail
+    total = 0
+    for r, nr in enumerate(n, start=1):
+        nb = body if r == 1 else int((st[f"active{r}"][:nr] < body).sum().item())
+        nt = nr - nb
+        groups_v = nb * E // 64
+        groups_k = (nb + 63) // 64 * E
+        total += 2 * (nb * E // 2) + 4 * (groups_v + groups_k) + 2 * nt * E * 2
+    return int(total)
 
 
 # ----------------------------------------------------------------------------- decode (CUDA arm)
@@ -722,6 +762,9 @@ def main():
                          "oracle keeps explicit S x S distributions)")
     ap.add_argument("--sm-pairs", action="store_true",
                     help="prefill workloads: the running update on SM pairs (cta_group::2)")
+    ap.add_argument("--kv-scheme", choices=["spec", "paper"], default="spec",
+                    help="prefill workloads: K/V streams as INT8 + INT4/INT2 symmetric residuals (spec) or the "
+                         "pages' own setting, INT4 asymmetric groups of 64 with a 64-token bf16 tail (paper)")
     ap.add_argument("--batch", type=int, default=None,
                     help="decode workloads: sequences per GPU (a smaller case for profiler captures)")
     args = ap.parse_args()
@@ -732,6 +775,8 @@ def main():
         cfg = cfg.with_(batch=args.batch)
     if args.fixed_mass and (cfg.decode or args.impl != "cuda"):
         ap.error("--fixed-mass applies to the CUDA arm on prefill workloads only")
+    if args.kv_scheme == "paper" and (cfg.decode or args.impl != "cuda" or args.fixed_mass):
+        ap.error("--kv-scheme paper applies to the CUDA arm's running update on prefill workloads only")
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -750,7 +795,7 @@ def main():
         torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
     out = (run_decode_cuda if cfg.decode else run_cuda)(args, cfg, rank, world, local_rank)
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fixed_mass:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.fixed_mass and args.kv_scheme == "spec":
         if cfg.decode:
             t_est, sample = DecodeOracleSample(cfg).step()
             value = round(cfg.batch / t_est, 4)

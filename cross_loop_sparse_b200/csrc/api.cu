@@ -43,6 +43,10 @@ int launch_decode_qkv(const flashloop_params*, int, const uint16_t*, const uint1
                       cudaStream_t);
 int launch_decode_out(const flashloop_params*, const uint16_t*, flashloop_decode_state*, cudaStream_t);
 int launch_colmass_tc(const flashloop_params*, const ColmassArgs&, void*, void*, cudaStream_t);
+int launch_paper_quant(const flashloop_params*, int, const float*, const float*, const int32_t*, const int32_t*,
+                       int, const flashloop_state*, cudaStream_t);
+int launch_paper_selcol(const flashloop_params*, int, const int32_t*, int, int, const flashloop_state*, __half*,
+                        __half*, __half*, __half*, cudaStream_t);
 
 // ---------------------------------------------------------------------------
 // checks
@@ -72,10 +76,11 @@ static int check_params(const flashloop_params* p) {
   if (p->d_model != p->n_heads * p->head_dim) return FLASHLOOP_ERR_INVALID_ARG;
   if (p->d_model % 128 != 0) return FLASHLOOP_ERR_UNSUPPORTED;
   if (!(p->tau >= 0.f) || !(p->rope_theta > 0.f)) return FLASHLOOP_ERR_INVALID_ARG;
-  if (p->bits[0] != 8) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (p->kv_scheme != 0 && p->kv_scheme != 1) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (p->kv_scheme == 0 && p->bits[0] != 8) return FLASHLOOP_ERR_UNSUPPORTED;
   for (int r = 2; r <= p->n_loops; ++r) {
     const int b = p->bits[r - 1];
-    if (b != 8 && b != 4 && b != 2) return FLASHLOOP_ERR_UNSUPPORTED;
+    if (p->kv_scheme == 0 && b != 8 && b != 4 && b != 2) return FLASHLOOP_ERR_UNSUPPORTED;
     const int k = p->topk[r - 1];
     if (k < 1 || k > p->seq) return FLASHLOOP_ERR_INVALID_ARG;
     if (r >= 3 && k > p->topk[r - 2]) return FLASHLOOP_ERR_INVALID_ARG;  // nested selection
@@ -210,6 +215,7 @@ int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const f
   int rc = check_common(p);
   if (rc != FLASHLOOP_OK) return rc;
   if (loop < 1 || loop > p->n_loops || !k_new || !v_new || !st) return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->kv_scheme != 0) return FLASHLOOP_ERR_UNSUPPORTED;  // see flashloop_paper_kv_quant
   if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
     return FLASHLOOP_ERR_INVALID_ARG;
   if (loop >= 2) {
@@ -231,6 +237,7 @@ int flashloop_qkv_quant(const flashloop_params* p, int32_t loop, const uint16_t*
   if (rc != FLASHLOOP_OK) return rc;
   if (loop < 1 || loop > p->n_loops || !x || !w_qkv || !st || !st->rope_cs)
     return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->kv_scheme != 0) return FLASHLOOP_ERR_UNSUPPORTED;  // the fused quantiser writes the INT8 / INT4 / INT2 streams
   if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
     return FLASHLOOP_ERR_INVALID_ARG;
   if (active != nullptr && n_active == nullptr) return FLASHLOOP_ERR_INVALID_ARG;
@@ -258,21 +265,37 @@ int flashloop_topk_columns(const flashloop_params* p, const float* mass, const i
   return launch_topk(p, mass, candidates, n_cand, k, out, nullptr, as_stream(stream));
 }
 
+// The pages' streams of loops 1..loop are present (params.kv_scheme == 1).
+static int check_paper_streams(const flashloop_params* p, const flashloop_state* st, int loop) {
+  if (!st->paper_k || !st->paper_v) return FLASHLOOP_ERR_INVALID_ARG;
+  for (const flashloop_paper_kv* kv : {st->paper_k, st->paper_v})
+    for (int r = 1; r <= loop; ++r)
+      if (!kv->codes[r - 1] || !kv->scale[r - 1] || !kv->minv[r - 1] || !kv->tail[r - 1])
+        return FLASHLOOP_ERR_INVALID_ARG;
+  (void)p;
+  return FLASHLOOP_OK;
+}
+
 static int check_state(const flashloop_params* p, const flashloop_state* st, int loop) {
   if (!st || !st->n_active || !st->O || !st->err_word || !st->workspace) return FLASHLOOP_ERR_INVALID_ARG;
   if (st->workspace_bytes < workspace_layout(p).total) return FLASHLOOP_ERR_INVALID_ARG;
   for (int i = 0; i < 3; ++i)
     if (!st->q[i] || !st->m[i] || !st->Z[i] || !st->N[i]) return FLASHLOOP_ERR_INVALID_ARG;
-  if (!st->colmass[0] || !st->k.base_codes || !st->v.base_codes) return FLASHLOOP_ERR_INVALID_ARG;
+  if (!st->colmass[0]) return FLASHLOOP_ERR_INVALID_ARG;
   if (p->fixed_mass)
     for (int i = 0; i < 3; ++i)
       if (!st->G[i]) return FLASHLOOP_ERR_INVALID_ARG;
   for (int r = 2; r <= loop; ++r)
     if (!st->active[r - 1] || !st->slot[r - 1]) return FLASHLOOP_ERR_INVALID_ARG;
-  for (int r = 2; r <= loop; ++r)
-    if (!st->k.res_codes[r - 1] || !st->v.res_codes[r - 1] || !st->k.res_scales[r - 1] ||
-        !st->v.res_scales[r - 1])
-      return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->kv_scheme == 1) {
+    if (check_paper_streams(p, st, loop) != FLASHLOOP_OK) return FLASHLOOP_ERR_INVALID_ARG;
+  } else {
+    if (!st->k.base_codes || !st->v.base_codes) return FLASHLOOP_ERR_INVALID_ARG;
+    for (int r = 2; r <= loop; ++r)
+      if (!st->k.res_codes[r - 1] || !st->v.res_codes[r - 1] || !st->k.res_scales[r - 1] ||
+          !st->v.res_scales[r - 1])
+        return FLASHLOOP_ERR_INVALID_ARG;
+  }
   if (loop >= 2) {
     const int sel = flashloop_selection_loop(p, loop);
     if (!st->cols[sel - 1]) return FLASHLOOP_ERR_INVALID_ARG;
@@ -313,8 +336,27 @@ int flashloop_selcol_dequant(const flashloop_params* p, int32_t loop, flashloop_
   rc = check_state(p, st, loop);
   if (rc != FLASHLOOP_OK) return rc;
   const ColBuffers b = col_buffers(p, loop, st);
+  if (p->kv_scheme == 1)
+    return launch_paper_selcol(p, loop, b.cols, b.kc, b.kcp, st, b.k_old, b.k_new, b.v_old, b.v_new,
+                               as_stream(stream));
   return launch_selcol_dequant(p, loop, b.cols, b.kc, b.kcp, st, b.k_old, b.k_new, b.v_old, b.v_new,
                                as_stream(stream));
+}
+
+int flashloop_paper_kv_quant(const flashloop_params* p, int32_t loop, const float* k_new, const float* v_new,
+                             const int32_t* active, const int32_t* n_active, flashloop_state* st, void* stream) {
+  int rc = check_common(p);
+  if (rc != FLASHLOOP_OK) return rc;
+  if (p->kv_scheme != 1) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (loop < 1 || loop > p->n_loops || !k_new || !v_new || !st || !st->err_word) return FLASHLOOP_ERR_INVALID_ARG;
+  if (check_paper_streams(p, st, loop) != FLASHLOOP_OK) return FLASHLOOP_ERR_INVALID_ARG;
+  if (loop >= 2) {
+    if (!active || !n_active) return FLASHLOOP_ERR_INVALID_ARG;
+    for (int l = 2; l <= loop; ++l)
+      if (!st->slot[l - 1]) return FLASHLOOP_ERR_INVALID_ARG;
+  }
+  return launch_paper_quant(p, loop, k_new, v_new, loop == 1 ? nullptr : active, loop == 1 ? nullptr : n_active,
+                            capacity_of(p, loop), st, as_stream(stream));
 }
 
 int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashloop_state* st,
@@ -401,8 +443,17 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
   cudaStream_t s = as_stream(stream);
   const int cur = slot_of_loop(loop);
   const int cap = capacity_of(p, loop);
+  // the pages' cache setting: the projection writes float32 K / V of the active
+  // rows to the workspace, then the asymmetric quantiser codes them
+  float* kf = p->kv_scheme == 1 ? ws_ptr<float>(st->workspace, workspace_layout(p).kv_f32) : nullptr;
+  float* vf = kf ? kf + (size_t)p->seq * p->d_model : nullptr;
   if (loop == 1) {
-    rc = launch_qkv_quant_gemm(p, 1, x_cur, nullptr, nullptr, p->seq, w_qkv, st, st->q[0], s);
+    if (p->kv_scheme == 1) {
+      rc = launch_qkv_gemm(p, x_cur, nullptr, nullptr, p->seq, w_qkv, st->rope_cs, st->q[0], kf, vf, st->err_word, s);
+      if (rc == FLASHLOOP_OK) rc = launch_paper_quant(p, 1, kf, vf, nullptr, nullptr, p->seq, st, s);
+    } else {
+      rc = launch_qkv_quant_gemm(p, 1, x_cur, nullptr, nullptr, p->seq, w_qkv, st, st->q[0], s);
+    }
     if (rc != FLASHLOOP_OK) return rc;
     rc = flashloop_selcol_dequant(p, 1, st, stream);
     if (rc != FLASHLOOP_OK) return rc;
@@ -421,7 +472,12 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
     rc = launch_gate(p, x_cur, x_prev, prev_act, n_prev, capacity_of(p, loop - 1), act,
                      st->slot[loop - 1], n_act, cap, st->workspace, st->err_word, s);
   if (rc != FLASHLOOP_OK) return rc;
-  rc = launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, st->q[cur], s);
+  if (p->kv_scheme == 1) {
+    rc = launch_qkv_gemm(p, x_cur, act, n_act, cap, w_qkv, st->rope_cs, st->q[cur], kf, vf, st->err_word, s);
+    if (rc == FLASHLOOP_OK) rc = launch_paper_quant(p, loop, kf, vf, act, n_act, cap, st, s);
+  } else {
+    rc = launch_qkv_quant_gemm(p, loop, x_cur, act, n_act, cap, w_qkv, st, st->q[cur], s);
+  }
   if (rc != FLASHLOOP_OK) return rc;
   const int sel = flashloop_selection_loop(p, loop);
   if (sel == loop && loop == 2 && p->seq > 49152) return FLASHLOOP_ERR_UNSUPPORTED;
@@ -455,6 +511,7 @@ int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x
   if (rc != FLASHLOOP_OK) return rc;
   if (loop < 1 || loop > p->n_loops || !x_cur || !w_qkv || !st || !st->rope_cs || !st->err_word)
     return FLASHLOOP_ERR_INVALID_ARG;
+  if (p->kv_scheme != 0) return FLASHLOOP_ERR_UNSUPPORTED;  // decode contexts keep the INT8 / INT4 / INT2 streams
   if (!st->k.base_codes || !st->k.base_scales || !st->v.base_codes || !st->v.base_scales)
     return FLASHLOOP_ERR_INVALID_ARG;
   cudaStream_t s = as_stream(stream);
@@ -489,6 +546,7 @@ static int check_decode_params(const flashloop_params* p) {
   if (rc != FLASHLOOP_OK) return rc;
   if (p->batch < 1 || p->batch > 64) return FLASHLOOP_ERR_INVALID_ARG;
   if (p->fixed_mass) return FLASHLOOP_ERR_UNSUPPORTED;  // decode keeps the running (m, N, Z) form
+  if (p->kv_scheme != 0) return FLASHLOOP_ERR_UNSUPPORTED;  // decode reads the INT8 / INT4 / INT2 streams
   const int hd = p->n_heads * p->head_dim, hg = hd / 32;
   if (hd % 256 != 0 || 256 % hg != 0 || hg % 8 != 0) return FLASHLOOP_ERR_UNSUPPORTED;
   if (p->n_loops >= 2 && p->topk[1] > p->seq + 1) return FLASHLOOP_ERR_INVALID_ARG;

@@ -108,6 +108,149 @@ __device__ __forceinline__ int at_tiles(const AtArgs& g, int h, int rt, int n_ro
   return (at_row_count(g, h, last, tok) + kAtCols - 1) / kAtCols;
 }
 
+// Barriers and the abort flag shared by a block's roles.
+struct AtBars {
+  uint64_t* kv_full;   // [stages]
+  uint64_t* kv_empty;  // [stages]
+  uint64_t* s_full;    // [2]
+  uint64_t* p_full;    // [2]
+  uint64_t* pv_done;   // [2]
+  uint64_t* q_ready;   // [1]
+  volatile int* abort_flag;
+};
+
+// Load role (one thread): the K (64 x DH) and V^T (DH x 64) tiles, new and
+// old, of every work item into the ring of stages by TMA.
+template <int DH, int MODE>
+__device__ __forceinline__ void at_load_role(uint8_t* smem, const AtBars& B, const CUtensorMap* tkn,
+                                             const CUtensorMap* tko, const CUtensorMap* tvn, const CUtensorMap* tvo,
+                                             const AtArgs& g, int n_rows, int row_tiles, int total, bool has_old,
+                                             int lane) {
+  using C = AtCfg<DH>;
+  if (lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    constexpr bool load_v = MODE != kAtFixedMassStats;
+    const uint32_t bytes = (has_old ? 2 : 1) * (C::kKBytes + (load_v ? C::kVBytes : 0));
+    int issued[kAtStages];
+    for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
+    for (int item = blockIdx.x; item < total && !*B.abort_flag; item += gridDim.x) {
+      const int h = item / row_tiles, rt = item % row_tiles;
+      const int nt = at_tiles(g, h, rt, n_rows);
+      for (int t = 0; t < nt && !*B.abort_flag; ++t) {
+        if (!mbar_wait_sleep(&B.kv_empty[stage], phase ^ 1)) {
+          set_error(g.err, kDevErrTimeout);
+          *B.abort_flag = 1;
+          break;
+        }
+        uint8_t* st = smem + stage * C::kStageBytes;
+        mbar_arrive_expect_tx(&B.kv_full[stage], bytes);
+#pragma unroll
+        for (int c = 0; c < DH / 64; ++c)
+          tma_load_3d(st + c * (kAtCols * 128), tkn, c * 64, t * kAtCols, h, &B.kv_full[stage]);
+        if (load_v) tma_load_3d(st + 2 * C::kKBytes, tvn, t * kAtCols, 0, h, &B.kv_full[stage]);
+        if (has_old) {
+#pragma unroll
+          for (int c = 0; c < DH / 64; ++c)
+            tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), tko, c * 64, t * kAtCols, h, &B.kv_full[stage]);
+          if (load_v) tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, tvo, t * kAtCols, 0, h, &B.kv_full[stage]);
+        }
+        issued[stage] = phase;
+        if (++stage == kAtStages) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    // never leave with a copy in flight: wait (bounded) for the last load of every stage
+    for (int s2 = 0; s2 < kAtStages; ++s2)
+      if (issued[s2] >= 0) (void)mbar_wait(&B.kv_full[s2], (uint32_t)issued[s2]);
+  }
+}
+
+// MMA role (one thread): S(t) = [Q_new K_new^T | Q_old K_old^T] into score
+// buffer t & 1 while the rows process S(t-1), then P(t-1).V into N.
+template <int DH, int MODE>
+__device__ __forceinline__ void at_mma_role(uint8_t* smem, const AtBars& B, uint32_t tmem, const AtArgs& g,
+                                            int n_rows, int row_tiles, int total, bool has_old, int lane) {
+  using C = AtCfg<DH>;
+  if (lane == 0) {
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t u = 0;        // global tile counter (S buffer = u & 1)
+    uint32_t item_no = 0;
+    bool ok = true;
+    for (int item = blockIdx.x; item < total && ok && !*B.abort_flag; item += gridDim.x, ++item_no) {
+      const int h = item / row_tiles, rt = item % row_tiles;
+      const int nt = at_tiles(g, h, rt, n_rows);
+      if (!mbar_wait_sleep(B.q_ready, item_no & 1)) {
+        set_error(g.err, kDevErrTimeout);
+        *B.abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      int prev_stage = -1;
+      for (int t = 0; t <= nt; ++t) {
+        if (t < nt) {
+          // S(t) into buffer u & 1
+          if (!mbar_wait_sleep(&B.kv_full[stage], phase)) {
+            set_error(g.err, kDevErrTimeout);
+            *B.abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sb = tmem + C::kColS + (u & 1) * 128;
+          const uint32_t k_addr = smem_u32(smem + stage * C::kStageBytes);
+#pragma unroll
+          for (int ks = 0; ks < DH / 16; ++ks) {
+            const uint32_t kd = k_addr + (ks >> 2) * (kAtCols * 128) + (ks & 3) * 32;
+            umma_f16_ts(sb, tmem + C::kColQn + ks * 8, sw128_kmajor_desc(kd), C::kIdescS, ks > 0);
+            if (has_old)
+              umma_f16_ts(sb + 64, tmem + C::kColQo + ks * 8, sw128_kmajor_desc(kd + C::kKBytes), C::kIdescS,
+                          ks > 0);
+          }
+          umma_commit(&B.s_full[u & 1]);
+        }
+        if (t > 0) {
+          // P(t-1).V into N
+          const uint32_t up = u - 1;
+          if (!mbar_wait_sleep(&B.p_full[up & 1], (up >> 1) & 1)) {
+            set_error(g.err, kDevErrTimeout);
+            *B.abort_flag = 1;
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (MODE != kAtFixedMassStats) {  // the statistics pass has no P.V
+            const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
+            const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKBytes);
+#pragma unroll
+            for (int ks = 0; ks < kAtCols / 16; ++ks)
+              umma_f16_ts(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
+            if (has_old) {
+#pragma unroll
+              for (int ks = 0; ks < kAtCols / 16; ++ks)
+                umma_f16_ts(tmem + C::kColN, pcol + 32 + ks * 8, sw128_kmajor_desc(v_addr + C::kVBytes + ks * 32),
+                            C::kIdescPV, 1u);
+            }
+          }
+          umma_commit(&B.kv_empty[prev_stage]);
+          umma_commit(&B.pv_done[up & 1]);
+        }
+        if (t < nt) {
+          prev_stage = stage;
+          if (++stage == kAtStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          ++u;
+        }
+      }
+    }
+  }
+}
+
 template <int DH, int MODE>
 __global__ void __launch_bounds__(kAtThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
@@ -156,124 +299,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
+  const AtBars B{kv_full, kv_empty, s_full, p_full, pv_done, q_ready, abort_flag};
   if (warp == 8) {
-    // ------------------------------------------------------------ TMA loads
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      constexpr bool load_v = MODE != kAtFixedMassStats;
-      const uint32_t bytes = (has_old ? 2 : 1) * (C::kKBytes + (load_v ? C::kVBytes : 0));
-      int issued[kAtStages];
-      for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
-      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
-        const int h = item / row_tiles, rt = item % row_tiles;
-        const int nt = at_tiles(g, h, rt, n_rows);
-        for (int t = 0; t < nt && !*abort_flag; ++t) {
-          if (!mbar_wait_sleep(&kv_empty[stage], phase ^ 1)) {
-            set_error(g.err, kDevErrTimeout);
-            *abort_flag = 1;
-            break;
-          }
-          uint8_t* st = smem + stage * C::kStageBytes;
-          mbar_arrive_expect_tx(&kv_full[stage], bytes);
-#pragma unroll
-          for (int c = 0; c < DH / 64; ++c)
-            tma_load_3d(st + c * (kAtCols * 128), &tm_kn, c * 64, t * kAtCols, h, &kv_full[stage]);
-          if (load_v) tma_load_3d(st + 2 * C::kKBytes, &tm_vn, t * kAtCols, 0, h, &kv_full[stage]);
-          if (has_old) {
-#pragma unroll
-            for (int c = 0; c < DH / 64; ++c)
-              tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), &tm_ko, c * 64, t * kAtCols, h, &kv_full[stage]);
-            if (load_v) tma_load_3d(st + 2 * C::kKBytes + C::kVBytes, &tm_vo, t * kAtCols, 0, h, &kv_full[stage]);
-          }
-          issued[stage] = phase;
-          if (++stage == kAtStages) {
-            stage = 0;
-            phase ^= 1;
-          }
-        }
-      }
-      // never leave with a copy in flight: wait (bounded) for the last load of every stage
-      for (int s2 = 0; s2 < kAtStages; ++s2)
-        if (issued[s2] >= 0) (void)mbar_wait(&kv_full[s2], (uint32_t)issued[s2]);
-    }
+    at_load_role<DH, MODE>(smem, B, &tm_kn, &tm_ko, &tm_vn, &tm_vo, g, n_rows, row_tiles, total, has_old, lane);
   } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issue
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      uint32_t u = 0;        // global tile counter (S buffer = u & 1)
-      uint32_t item_no = 0;
-      bool ok = true;
-      for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x, ++item_no) {
-        const int h = item / row_tiles, rt = item % row_tiles;
-        const int nt = at_tiles(g, h, rt, n_rows);
-        if (!mbar_wait_sleep(q_ready, item_no & 1)) {
-          set_error(g.err, kDevErrTimeout);
-          *abort_flag = 1;
-          break;
-        }
-        tc_fence_after();
-        int prev_stage = -1;
-        for (int t = 0; t <= nt; ++t) {
-          if (t < nt) {
-            // S(t) into buffer u & 1
-            if (!mbar_wait_sleep(&kv_full[stage], phase)) {
-              set_error(g.err, kDevErrTimeout);
-              *abort_flag = 1;
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            const uint32_t sb = tmem + C::kColS + (u & 1) * 128;
-            const uint32_t k_addr = smem_u32(smem + stage * C::kStageBytes);
-#pragma unroll
-            for (int ks = 0; ks < DH / 16; ++ks) {
-              const uint32_t kd = k_addr + (ks >> 2) * (kAtCols * 128) + (ks & 3) * 32;
-              umma_f16_ts(sb, tmem + C::kColQn + ks * 8, sw128_kmajor_desc(kd), C::kIdescS, ks > 0);
-              if (has_old)
-                umma_f16_ts(sb + 64, tmem + C::kColQo + ks * 8, sw128_kmajor_desc(kd + C::kKBytes), C::kIdescS,
-                            ks > 0);
-            }
-            umma_commit(&s_full[u & 1]);
-          }
-          if (t > 0) {
-            // P(t-1).V into N
-            const uint32_t up = u - 1;
-            if (!mbar_wait_sleep(&p_full[up & 1], (up >> 1) & 1)) {
-              set_error(g.err, kDevErrTimeout);
-              *abort_flag = 1;
-              ok = false;
-              break;
-            }
-            tc_fence_after();
-            if (MODE != kAtFixedMassStats) {  // the statistics pass has no P.V
-              const uint32_t pcol = tmem + C::kColS + (up & 1) * 128;
-              const uint32_t v_addr = smem_u32(smem + prev_stage * C::kStageBytes + 2 * C::kKBytes);
-#pragma unroll
-              for (int ks = 0; ks < kAtCols / 16; ++ks)
-                umma_f16_ts(tmem + C::kColN, pcol + ks * 8, sw128_kmajor_desc(v_addr + ks * 32), C::kIdescPV, 1u);
-              if (has_old) {
-#pragma unroll
-                for (int ks = 0; ks < kAtCols / 16; ++ks)
-                  umma_f16_ts(tmem + C::kColN, pcol + 32 + ks * 8, sw128_kmajor_desc(v_addr + C::kVBytes + ks * 32),
-                              C::kIdescPV, 1u);
-              }
-            }
-            umma_commit(&kv_empty[prev_stage]);
-            umma_commit(&pv_done[up & 1]);
-          }
-          if (t < nt) {
-            prev_stage = stage;
-            if (++stage == kAtStages) {
-              stage = 0;
-              phase ^= 1;
-            }
-            ++u;
-          }
-        }
-      }
-    }
+    at_mma_role<DH, MODE>(smem, B, tmem, g, n_rows, row_tiles, total, has_old, lane);
   } else {
     // ------------------------------------------------------------ rows
     // Two threads per row: half 0 takes columns [0, 32) of each tile (and
@@ -582,6 +612,357 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         g.m_out[(size_t)h * g.S + tok] = m_ref / kAtLog2e;
         g.z_out[(size_t)h * g.S + tok] = z_row;
         if (g.dense && g.g_out) g.g_out[(size_t)h * g.S + tok] = 1.f;
+      }
+      tc_fence_before();
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+// The running update of loops >= 2 with the row pass split by tiles instead
+// of by columns ("ping-pong"): row group 0 (warps 0-3) handles the tiles with
+// an even block-wide tile counter, group 1 (warps 4-7) the odd ones, one
+// thread per row over all 64 new and 64 old columns of its tile.  While one
+// group computes the exponentials of tile t, the other loads and reduces tile
+// t+1, so the exponential unit and the tensor pipe stay busy across tiles.
+// The row's reference (log2 units) passes from the group of tile t to the
+// group of tile t+1 through shared memory at a named barrier (an arrive on
+// one side, a sync on the other; one barrier per group and lane quarter).
+// Only the new scores can raise it: the old scores are the previous loop's,
+// already within 8 of the reference it left behind, and the reference never
+// decreases.  Each group keeps its own part of Z in the frame of the last tile
+// it handled; the parts are brought to the final frame at the end of the
+// item.  The rare raise rescales the whole row of N (after P(t-1).V) in the
+// handling thread.  Producer and MMA roles are those of attn_tc_kernel.
+template <int DH>
+__global__ void __launch_bounds__(kAtThreads, 1)
+attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
+               const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_vo, AtArgs g) {
+  using C = AtCfg<DH>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAtStages * C::kStageBytes);
+  uint64_t* kv_full = bars;
+  uint64_t* kv_empty = bars + kAtStages;
+  uint64_t* s_full = bars + 2 * kAtStages;
+  uint64_t* p_full = s_full + 2;
+  uint64_t* pv_done = p_full + 2;
+  uint64_t* q_ready = pv_done + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int n_rows = g.n_rows ? *g.n_rows : g.S;
+  if (n_rows > g.row_cap) n_rows = g.row_cap;
+  if (n_rows < 0) n_rows = 0;
+  const int row_tiles = (n_rows + kAtRows - 1) / kAtRows;
+  const int total = row_tiles * g.H;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kAtStages; ++s) {
+      mbar_init(&kv_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&p_full[b], kAtRowThreads / 2);  // the 128 threads of the tile's group
+      mbar_init(&pv_done[b], 1);
+    }
+    mbar_init(q_ready, kAtRowThreads);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const AtBars B{kv_full, kv_empty, s_full, p_full, pv_done, q_ready, abort_flag};
+  if (warp == 8) {
+    at_load_role<DH, kAtRunning>(smem, B, &tm_kn, &tm_ko, &tm_vn, &tm_vo, g, n_rows, row_tiles, total, true, lane);
+  } else if (warp == 9) {
+    at_mma_role<DH, kAtRunning>(smem, B, tmem, g, n_rows, row_tiles, total, true, lane);
+  } else {
+    // A named barrier cannot time out, so both groups always execute the same
+    // barrier sequence: after a failed wait (or an abort raised elsewhere) a
+    // warp turns "dead" - it skips waits, tensor-memory work and writes but
+    // keeps the control flow.
+    const int quarter = warp & 3, grp = warp >> 2;
+    const int row = quarter * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
+    const int bar_give = 1 + grp * 4 + quarter;          // this group's reference is ready
+    const int bar_take = 1 + (grp ^ 1) * 4 + quarter;    // the other group's reference is ready
+    const int bar_end = 9 + quarter;                     // end of item: the two parts of Z
+    float* xm = reinterpret_cast<float*>(tmem_slot + 4);  // [2 groups][128] reference after the group's tile
+    float* xz = xm + 2 * 128;                             // [2][128] part of Z
+    float* xf = xz + 2 * 128;                             // [2][128] frame of that part
+    const int HD = g.H * DH;
+    constexpr int kHalfCols = DH / 2;
+    bool dead = false;
+    auto wait_or_die = [&](uint64_t* bar, uint32_t parity) {
+      if (!dead && __any_sync(0xffffffffu, *abort_flag != 0)) dead = true;
+      if (dead) return;
+      if (!__all_sync(0xffffffffu, mbar_wait_sleep(bar, parity))) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        dead = true;
+        return;
+      }
+      tc_fence_after();
+    };
+    uint32_t u = 0;
+    for (int item = blockIdx.x; item < total; item += gridDim.x) {
+      const int h = item / row_tiles, rt = item % row_tiles;
+      const int nt = at_tiles(g, h, rt, n_rows);
+      const int a = rt * kAtRows + row;
+      int tok = -1;
+      if (a < n_rows) {
+        tok = g.rows ? __ldg(g.rows + a) : a;
+        if (tok < 0 || tok >= g.S) {
+          if (grp == 0) set_error(g.err, FLASHLOOP_DEVERR_INDEX);
+          tok = -1;
+        }
+      }
+      // the previous loop's state: reference m_in (log2 units) and Z_in,
+      // carried by group 0's part of Z
+      float m_init = 0.f, z_part = 0.f;
+      if (tok >= 0) {
+        const size_t hi = (size_t)h * g.S + tok;
+        m_init = g.m_in[hi] * kAtLog2e;
+        if (grp == 0) z_part = g.z_in[hi];
+      }
+      float frame = m_init;  // frame of z_part
+      // Q (fp16 pairs, exact from bf16) and this group's half of N into TMEM:
+      // group 0 Q_new and N[0, DH/2), group 1 Q_old and N[DH/2, DH).  The
+      // rebuilt keys carry log2(e)/sqrt(dh), so S is in log2 units.
+      if (!dead) {
+        const uint16_t* qsrc = grp == 0 ? g.q_new : g.q_old;
+        const uint32_t qcol = grp == 0 ? C::kColQn : C::kColQo;
+        uint32_t qv[DH / 16][8];
+#pragma unroll
+        for (int v = 0; v < DH / 16; ++v) {
+          if (tok >= 0) {
+            ld_global_v8(qsrc + (size_t)tok * HD + (size_t)h * DH + v * 16, qv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) qv[v][e] = 0u;
+          }
+        }
+        bool q_ok = true;  // q must fit fp16, the MMA operand type
+#pragma unroll
+        for (int c0 = 0; c0 < DH; c0 += 32) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 f = bf16x2_to_float2(qv[c0 / 16 + e / 8][e % 8]);
+            q_ok = q_ok && half_range_ok(f.x) && half_range_ok(f.y);
+            r[e] = bf16x2_to_half2_bits(qv[c0 / 16 + e / 8][e % 8]);
+          }
+          __syncwarp();
+          tmem_st16(tmem + lane_base + qcol + c0 / 2, r);
+        }
+        if (!q_ok) set_error(g.err, FLASHLOOP_DEVERR_RANGE);
+        uint32_t nv[kHalfCols / 8][8];
+#pragma unroll
+        for (int v = 0; v < kHalfCols / 8; ++v) {
+          if (tok >= 0) {
+            ld_global_v8(g.n_in + ((size_t)h * g.S + tok) * DH + grp * kHalfCols + 8 * v, nv[v]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) nv[v][e] = 0u;
+          }
+        }
+#pragma unroll
+        for (int c0 = 0; c0 < kHalfCols; c0 += 16) {
+          uint32_t r[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) r[e] = nv[c0 / 8 + e / 8][e % 8];
+          __syncwarp();
+          tmem_st16(tmem + lane_base + C::kColN + grp * kHalfCols + c0, r);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(q_ready);
+        // bring the next item's rows (this thread's q and half of N) into L2
+        const int item_next = item + gridDim.x;
+        if (item_next < total) {
+          const int hn = item_next / row_tiles, an = (item_next % row_tiles) * kAtRows + row;
+          const int tn = an < n_rows ? (g.rows ? __ldg(g.rows + an) : an) : -1;
+          if (tn >= 0 && tn < g.S) {
+            const uint16_t* qn = (grp == 0 ? g.q_new : g.q_old) + (size_t)tn * HD + (size_t)hn * DH;
+#pragma unroll
+            for (int c = 0; c < DH * 2; c += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(qn) + c);
+            const float* nn = g.n_in + ((size_t)hn * g.S + tn) * DH + grp * kHalfCols;
+#pragma unroll
+            for (int c = 0; c < kHalfCols * 4; c += 128) prefetch_l2(reinterpret_cast<const uint8_t*>(nn) + c);
+          }
+        }
+      }
+
+      // the row's causal prefix of the selection (columns ascend, so the
+      // valid columns of every tile form a prefix of it)
+      const int nc_row = tok < 0 ? 0 : at_row_count(g, h, a, tok);
+      for (int t = 0; t < nt; ++t, ++u) {
+        const uint32_t b = u & 1;
+        if ((int)b != grp) continue;  // the other group's tile
+        const int nvalid = min(max(nc_row - t * kAtCols, 0), kAtCols);
+        wait_or_die(&s_full[b], (u >> 1) & 1);
+        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
+        uint32_t sc[64];
+        float mx = -INFINITY;
+        if (!dead) {
+          __syncwarp();
+          tmem_ld32(sbase, *reinterpret_cast<uint32_t(*)[32]>(sc));
+          tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
+          tmem_wait_ld();
+          if (nvalid < kAtCols) {
+#pragma unroll
+            for (int e = 0; e < 64; ++e)
+              if (e >= nvalid) sc[e] = 0xff800000u;  // -inf
+          }
+          float t32[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) t32[e] = fmaxf(__uint_as_float(sc[e]), __uint_as_float(sc[e + 32]));
+#pragma unroll
+          for (int w = 16; w > 0; w >>= 1)
+#pragma unroll
+            for (int e = 0; e < w; ++e) t32[e] = fmaxf(t32[e], t32[e + w]);
+          mx = t32[0];
+        }
+        // the reference after tile t-1 (this item's), from the other group
+        float m_prev = m_init;
+        if (t > 0) {
+          named_bar_sync(bar_take, 64);
+          m_prev = xm[(grp ^ 1) * 128 + row];
+        }
+        const bool need = mx > m_prev + kRescaleThreshold;
+        const float m_ref = need ? mx : m_prev;
+        if (t + 1 < nt) {
+          xm[grp * 128 + row] = m_ref;
+          named_bar_arrive(bar_give, 64);
+        }
+        if (dead) continue;
+        if (__any_sync(0xffffffffu, need)) {
+          // raise the reference of this warp's rows: N scales by 2^(m_prev - m_ref)
+          // once P(t-1).V has landed
+          const float f = need ? ex2(m_prev - m_ref) : 1.f;
+          if (t > 0) {
+            const uint32_t up = u - 1;
+            wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+            if (dead) continue;
+          }
+#pragma unroll 1
+          for (int cc = 0; cc < DH; cc += 16) {
+            uint32_t r[16];
+            __syncwarp();
+            tmem_ld16(tmem + lane_base + C::kColN + cc, r);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
+            __syncwarp();
+            tmem_st16(tmem + lane_base + C::kColN + cc, r);
+          }
+          tmem_wait_st();
+        }
+        if (frame != m_ref) {
+          z_part *= ex2(frame - m_ref);
+          frame = m_ref;
+        }
+        // P_new = 2^(S_new - m_ref) over columns [0, 32) of the buffer (fp16 pairs)
+        float za[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float p0 = ex2(__uint_as_float(sc[32 * hf + 2 * e2]) - m_ref);
+            const float p1 = ex2(__uint_as_float(sc[32 * hf + 2 * e2 + 1]) - m_ref);
+            za[e2 & 3] += p0 + p1;
+            pk[e2] = pack_half2(p0, p1);
+          }
+          __syncwarp();
+          tmem_st16(sbase + 16 * hf, pk);
+        }
+        // -P_old = -2^(S_old - m_ref) over columns [32, 64)
+        __syncwarp();
+        tmem_ld32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(sc));
+        tmem_ld32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
+        tmem_wait_ld();
+        if (nvalid < kAtCols) {
+#pragma unroll
+          for (int e = 0; e < 64; ++e)
+            if (e >= nvalid) sc[e] = 0xff800000u;
+        }
+        float zb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e2 = 0; e2 < 16; ++e2) {
+            const float p0 = ex2(__uint_as_float(sc[32 * hf + 2 * e2]) - m_ref);
+            const float p1 = ex2(__uint_as_float(sc[32 * hf + 2 * e2 + 1]) - m_ref);
+            zb[e2 & 3] += p0 + p1;
+            pk[e2] = pack_half2(-p0, -p1);
+          }
+          __syncwarp();
+          tmem_st16(sbase + 32 + 16 * hf, pk);
+        }
+        z_part += ((za[0] + za[1]) + (za[2] + za[3])) - ((zb[0] + zb[1]) + (zb[2] + zb[3]));
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_full[b]);
+      }
+      if (nt > 0) {  // every contribution of the item has reached N
+        const uint32_t up = u - 1;
+        wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+      }
+      // the two parts of Z in the final frame (frames only rise: the larger)
+      xz[grp * 128 + row] = z_part;
+      xf[grp * 128 + row] = frame;
+      named_bar_sync(bar_end, 64);
+      const float z_other = xz[(grp ^ 1) * 128 + row];
+      const float f_other = xf[(grp ^ 1) * 128 + row];
+      named_bar_sync(bar_end, 64);
+      if (dead) continue;
+      const float m_fin = fmaxf(frame, f_other);
+      const float z_row = (frame == m_fin ? z_part : z_part * ex2(frame - m_fin)) +
+                          (f_other == m_fin ? z_other : z_other * ex2(f_other - m_fin));
+      const float inv = 1.f / z_row;
+#pragma unroll 1
+      for (int cc = 0; cc < kHalfCols; cc += 16) {
+        uint32_t r[16];
+        __syncwarp();
+        tmem_ld16(tmem + lane_base + C::kColN + grp * kHalfCols + cc, r);
+        tmem_wait_ld();
+        if (tok >= 0) {
+          const int col = grp * kHalfCols + cc;
+          float* nd = g.n_out + ((size_t)h * g.S + tok) * DH + col;
+          uint32_t w[8];
+#pragma unroll
+          for (int v = 0; v < 2; ++v) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w[e] = r[8 * v + e];
+            st_global_v8(nd + 8 * v, w);
+          }
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            w[q] = (uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q]) * inv) |
+                   ((uint32_t)float_to_bf16_bits(__uint_as_float(r[2 * q + 1]) * inv) << 16);
+          st_global_v8(g.o + (size_t)tok * HD + (size_t)h * DH + col, w);
+        }
+      }
+      if (tok >= 0 && grp == 0) {
+        g.m_out[(size_t)h * g.S + tok] = m_fin / kAtLog2e;
+        g.z_out[(size_t)h * g.S + tok] = z_row;
       }
       tc_fence_before();
     }
@@ -1093,14 +1474,16 @@ int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaSt
     kernel<<<grid, kAtThreads, smem, stream>>>(tkn, tko, tvn, tvo, g);
     return FLASHLOOP_OK;
   };
+  // the running update: the ping-pong row pass; the fixed-mass passes: the
+  // column-split row pass of attn_tc_kernel
   if (dh == 128) {
     if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<128, kAtFixedMassStats>, AtCfg<128>::kSmem);
     else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<128, kAtFixedMassUpdate>, AtCfg<128>::kSmem);
-    else rc = launch(attn_tc_kernel<128, kAtRunning>, AtCfg<128>::kSmem);
+    else rc = launch(attn_pp_kernel<128>, AtCfg<128>::kSmem);
   } else {
     if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<64, kAtFixedMassStats>, AtCfg<64>::kSmem);
     else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<64, kAtFixedMassUpdate>, AtCfg<64>::kSmem);
-    else rc = launch(attn_tc_kernel<64, kAtRunning>, AtCfg<64>::kSmem);
+    else rc = launch(attn_pp_kernel<64>, AtCfg<64>::kSmem);
   }
   if (rc != FLASHLOOP_OK) return rc;
   return launch_status();

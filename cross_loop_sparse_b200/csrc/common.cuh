@@ -66,6 +66,7 @@ struct Workspace {
   size_t cm_rows;   // column-mass scratch: row max (log2), 1/Z [H, S] each, row tokens [S]
   size_t cols_kv;   // fp16 dequantised selected columns: 4 x [H, kmax, dh] or 2 x [H, S, dh]
   size_t row_cnt;   // int32 [H, S]: per head and active row, the selected columns at or before its token
+  size_t kv_f32;    // float32 K and V of the loop's active rows, 2 x [S, H, dh] (kv_scheme 1 only)
   size_t total;
 };
 
@@ -94,6 +95,7 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   size_t dense = 2 * H * (size_t)pad8(p->seq) * dh;
   w.cols_kv = off; off = align256(off + (sel > dense ? sel : dense) * sizeof(__half));
   w.row_cnt = off; off = align256(off + H * S * sizeof(int32_t));
+  w.kv_f32 = off; off = align256(off + (p->kv_scheme == 1 ? 2 * S * H * dh * sizeof(float) : 0));
   w.total = off;
   return w;
 }

@@ -70,6 +70,21 @@ __device__ __forceinline__ void rope_rot(float& x1, float& x2, float c, float s)
   x2 = y2;
 }
 
+// acc += code * s for the 32 BITS-bit two's-complement codes of one group
+// (packed words w); BITS is a template constant so that every field index is
+// a constant and the words stay in registers.
+template <int BITS>
+__device__ __forceinline__ void add_codes(const uint32_t (&w)[8], float s, float (&acc)[32]) {
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    constexpr uint32_t kMask = (1u << BITS) - 1u;
+    const int bit = e * BITS;
+    int c = static_cast<int>((w[bit >> 5] >> (bit & 31)) & kMask);
+    if (c >= (1 << (BITS - 1))) c -= (1 << BITS);
+    acc[e] = acc[e] + static_cast<float>(c) * s;
+  }
+}
+
 // Rebuild Xhat^(upto) of 32 consecutive elements (group g) of one (token, head).
 template <int DH>
 __device__ __forceinline__ void recon_group(const KVStreams& kv, const LoopTables& lt, int t, int h, int H,
@@ -92,33 +107,30 @@ __device__ __forceinline__ void recon_group(const KVStreams& kv, const LoopTable
     const int b = lt.bits[l - 1];
     const uint8_t* row = kv.res_codes[l - 1] + ((size_t)sl * H + h) * (DH * b / 8) + g * 4 * b;
     const float s = __half2float(__ushort_as_half(kv.res_scales[l - 1][((size_t)sl * H + h) * (DH / 32) + g]));
-    uint32_t w[8];
+    uint32_t w[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (b == 8) {
       const uint4 a0 = *reinterpret_cast<const uint4*>(row);
       const uint4 a1 = *reinterpret_cast<const uint4*>(row + 16);
       w[0] = a0.x; w[1] = a0.y; w[2] = a0.z; w[3] = a0.w; w[4] = a1.x; w[5] = a1.y; w[6] = a1.z; w[7] = a1.w;
+      add_codes<8>(w, s, acc);
     } else if (b == 4) {
       const uint4 a0 = *reinterpret_cast<const uint4*>(row);
       w[0] = a0.x; w[1] = a0.y; w[2] = a0.z; w[3] = a0.w;
+      add_codes<4>(w, s, acc);
     } else {
       const uint2 a0 = *reinterpret_cast<const uint2*>(row);
       w[0] = a0.x; w[1] = a0.y;
-    }
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const int bit = e * b;
-      const uint32_t f = (w[bit >> 5] >> (bit & 31)) & ((1u << b) - 1u);
-      int c = static_cast<int>(f);
-      if (c >= (1 << (b - 1))) c -= (1 << b);
-      acc[e] = acc[e] + static_cast<float>(c) * s;
+      add_codes<2>(w, s, acc);
     }
   }
 }
 
-// Quantise 32 values and store their packed codes (32*bits/8 bytes) and scale.
-__device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits, uint8_t* codes,
-                                                  uint16_t* scale) {
-  const int qmax = (1 << (bits - 1)) - 1;
+// Quantise 32 values and store their packed codes (32*BITS/8 bytes) and
+// scale; BITS is a template constant so that the packed words stay in
+// registers.
+template <int BITS>
+__device__ __forceinline__ void quant_store_group_b(const float (&x)[32], uint8_t* codes, uint16_t* scale) {
+  constexpr int qmax = (1 << (BITS - 1)) - 1;
   float amax = 0.f;
 #pragma unroll
   for (int e = 0; e < 32; ++e) amax = fmaxf(amax, fabsf(x[e]));
@@ -131,18 +143,25 @@ __device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits
 #pragma unroll
   for (int e = 0; e < 32; ++e) {
     const int c = s > 0.f ? static_cast<int>(quant_code(x[e], s, rs, qmax)) : 0;
-    const int bit = e * bits;
-    w[bit >> 5] |= (static_cast<uint32_t>(c) & ((1u << bits) - 1u)) << (bit & 31);
+    const int bit = e * BITS;
+    w[bit >> 5] |= (static_cast<uint32_t>(c) & ((1u << BITS) - 1u)) << (bit & 31);
   }
-  if (bits == 8) {
+  if (BITS == 8) {
     *reinterpret_cast<uint4*>(codes) = make_uint4(w[0], w[1], w[2], w[3]);
     *reinterpret_cast<uint4*>(codes + 16) = make_uint4(w[4], w[5], w[6], w[7]);
-  } else if (bits == 4) {
+  } else if (BITS == 4) {
     *reinterpret_cast<uint4*>(codes) = make_uint4(w[0], w[1], w[2], w[3]);
   } else {
     *reinterpret_cast<uint2*>(codes) = make_uint2(w[0], w[1]);
   }
   *scale = sbits;
+}
+
+__device__ __forceinline__ void quant_store_group(const float (&x)[32], int bits, uint8_t* codes,
+                                                  uint16_t* scale) {
+  if (bits == 8) quant_store_group_b<8>(x, codes, scale);
+  else if (bits == 4) quant_store_group_b<4>(x, codes, scale);
+  else quant_store_group_b<2>(x, codes, scale);
 }
 
 __device__ __forceinline__ void prefetch_l2(const void* p) {

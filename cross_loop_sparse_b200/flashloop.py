@@ -16,6 +16,8 @@ import torch
 
 MAX_LOOPS = 16
 GROUP = 32
+PAPER_GROUP = 64   # the pages' cache setting: groups of 64 and a 64-token bf16 tail
+PAPER_TAIL = 64
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libflashloop.so")
 HEADER_PATH = os.path.join(os.path.dirname(_PKG), "include", "flashloop.h")
@@ -41,16 +43,17 @@ class Params(ctypes.Structure):
                 ("n_loops", c_int32), ("batch", c_int32), ("tau", c_float), ("rope_theta", c_float),
                 ("topk", c_int32 * MAX_LOOPS), ("bits", c_int32 * MAX_LOOPS),
                 ("capacity", c_int32 * MAX_LOOPS), ("gate_topk", c_int32), ("fixed_mass", c_int32),
-                ("attn_pairs", c_int32)]
+                ("attn_pairs", c_int32), ("kv_scheme", c_int32)]
 
     @classmethod
     def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None,
-                    fixed_mass=False, attn_pairs=False):
+                    fixed_mass=False, attn_pairs=False, kv_scheme="spec"):
         """Params of a workload.Config; capacities default to S (no overflow possible).
         token_budgets (per loop) selects top-k token retention with those budgets;
         fixed_mass selects the fixed-mass form of the sparse update; attn_pairs runs
         the running update on SM pairs."""
         p = cls()
+        p.kv_scheme = {"spec": 0, "paper": 1}[kv_scheme]
         p.fixed_mass = 1 if fixed_mass else 0
         p.attn_pairs = int(attn_pairs)
         p.seq = cfg.seq if seq is None else seq
@@ -75,12 +78,18 @@ class KV(ctypes.Structure):
                 ("res_codes", c_void_p * MAX_LOOPS), ("res_scales", c_void_p * MAX_LOOPS)]
 
 
+class PaperKV(ctypes.Structure):
+    _fields_ = [("codes", c_void_p * MAX_LOOPS), ("scale", c_void_p * MAX_LOOPS),
+                ("minv", c_void_p * MAX_LOOPS), ("tail", c_void_p * MAX_LOOPS)]
+
+
 class StateC(ctypes.Structure):
     _fields_ = [("k", KV), ("v", KV), ("active", c_void_p * MAX_LOOPS), ("slot", c_void_p * MAX_LOOPS),
                 ("n_active", c_void_p), ("q", c_void_p * 3), ("m", c_void_p * 3), ("Z", c_void_p * 3),
                 ("N", c_void_p * 3), ("colmass", c_void_p * 2), ("cols", c_void_p * MAX_LOOPS),
                 ("O", c_void_p), ("Y", c_void_p), ("rope_cs", c_void_p), ("err_word", c_void_p),
-                ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("G", c_void_p * 3)]
+                ("workspace", c_void_p), ("workspace_bytes", c_size_t), ("G", c_void_p * 3),
+                ("paper_k", POINTER(PaperKV)), ("paper_v", POINTER(PaperKV))]
 
 
 class DecodeStateC(ctypes.Structure):
@@ -106,6 +115,7 @@ _SIG = {
     "flashloop_qkv_gathered": (_I, [_P, _V, _V, _V, _I, _V, _V, _V, _V, _V, _V]),
     "flashloop_kv_quant_residual": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
     "flashloop_qkv_quant": (_I, [_P, _I, _V, _V, _V, _V, _S, _V, _V]),
+    "flashloop_paper_kv_quant": (_I, [_P, _I, _V, _V, _V, _V, _S, _V]),
     "flashloop_topk_columns": (_I, [_P, _V, _V, _I, _I, _V, _V]),
     "flashloop_selcol_dequant": (_I, [_P, _I, _S, _V]),
     "flashloop_sparse_attn_update": (_I, [_P, _I, _S, _I, _V]),
@@ -231,6 +241,12 @@ def flashloop_qkv_quant(params, loop, x, active, n_active, w_qkv, state, q_out, 
         ctypes.byref(state.c), _ptr(q_out), _stream(stream)))
 
 
+def flashloop_paper_kv_quant(params, loop, k_new, v_new, active, n_active, state, stream=None):
+    return _check("flashloop_paper_kv_quant", _lib.flashloop_paper_kv_quant(
+        ctypes.byref(params), loop, _ptr(k_new), _ptr(v_new), _ptr(active), _ptr(n_active),
+        ctypes.byref(state.c), _stream(stream)))
+
+
 def flashloop_topk_columns(params, mass, candidates, n_cand, k, out, stream=None):
     return _check("flashloop_topk_columns", _lib.flashloop_topk_columns(
         ctypes.byref(params), _ptr(mass), _ptr(candidates), n_cand, k, _ptr(out), _stream(stream)))
@@ -329,7 +345,29 @@ class FlashLoopState:
         z = lambda shape, dt: torch.zeros(shape, dtype=dt, device=dev)  # noqa: E731
         self.t = {}
         c = StateC()
-        for name, kv in (("k", c.k), ("v", c.v)):
+        self._paper = []
+        if params.kv_scheme == 1:
+            # the pages' cache setting: per loop INT4 codes, fp16 scales and minima, bf16 tail
+            tail = min(PAPER_TAIL, S)
+            body = S - tail
+            for name in ("k", "v"):
+                kv = PaperKV()
+                for r in range(1, R + 1):
+                    rows = max(body if r == 1 else params.capacity[r - 1], 1)
+                    groups = (rows + PAPER_GROUP - 1) // PAPER_GROUP
+                    gshape = (groups, H, dh) if name == "k" else (rows, H, dh // PAPER_GROUP)
+                    self.t[f"p{name}_codes{r}"] = z((rows, H, dh // 2), torch.uint8)
+                    self.t[f"p{name}_scale{r}"] = z(gshape, torch.float16)
+                    self.t[f"p{name}_min{r}"] = z(gshape, torch.float16)
+                    self.t[f"p{name}_tail{r}"] = z((max(tail, 1), H, dh), torch.bfloat16)
+                    kv.codes[r - 1] = self.t[f"p{name}_codes{r}"].data_ptr()
+                    kv.scale[r - 1] = self.t[f"p{name}_scale{r}"].data_ptr()
+                    kv.minv[r - 1] = self.t[f"p{name}_min{r}"].data_ptr()
+                    kv.tail[r - 1] = self.t[f"p{name}_tail{r}"].data_ptr()
+                self._paper.append(kv)
+            c.paper_k = ctypes.pointer(self._paper[0])
+            c.paper_v = ctypes.pointer(self._paper[1])
+        for name, kv in (("k", c.k), ("v", c.v)) if params.kv_scheme == 0 else ():
             base = z((S, H, dh), torch.int8)
             bs = z((S, H, dh // GROUP), torch.float16)
             self.t[f"{name}_base"], self.t[f"{name}_base_s"] = base, bs

@@ -81,6 +81,8 @@ typedef struct flashloop_params {
   int32_t fixed_mass; /* 0: running (m, N, Z) update; else the fixed-mass form (see flashloop_sparse_attn_update) */
   int32_t attn_pairs; /* running update: 0 one SM per 128-row tile; 1 / 2 SM pairs sharing each K/V tile
                          (cta_group::2) with two / four row threads per row */
+  int32_t kv_scheme;  /* 0: INT8 base + INT4/INT2 symmetric residuals (flashloop_kv streams);
+                         1: the pages' own setting (flashloop_paper_kv streams, see below; prefill only) */
 } flashloop_params;
 
 /* One quantised cache (K or V) of a sequence: the loop-1 base over every
@@ -95,6 +97,33 @@ typedef struct flashloop_kv {
   uint8_t* res_codes[FLASHLOOP_MAX_LOOPS];     /* loop r: [capacity_r, H, dh*bits_r/8] */
   uint16_t* res_scales[FLASHLOOP_MAX_LOOPS];   /* loop r: [capacity_r, H, dh/32] fp16 */
 } flashloop_kv;
+
+/* One cache (K or V) in the pages' own setting [FlashLoop App. E "Quantization
+ * setting"; the "Looping a Transformer Quadruples the Bill" page, §3]:
+ * INT4 asymmetric codes in groups of 64 with an fp16 scale and an fp16 minimum
+ * per group (value = code * scale + minimum, codes 0..15), the last
+ * FLASHLOOP_PAPER_TAIL tokens kept in bf16 instead.
+ *  - Body tokens t < body = S - tail (tail = min(FLASHLOOP_PAPER_TAIL, S)):
+ *    loop 1 codes the values themselves, row t; loop r >= 2 codes the residual
+ *    against the reconstruction of loop r-1 for the loop's active body tokens,
+ *    row = the token's position in the loop's active list (its slot).
+ *  - Keys are grouped per channel over 64 consecutive rows (row / 64 is the
+ *    group; a last partial group takes its minimum and maximum over its rows);
+ *    values per row over 64 consecutive channels.
+ *  - Reconstruction of loop r: the loop-1 codes plus, in loop order, the
+ *    residual of every loop 2..r where the token was active (float32); a tail
+ *    token's value is the bf16 value stored at the latest loop <= r where it
+ *    was active (every token is active at loop 1).
+ * Codes are packed two per byte along head_dim (element 2i in the low nibble). */
+#define FLASHLOOP_PAPER_GROUP 64
+#define FLASHLOOP_PAPER_TAIL 64
+typedef struct flashloop_paper_kv {
+  uint8_t* codes[FLASHLOOP_MAX_LOOPS];   /* loop r: [rows_r, H, dh/2] (rows_1 = body, rows_r = capacity_r) */
+  uint16_t* scale[FLASHLOOP_MAX_LOOPS];  /* fp16; keys [ceil(rows_r/64), H, dh], values [rows_r, H, dh/64] */
+  uint16_t* minv[FLASHLOOP_MAX_LOOPS];   /* fp16, the layout of scale */
+  uint16_t* tail[FLASHLOOP_MAX_LOOPS];   /* bf16 [tail, H, dh] at position t - body (rows of tokens
+                                            inactive at loop r are not written) */
+} flashloop_paper_kv;
 
 /* Whole per-sequence state of the sublayer (all device memory, caller-owned;
  * a checkpoint is a copy of these buffers).
@@ -121,6 +150,11 @@ typedef struct flashloop_state {
   size_t workspace_bytes;               /* >= flashloop_workspace_bytes(params) */
   float* G[3];                          /* [H, S] selected-column factor g, one per m/Z/N slot
                                            (params.fixed_mass only; NULL otherwise) */
+  /* params.kv_scheme == 1: the K and V streams in the pages' setting (k and v above are then
+     unused).  The structs themselves are host memory, read on the host; the buffers they point
+     to are device memory. */
+  const flashloop_paper_kv* paper_k;
+  const flashloop_paper_kv* paper_v;
 } flashloop_state;
 
 /* ---------------------------------------------------------------- sizing */
@@ -218,6 +252,20 @@ int flashloop_qkv_gathered(const flashloop_params* p, const uint16_t* x, const i
 int flashloop_kv_quant_residual(const flashloop_params* p, int32_t loop, const float* k_new,
                                 const float* v_new, const int32_t* active, const int32_t* n_active,
                                 flashloop_state* st, void* stream);
+
+/* (f2) The pages' own cache setting: quantisation of loop `loop`'s keys and
+ * values into st->paper_k / st->paper_v (params.kv_scheme == 1; see
+ * flashloop_paper_kv for the format).  k_new / v_new are float32 [rows, H, dh]
+ * with row a the a-th token of active[0..*n_active) (loop 1: every token,
+ * active may be NULL), keys after RoPE.  Body tokens are quantised (loop 1:
+ * the values; loop r >= 2: the residual against the reconstruction of loop
+ * r-1, with x - minimum and the division by the scale in IEEE float32 and
+ * round-half-even, codes clamped to 0..15, a zero scale giving code 0); tail
+ * tokens store bf16(x) in tail[loop-1].  The slot map of loop r (st->slot) must
+ * hold the loop's active list.  [FlashLoop App. E; the "Quadruples the Bill"
+ * page, §3.] */
+int flashloop_paper_kv_quant(const flashloop_params* p, int32_t loop, const float* k_new, const float* v_new,
+                             const int32_t* active, const int32_t* n_active, flashloop_state* st, void* stream);
 
 /* (a2)+(a3) fused: the gathered projection of flashloop_qkv_gathered whose
  * epilogue quantises k and v of loop `loop` straight into the state's

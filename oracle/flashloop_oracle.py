@@ -371,8 +371,8 @@ class PaperKVStream:
             return dequantize_asym(codes[rows], s16[rows], lo16[rows]).reshape(rows.size, self.H, self.dh)
         G = self.group
         grp, off = rows // G, rows % G
-        full = dequantize_asym(codes[grp], s16[grp], lo16[grp])          # [r, H, dh, G]
-        return np.take_along_axis(full, off[:, None, None, None], axis=3)[..., 0]
+        c = codes[grp, :, :, off]                                        # [r, H, dh]: row `off` of group `grp`
+        return c.astype(np.float32) * s16[grp].astype(np.float32) + lo16[grp].astype(np.float32)
 
     # -- loop 1 ---------------------------------------------------------------
     def write_base(self, x):

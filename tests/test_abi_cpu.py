@@ -42,6 +42,8 @@ int main(void) {
          offsetof(flashloop_state, colmass));
   printf("%zu %zu %zu %zu\n", offsetof(flashloop_params, gate_topk), offsetof(flashloop_params, fixed_mass),
          offsetof(flashloop_params, attn_pairs), offsetof(flashloop_state, G));
+  printf("%zu %zu %zu %zu %zu\n", offsetof(flashloop_params, kv_scheme), sizeof(flashloop_paper_kv),
+         offsetof(flashloop_paper_kv, tail), offsetof(flashloop_state, paper_k), offsetof(flashloop_state, paper_v));
   return 0;
 }
 '''
@@ -57,7 +59,8 @@ int main(void) {
             F.StateC.n_active.offset, F.StateC.workspace_bytes.offset,
             F.StateC.cols.offset, F.StateC.rope_cs.offset, F.StateC.colmass.offset,
             F.Params.gate_topk.offset, F.Params.fixed_mass.offset, F.Params.attn_pairs.offset,
-            F.StateC.G.offset]
+            F.StateC.G.offset, F.Params.kv_scheme.offset, ctypes.sizeof(F.PaperKV), F.PaperKV.tail.offset,
+            F.StateC.paper_k.offset, F.StateC.paper_v.offset]
     assert got == want
 
 
