@@ -624,35 +624,220 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
   }
 }
 
-// The running update of loops >= 2 with the row pass split by tiles instead
-// of by columns ("ping-pong"): row group 0 (warps 0-3) handles the tiles with
-// an even block-wide tile counter, group 1 (warps 4-7) the odd ones, one
-// thread per row over all 64 new and 64 old columns of its tile.  While one
-// group computes the exponentials of tile t, the other loads and reduces tile
-// t+1, so the exponential unit and the tensor pipe stay busy across tiles.
+// The running update of loops >= 2 ("ping-pong" kernel).
+//
+// Row pass split by tiles: row group 0 (warps 0-3) handles the tiles with an
+// even block-wide tile counter, group 1 (warps 4-7) the odd ones, one thread
+// per row over all 64 new and 64 old columns of its tile.  While one group
+// computes the exponentials of tile t, the other loads and reduces tile t+1.
 // The row's reference (log2 units) passes from the group of tile t to the
 // group of tile t+1 through shared memory at a named barrier (an arrive on
 // one side, a sync on the other; one barrier per group and lane quarter).
 // Only the new scores can raise it: the old scores are the previous loop's,
 // already within 8 of the reference it left behind, and the reference never
-// decreases.  Each group keeps its own part of Z in the frame of the last tile
-// it handled; the parts are brought to the final frame at the end of the
+// decreases.  Each group keeps its own part of Z in the frame of the last
+// tile it handled; the parts are brought to the final frame at the end of the
 // item.  The rare raise rescales the whole row of N (after P(t-1).V) in the
-// handling thread.  Producer and MMA roles are those of attn_tc_kernel.
+// handling thread.
+//
+// TMEM: Q_new | Q_old (fp16 pairs), N (f32), one score buffer
+// [S_new | S_old] and two P buffers [P_new | -P_old] (fp16 pairs).  The rows
+// copy S_new(t) to registers and release its half of the score buffer at
+// once (then S_old(t) the same way, after the new exponentials), so S(t+1)
+// is computed while they take the exponentials of S(t); P(t) goes to P
+// buffer t & 1 and P(t).V runs behind.  Two threads issue the MMAs: one the score
+// MMAs (as soon as the buffer is free and the K tiles are in), one the P.V
+// MMAs (as soon as P and the V tiles are in), so that neither kind waits
+// for the other.  K and V arrive in two rings of kAtStages slots (a slot
+// holds the new and the old tile): a K slot is released when its score MMAs
+// complete, a V slot after its P.V.  One thread loads each ring.
+constexpr int kPpThreads = 384;  // 8 row warps; K loads (+ TMEM allocation), S MMAs, V loads, P.V MMAs
+
 template <int DH>
-__global__ void __launch_bounds__(kAtThreads, 1)
+struct PpCfg {
+  static constexpr uint32_t kColQn = 0;
+  static constexpr uint32_t kColQo = DH / 2;
+  static constexpr uint32_t kColN = DH;
+  static constexpr uint32_t kColS = 2 * DH;        // S_new at +0, S_old at +64
+  static constexpr uint32_t kColP = 2 * DH + 128;  // P buffer b at +64 b: P_new at +0, -P_old at +32
+};
+
+template <int DH, bool IS_V>
+__device__ __forceinline__ void pp_load_role(uint8_t* ring, uint64_t* full, uint64_t* empty, const CUtensorMap* tn,
+                                             const CUtensorMap* to, const AtArgs& g, int n_rows, int row_tiles,
+                                             int total, volatile int* abort_flag) {
+  using C = AtCfg<DH>;
+  constexpr uint32_t kPart = IS_V ? C::kVBytes : C::kKBytes;
+  int stage = 0;
+  uint32_t phase = 0;
+  int issued[kAtStages];
+  for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
+  for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
+    const int h = item / row_tiles, rt = item % row_tiles;
+    const int nt = at_tiles(g, h, rt, n_rows);
+    for (int t = 0; t < nt && !*abort_flag; ++t) {
+      if (!mbar_wait_sleep(&empty[stage], phase ^ 1)) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      uint8_t* st = ring + stage * 2 * kPart;
+      mbar_arrive_expect_tx(&full[stage], 2 * kPart);
+      if (IS_V) {
+        tma_load_3d(st, tn, t * kAtCols, 0, h, &full[stage]);
+        tma_load_3d(st + kPart, to, t * kAtCols, 0, h, &full[stage]);
+      } else {
+#pragma unroll
+        for (int c = 0; c < DH / 64; ++c) tma_load_3d(st + c * (kAtCols * 128), tn, c * 64, t * kAtCols, h, &full[stage]);
+#pragma unroll
+        for (int c = 0; c < DH / 64; ++c)
+          tma_load_3d(st + kPart + c * (kAtCols * 128), to, c * 64, t * kAtCols, h, &full[stage]);
+      }
+      issued[stage] = phase;
+      if (++stage == kAtStages) {
+        stage = 0;
+        phase ^= 1;
+      }
+    }
+  }
+  // never leave with a copy in flight: wait (bounded) for the last load of every slot
+  for (int s2 = 0; s2 < kAtStages; ++s2)
+    if (issued[s2] >= 0) (void)mbar_wait(&full[s2], (uint32_t)issued[s2]);
+}
+
+// Score-MMA role (one thread): S(t) = [Q_new K_new^T | Q_old K_old^T] into the
+// score buffer once the rows have copied S(t-1) out, the K slot released when
+// the MMAs complete.
+// s_empty: [0] the S_new half of the buffer, [1] the S_old half (one
+// completion per tile, waited here in order).  s_full: [half * 2 + (t & 1)],
+// one barrier per half and tile parity, so that each row group waits only on
+// barriers that complete on its own tiles (a phase it waits for is never two
+// completions behind).
+template <int DH>
+__device__ __forceinline__ void pp_s_role(const uint8_t* kring, uint64_t* k_full, uint64_t* k_empty, uint64_t* s_full,
+                                          uint64_t* s_empty, uint64_t* q_ready, volatile int* abort_flag,
+                                          uint32_t tmem, const AtArgs& g, int n_rows, int row_tiles, int total) {
+  using C = AtCfg<DH>;
+  using P = PpCfg<DH>;
+  int ks = 0;
+  uint32_t kph = 0, u = 0, item_no = 0;
+  bool ok = true;
+  for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x, ++item_no) {
+    const int h = item / row_tiles, rt = item % row_tiles;
+    const int nt = at_tiles(g, h, rt, n_rows);
+    if (!mbar_wait_sleep(q_ready, item_no & 1)) {
+      ok = false;
+      break;
+    }
+    for (int t = 0; t < nt; ++t, ++u) {
+      const uint32_t k_addr = smem_u32(kring + ks * 2 * C::kKBytes);
+      // S_new(t) once the K tiles are in and the rows copied S_new(t-1) out
+      if (!mbar_wait_sleep(&k_full[ks], kph) || (u > 0 && !mbar_wait_sleep(&s_empty[0], (u - 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint32_t kd = k_addr + (kk >> 2) * (kAtCols * 128) + (kk & 3) * 32;
+        umma_f16_ts(tmem + P::kColS, tmem + P::kColQn + kk * 8, sw128_kmajor_desc(kd), C::kIdescS, kk > 0);
+      }
+      umma_commit(&s_full[u & 1]);
+      // S_old(t) once the rows copied S_old(t-1) out
+      if (u > 0 && !mbar_wait_sleep(&s_empty[1], (u - 1) & 1)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < DH / 16; ++kk) {
+        const uint32_t kd = k_addr + C::kKBytes + (kk >> 2) * (kAtCols * 128) + (kk & 3) * 32;
+        umma_f16_ts(tmem + P::kColS + 64, tmem + P::kColQo + kk * 8, sw128_kmajor_desc(kd), C::kIdescS, kk > 0);
+      }
+      umma_commit(&s_full[2 + (u & 1)]);
+      umma_commit(&k_empty[ks]);
+      if (++ks == kAtStages) {
+        ks = 0;
+        kph ^= 1;
+      }
+    }
+  }
+  if (!ok) {
+    set_error(g.err, kDevErrTimeout);
+    *abort_flag = 1;
+  }
+}
+
+// P.V role (one thread): N += [P_new | -P_old] [V_new; V_old] for every tile
+// once its P buffer and V tiles are in, the V slot released when it completes.
+// pv_done[t & 1] and pv_done4[t & 3] both complete when P(t).V has: a row
+// group waits on pv_done for its own tiles and on pv_done4 for the other
+// group's (four barriers keep that wait within one phase, see the rows).
+template <int DH>
+__device__ __forceinline__ void pp_pv_role(const uint8_t* vring, uint64_t* v_full, uint64_t* v_empty,
+                                           uint64_t* p_full, uint64_t* pv_done, uint64_t* pv_done4,
+                                           volatile int* abort_flag,
+                                           uint32_t tmem, const AtArgs& g, int n_rows, int row_tiles, int total) {
+  using C = AtCfg<DH>;
+  using P = PpCfg<DH>;
+  int vs = 0;
+  uint32_t vph = 0, u = 0;
+  bool ok = true;
+  for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x) {
+    const int h = item / row_tiles, rt = item % row_tiles;
+    const int nt = at_tiles(g, h, rt, n_rows);
+    for (int t = 0; t < nt; ++t, ++u) {
+      if (!mbar_wait_sleep(&p_full[u & 1], (u >> 1) & 1) || !mbar_wait_sleep(&v_full[vs], vph)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t pcol = tmem + P::kColP + (u & 1) * 64;
+      const uint32_t v_addr = smem_u32(vring + vs * 2 * C::kVBytes);
+#pragma unroll
+      for (int kk = 0; kk < kAtCols / 16; ++kk)
+        umma_f16_ts(tmem + P::kColN, pcol + kk * 8, sw128_kmajor_desc(v_addr + kk * 32), C::kIdescPV, 1u);
+#pragma unroll
+      for (int kk = 0; kk < kAtCols / 16; ++kk)
+        umma_f16_ts(tmem + P::kColN, pcol + 32 + kk * 8, sw128_kmajor_desc(v_addr + C::kVBytes + kk * 32),
+                    C::kIdescPV, 1u);
+      umma_commit(&v_empty[vs]);
+      umma_commit(&pv_done[u & 1]);
+      umma_commit(&pv_done4[u & 3]);
+      if (++vs == kAtStages) {
+        vs = 0;
+        vph ^= 1;
+      }
+    }
+  }
+  if (!ok) {
+    set_error(g.err, kDevErrTimeout);
+    *abort_flag = 1;
+  }
+}
+
+template <int DH>
+__global__ void __launch_bounds__(kPpThreads, 1)
 attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant__ CUtensorMap tm_ko,
                const __grid_constant__ CUtensorMap tm_vn, const __grid_constant__ CUtensorMap tm_vo, AtArgs g) {
   using C = AtCfg<DH>;
+  using P = PpCfg<DH>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  // K ring: kAtStages slots of [K_new | K_old]; V ring: slots of [V_new^T | V_old^T]
+  uint8_t* kring = smem;
+  uint8_t* vring = smem + kAtStages * 2 * C::kKBytes;
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kAtStages * C::kStageBytes);
-  uint64_t* kv_full = bars;
-  uint64_t* kv_empty = bars + kAtStages;
-  uint64_t* s_full = bars + 2 * kAtStages;
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 2;
-  uint64_t* q_ready = pv_done + 2;
+  uint64_t* k_full = bars;                   // [stages]
+  uint64_t* k_empty = bars + kAtStages;      // [stages]
+  uint64_t* v_full = bars + 2 * kAtStages;   // [stages]
+  uint64_t* v_empty = bars + 3 * kAtStages;  // [stages]
+  uint64_t* s_full = bars + 4 * kAtStages;   // [4] S_new(t) / S_old(t) landed: [half * 2 + (t & 1)]
+  uint64_t* s_empty = s_full + 4;            // [2] the rows copied S_new(t) / S_old(t) out
+  uint64_t* p_full = s_empty + 2;            // [2] P(t) in P buffer t & 1
+  uint64_t* pv_done = p_full + 2;            // [2] P(t).V complete, by t & 1
+  uint64_t* pv_done4 = pv_done + 2;          // [4] P(t).V complete, by t & 3
+  uint64_t* q_ready = pv_done4 + 4;          // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(q_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -665,12 +850,18 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAtStages; ++s) {
-      mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_full[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&v_empty[s], 1);
+    }
+    for (int b = 0; b < 4; ++b) {
+      mbar_init(&s_full[b], 1);
+      mbar_init(&pv_done4[b], 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&s_full[b], 1);
-      mbar_init(&p_full[b], kAtRowThreads / 2);  // the 128 threads of the tile's group
+      mbar_init(&s_empty[b], kAtRowThreads / 2);  // the 128 threads of the tile's group
+      mbar_init(&p_full[b], kAtRowThreads / 2);
       mbar_init(&pv_done[b], 1);
     }
     mbar_init(q_ready, kAtRowThreads);
@@ -686,11 +877,18 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
-  const AtBars B{kv_full, kv_empty, s_full, p_full, pv_done, q_ready, abort_flag};
   if (warp == 8) {
-    at_load_role<DH, kAtRunning>(smem, B, &tm_kn, &tm_ko, &tm_vn, &tm_vo, g, n_rows, row_tiles, total, true, lane);
+    if (lane == 0)
+      pp_load_role<DH, false>(kring, k_full, k_empty, &tm_kn, &tm_ko, g, n_rows, row_tiles, total, abort_flag);
   } else if (warp == 9) {
-    at_mma_role<DH, kAtRunning>(smem, B, tmem, g, n_rows, row_tiles, total, true, lane);
+    if (lane == 0)
+      pp_s_role<DH>(kring, k_full, k_empty, s_full, s_empty, q_ready, abort_flag, tmem, g, n_rows, row_tiles, total);
+  } else if (warp == 10) {
+    if (lane == 0)
+      pp_load_role<DH, true>(vring, v_full, v_empty, &tm_vn, &tm_vo, g, n_rows, row_tiles, total, abort_flag);
+  } else if (warp == 11) {
+    if (lane == 0)
+      pp_pv_role<DH>(vring, v_full, v_empty, p_full, pv_done, pv_done4, abort_flag, tmem, g, n_rows, row_tiles, total);
   } else {
     // A named barrier cannot time out, so both groups always execute the same
     // barrier sequence: after a failed wait (or an abort raised elsewhere) a
@@ -746,7 +944,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       // rebuilt keys carry log2(e)/sqrt(dh), so S is in log2 units.
       if (!dead) {
         const uint16_t* qsrc = grp == 0 ? g.q_new : g.q_old;
-        const uint32_t qcol = grp == 0 ? C::kColQn : C::kColQo;
+        const uint32_t qcol = grp == 0 ? P::kColQn : P::kColQo;
         uint32_t qv[DH / 16][8];
 #pragma unroll
         for (int v = 0; v < DH / 16; ++v) {
@@ -787,7 +985,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 #pragma unroll
           for (int e = 0; e < 16; ++e) r[e] = nv[c0 / 8 + e / 8][e % 8];
           __syncwarp();
-          tmem_st16(tmem + lane_base + C::kColN + grp * kHalfCols + c0, r);
+          tmem_st16(tmem + lane_base + P::kColN + grp * kHalfCols + c0, r);
         }
         tmem_wait_st();
         tc_fence_before();
@@ -816,27 +1014,29 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         if ((int)b != grp) continue;  // the other group's tile
         const int nvalid = min(max(nc_row - t * kAtCols, 0), kAtCols);
         wait_or_die(&s_full[b], (u >> 1) & 1);
-        const uint32_t sbase = tmem + lane_base + C::kColS + b * 128;
         uint32_t sc[64];
         float mx = -INFINITY;
         if (!dead) {
+          // copy S_new(t) out and hand its half of the score buffer back at once
           __syncwarp();
-          tmem_ld32(sbase, *reinterpret_cast<uint32_t(*)[32]>(sc));
-          tmem_ld32(sbase + 32, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
+          tmem_ld32(tmem + lane_base + P::kColS, *reinterpret_cast<uint32_t(*)[32]>(sc));
+          tmem_ld32(tmem + lane_base + P::kColS + 32, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
           tmem_wait_ld();
+          tc_fence_before();
+          mbar_arrive(&s_empty[0]);
           if (nvalid < kAtCols) {
 #pragma unroll
             for (int e = 0; e < 64; ++e)
               if (e >= nvalid) sc[e] = 0xff800000u;  // -inf
           }
-          float t32[32];
+          // eight running maxima (short chains, few live registers next to the
+          // 128 scores)
+          float m8[8];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) t32[e] = fmaxf(__uint_as_float(sc[e]), __uint_as_float(sc[e + 32]));
+          for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sc[e]);
 #pragma unroll
-          for (int w = 16; w > 0; w >>= 1)
-#pragma unroll
-            for (int e = 0; e < w; ++e) t32[e] = fmaxf(t32[e], t32[e + w]);
-          mx = t32[0];
+          for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sc[e]));
+          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
         }
         // the reference after tile t-1 (this item's), from the other group
         float m_prev = m_init;
@@ -851,25 +1051,32 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           named_bar_arrive(bar_give, 64);
         }
         if (dead) continue;
+        // P buffer b still feeds P(u-2).V until that completes (this group's
+        // own previous tile: pv_done[b] is then one phase from that wait)
+        if (u >= 2) {
+          wait_or_die(&pv_done[b], ((u - 2) >> 1) & 1);
+          if (dead) continue;
+        }
         if (__any_sync(0xffffffffu, need)) {
           // raise the reference of this warp's rows: N scales by 2^(m_prev - m_ref)
-          // once P(t-1).V has landed
+          // once P(t-1).V has landed.  P(u-2).V is complete (above), so is
+          // P(u-5).V, the previous completion of pv_done4[(u-1) & 3].
           const float f = need ? ex2(m_prev - m_ref) : 1.f;
           if (t > 0) {
             const uint32_t up = u - 1;
-            wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+            wait_or_die(&pv_done4[up & 3], (up >> 2) & 1);
             if (dead) continue;
           }
 #pragma unroll 1
           for (int cc = 0; cc < DH; cc += 16) {
             uint32_t r[16];
             __syncwarp();
-            tmem_ld16(tmem + lane_base + C::kColN + cc, r);
+            tmem_ld16(tmem + lane_base + P::kColN + cc, r);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
             __syncwarp();
-            tmem_st16(tmem + lane_base + C::kColN + cc, r);
+            tmem_st16(tmem + lane_base + P::kColN + cc, r);
           }
           tmem_wait_st();
         }
@@ -877,7 +1084,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           z_part *= ex2(frame - m_ref);
           frame = m_ref;
         }
-        // P_new = 2^(S_new - m_ref) over columns [0, 32) of the buffer (fp16 pairs)
+        const uint32_t pbase = tmem + lane_base + P::kColP + b * 64;
+        // P_new = 2^(S_new - m_ref) over columns [0, 32) of the P buffer (fp16 pairs)
         float za[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -890,13 +1098,17 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
             pk[e2] = pack_half2(p0, p1);
           }
           __syncwarp();
-          tmem_st16(sbase + 16 * hf, pk);
+          tmem_st16(pbase + 16 * hf, pk);
         }
         // -P_old = -2^(S_old - m_ref) over columns [32, 64)
+        wait_or_die(&s_full[2 + b], (u >> 1) & 1);
+        if (dead) continue;
         __syncwarp();
-        tmem_ld32(sbase + 64, *reinterpret_cast<uint32_t(*)[32]>(sc));
-        tmem_ld32(sbase + 96, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
+        tmem_ld32(tmem + lane_base + P::kColS + 64, *reinterpret_cast<uint32_t(*)[32]>(sc));
+        tmem_ld32(tmem + lane_base + P::kColS + 96, *reinterpret_cast<uint32_t(*)[32]>(sc + 32));
         tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&s_empty[1]);
         if (nvalid < kAtCols) {
 #pragma unroll
           for (int e = 0; e < 64; ++e)
@@ -914,16 +1126,19 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
             pk[e2] = pack_half2(-p0, -p1);
           }
           __syncwarp();
-          tmem_st16(sbase + 32 + 16 * hf, pk);
+          tmem_st16(pbase + 32 + 16 * hf, pk);
         }
         z_part += ((za[0] + za[1]) + (za[2] + za[3])) - ((zb[0] + zb[1]) + (zb[2] + zb[3]));
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(&p_full[b]);
       }
-      if (nt > 0) {  // every contribution of the item has reached N
+      if (nt > 0) {
+        // every contribution of the item has reached N.  Each group has seen
+        // P(last-2).V or P(last-3).V complete at its own last tile, so the
+        // previous completion of pv_done4[last & 3], P(last-4).V, is too.
         const uint32_t up = u - 1;
-        wait_or_die(&pv_done[up & 1], (up >> 1) & 1);
+        wait_or_die(&pv_done4[up & 3], (up >> 2) & 1);
       }
       // the two parts of Z in the final frame (frames only rise: the larger)
       xz[grp * 128 + row] = z_part;
@@ -941,7 +1156,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
       for (int cc = 0; cc < kHalfCols; cc += 16) {
         uint32_t r[16];
         __syncwarp();
-        tmem_ld16(tmem + lane_base + C::kColN + grp * kHalfCols + cc, r);
+        tmem_ld16(tmem + lane_base + P::kColN + grp * kHalfCols + cc, r);
         tmem_wait_ld();
         if (tok >= 0) {
           const int col = grp * kHalfCols + cc;
@@ -985,11 +1200,12 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 // thread (no cross-lane reduction).  A work item = 128 selected columns of
 // one head; it walks 64-row tiles from the first row whose token reaches the
 // item's smallest column token.  Rows come prepared per head: fp16 q (the
-// same type as the keys, as kind::f16 requires), 2^-m scale as m in log2
-// units, 1/Z and the row token.
+// same type as the keys, as kind::f16 requires), the frame m_i + log2(Z_i)
+// in log2 units (so a contribution is one exp2: 2^(s - m) / Z = 2^(s - frame))
+// and the row token.
 // Roles: warps 0-7 reduce (two per TMEM lane quarter, each 32 of a tile's 64
 // rows) and load the item's keys into TMEM (A operand); warp 8 allocates TMEM
-// and streams the row tiles (TMA for q, bulk copies for m, 1/Z, tokens);
+// and streams the row tiles (TMA for q, bulk copies for frames and tokens);
 // warp 9 issues the MMAs.  All waits are bounded.
 // ---------------------------------------------------------------------------
 constexpr int kCmtCols = 128, kCmtRows = 64, kCmtStages = 4, kCmtThreads = 320;
@@ -998,7 +1214,8 @@ constexpr int kCmtRowThreads = 256;
 template <int DH>
 struct CmtCfg {
   static constexpr int kQBytes = kCmtRows * DH * 2;  // q tile: 64 rows x DH (DH/64 swizzle chunks)
-  static constexpr int kSideBytes = 1024;            // m2, rz, tokens of the tile (3 x 256 B), padded
+  static constexpr int kSideBytes = 1024;            // frames and tokens of the tile (2 x 256 B); keeps
+                                                     // every stage's q tile on a 1024-byte swizzle atom
   static constexpr int kStageBytes = kQBytes + kSideBytes;
   static constexpr int kSmem = 1024 + kCmtStages * kStageBytes + 256 + 2 * 128 * 4;
   static constexpr uint32_t kColA = 0;       // keys, fp16 pairs: DH/2 columns
@@ -1012,8 +1229,7 @@ struct CmtArgs {
   int row_cap;
   const int32_t* cols;        // [H, kc] ascending tokens (NULL: identity)
   const int32_t* rtok;        // [n_cap] row tokens, -1 past the last row
-  const float* m2;            // [H, n_cap] row max, log2 units
-  const float* rz;            // [H, n_cap] 1 / Z
+  const float* m2;            // [H, n_cap] row frame m_i + log2(Z_i / g_i), log2 units (+inf: no row)
   const __half* k;            // [H, kcp, DH] rebuilt keys
   float* out;                 // [H, S], written at the column tokens
   int32_t* err;
@@ -1112,14 +1328,13 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
           }
           uint8_t* st = smem + stage * C::kStageBytes;
           const int a0 = a_begin + t * kCmtRows;
-          mbar_arrive_expect_tx(&full[stage], C::kQBytes + 3 * kCmtRows * 4);
+          mbar_arrive_expect_tx(&full[stage], C::kQBytes + 2 * kCmtRows * 4);
 #pragma unroll
           for (int c = 0; c < DH / 64; ++c)
             tma_load_3d(st + c * (kCmtRows * 128), &tm_q, c * 64, a0, h, &full[stage]);
           uint8_t* side = st + C::kQBytes;
           bulk_g2s(side, g.m2 + (size_t)h * g.n_cap + a0, kCmtRows * 4, &full[stage]);
-          bulk_g2s(side + 256, g.rz + (size_t)h * g.n_cap + a0, kCmtRows * 4, &full[stage]);
-          bulk_g2s(side + 512, g.rtok + a0, kCmtRows * 4, &full[stage]);
+          bulk_g2s(side + 256, g.rtok + a0, kCmtRows * 4, &full[stage]);
           issued[stage] = phase;
           if (++stage == kCmtStages) {
             stage = 0;
@@ -1228,15 +1443,33 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
           __syncwarp();
           tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + half * 32, r);
           tmem_wait_ld();
+          // p = 2^(s - m_i) / Z_i * g_i = 2^(s - frame_i); rows past the last
+          // have frame +inf (p = 0).  Row tokens ascend, so only a tile whose
+          // first row lies before this column's token needs the causal mask.
           const uint8_t* side = smem + stage * C::kStageBytes + C::kQBytes;
-          const float* sm2 = reinterpret_cast<const float*>(side) + half * 32;
-          const float* srz = reinterpret_cast<const float*>(side + 256) + half * 32;
-          const int* stok = reinterpret_cast<const int*>(side + 512) + half * 32;
+          const float4* sm4 = reinterpret_cast<const float4*>(side) + half * 8;
+          const int* stok = reinterpret_cast<const int*>(side + 256) + half * 32;
           float pa[4] = {0.f, 0.f, 0.f, 0.f};
+          if (stok[0] >= ctok) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = ex2(__uint_as_float(r[e]) - sm2[e]) * srz[e];
-            pa[e & 3] += stok[e] >= ctok ? v : 0.f;
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 f = sm4[e4];
+              pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
+              pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
+              pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
+              pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
+            }
+          } else {
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+              const float4 f = sm4[e4];
+              const float fr[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float v = ex2(__uint_as_float(r[4 * e4 + k]) - fr[k]);
+                pa[k] += stok[4 * e4 + k] >= ctok ? v : 0.f;
+              }
+            }
           }
           acc += (pa[0] + pa[1]) + (pa[2] + pa[3]);
           tc_fence_before();
@@ -1264,11 +1497,11 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
   }
 }
 
-// Rows of the column mass, per head: fp16 q, m in log2 units, 1/Z, and the
-// row tokens (-1 past the last row, up to n_cap).
+// Rows of the column mass, per head: fp16 q, the frame m + log2(Z / g) in
+// log2 units, and the row tokens (-1 past the last row, up to n_cap).
 template <int DH>
 __global__ void __launch_bounds__(256)
-colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, float* rz, int32_t* rtok) {
+colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, int32_t* rtok) {
   int n_rows = a.n_rows ? *a.n_rows : a.S;
   if (n_rows > a.row_cap) n_rows = a.row_cap;
   const int lane = threadIdx.x & 31;
@@ -1296,9 +1529,15 @@ colmass_prep_kernel(const ColmassArgs a, int n_cap, __half* q16, float* m2, floa
 #pragma unroll
     for (int e = 0; e < E; ++e) qd[lane * E + e] = __float2half_rn(x[e]);
     if (lane == 0) {
-      m2[(size_t)h * n_cap + r] = tok >= 0 ? a.m[(size_t)h * a.S + tok] * kAtLog2e : 0.f;
-      rz[(size_t)h * n_cap + r] =
-          tok >= 0 ? (a.g ? a.g[(size_t)h * a.S + tok] : 1.f) / a.z[(size_t)h * a.S + tok] : 0.f;
+      // the row's frame: 2^(s - m) * g / Z = 2^(s - (m + log2(Z / g))); no row, or
+      // g = 0, gives +inf (a zero contribution)
+      float fr = INFINITY;
+      if (tok >= 0) {
+        const size_t hi = (size_t)h * a.S + tok;
+        const float gz = (a.g ? a.g[hi] : 1.f) / a.z[hi];
+        if (gz > 0.f) fr = a.m[hi] * kAtLog2e - log2f(gz);
+      }
+      m2[(size_t)h * n_cap + r] = fr;
       if (h == 0) rtok[r] = tok;
     }
   }
@@ -1392,20 +1631,19 @@ int at_sm_count() {
 }
 
 // Column mass of loop `a` on the tensor cores (prep + kernel).  scratch_q
-// holds [H, n_cap, dh] fp16, scratch_rows [H, n_cap] x 2 floats + [n_cap] ints.
+// holds [H, n_cap, dh] fp16, scratch_rows [H, n_cap] floats + [n_cap] ints.
 int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scratch_q, void* scratch_rows,
                       cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
   const int n_cap = ((a.row_cap + kCmtRows - 1) / kCmtRows) * kCmtRows;
   __half* q16 = static_cast<__half*>(scratch_q);
   float* m2 = static_cast<float*>(scratch_rows);
-  float* rz = m2 + (size_t)H * n_cap;
-  int32_t* rtok = reinterpret_cast<int32_t*>(rz + (size_t)H * n_cap);
+  int32_t* rtok = reinterpret_cast<int32_t*>(m2 + (size_t)H * n_cap);
   long long items = (long long)n_cap * H;
   int pgrid = (int)((items + 7) / 8);
   if (pgrid > 148 * 16) pgrid = 148 * 16;
-  if (dh == 128) colmass_prep_kernel<128><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rz, rtok);
-  else colmass_prep_kernel<64><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rz, rtok);
+  if (dh == 128) colmass_prep_kernel<128><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rtok);
+  else colmass_prep_kernel<64><<<pgrid, 256, 0, stream>>>(a, n_cap, q16, m2, rtok);
   int rc = launch_status();
   if (rc != FLASHLOOP_OK) return rc;
   CUtensorMap tq;
@@ -1413,7 +1651,7 @@ int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scr
   if (rc != FLASHLOOP_OK) return rc;
   CmtArgs g{};
   g.S = a.S; g.H = H; g.kc = a.kc; g.kcp = a.kcp; g.n_cap = n_cap; g.n_rows = a.n_rows; g.row_cap = a.row_cap;
-  g.cols = a.cols; g.rtok = rtok; g.m2 = m2; g.rz = rz; g.k = a.k_new; g.out = a.out; g.err = a.err;
+  g.cols = a.cols; g.rtok = rtok; g.m2 = m2; g.k = a.k_new; g.out = a.out; g.err = a.err;
   const int max_items = ((a.kc + kCmtCols - 1) / kCmtCols) * H;
   int grid = at_sm_count();
   if (grid > max_items) grid = max_items;
@@ -1474,16 +1712,21 @@ int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaSt
     kernel<<<grid, kAtThreads, smem, stream>>>(tkn, tko, tvn, tvo, g);
     return FLASHLOOP_OK;
   };
+  auto launch_pp = [&](auto kernel, int smem) -> int {
+    FL_TRY(cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem));
+    kernel<<<grid, kPpThreads, smem, stream>>>(tkn, tko, tvn, tvo, g);
+    return FLASHLOOP_OK;
+  };
   // the running update: the ping-pong row pass; the fixed-mass passes: the
   // column-split row pass of attn_tc_kernel
   if (dh == 128) {
     if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<128, kAtFixedMassStats>, AtCfg<128>::kSmem);
     else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<128, kAtFixedMassUpdate>, AtCfg<128>::kSmem);
-    else rc = launch(attn_pp_kernel<128>, AtCfg<128>::kSmem);
+    else rc = launch_pp(attn_pp_kernel<128>, AtCfg<128>::kSmem);
   } else {
     if (a.mode == kAtFixedMassStats) rc = launch(attn_tc_kernel<64, kAtFixedMassStats>, AtCfg<64>::kSmem);
     else if (a.mode == kAtFixedMassUpdate) rc = launch(attn_tc_kernel<64, kAtFixedMassUpdate>, AtCfg<64>::kSmem);
-    else rc = launch(attn_pp_kernel<64>, AtCfg<64>::kSmem);
+    else rc = launch_pp(attn_pp_kernel<64>, AtCfg<64>::kSmem);
   }
   if (rc != FLASHLOOP_OK) return rc;
   return launch_status();
