@@ -645,13 +645,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 // copy S_new(t) to registers and release its half of the score buffer at
 // once (then S_old(t) the same way, after the new exponentials), so S(t+1)
 // is computed while they take the exponentials of S(t); P(t) goes to P
-// buffer t & 1 and P(t).V runs behind.  Two threads issue the MMAs: one the score
-// MMAs (as soon as the buffer is free and the K tiles are in), one the P.V
-// MMAs (as soon as P and the V tiles are in), so that neither kind waits
-// for the other.  K and V arrive in two rings of kAtStages slots (a slot
+// buffer t & 1 and P(t).V runs behind.  Three threads issue the MMAs (S_new,
+// S_old, P.V), each as soon as its inputs are in, so that none waits behind
+// another's MMAs.  K and V arrive in two rings of kAtStages slots (a slot
 // holds the new and the old tile): a K slot is released when its score MMAs
-// complete, a V slot after its P.V.  One thread loads each ring.
-constexpr int kPpThreads = 384;  // 8 row warps; K loads (+ TMEM allocation), S MMAs, V loads, P.V MMAs
+// complete, a V slot after its P.V.  One thread loads both rings.
+constexpr int kPpThreads = 384;  // 8 row warps; loads (+ TMEM allocation), S_new MMAs, S_old MMAs, P.V MMAs
 
 template <int DH>
 struct PpCfg {
@@ -662,77 +661,39 @@ struct PpCfg {
   static constexpr uint32_t kColP = 2 * DH + 128;  // P buffer b at +64 b: P_new at +0, -P_old at +32
 };
 
-template <int DH, bool IS_V>
-__device__ __forceinline__ void pp_load_role(uint8_t* ring, uint64_t* full, uint64_t* empty, const CUtensorMap* tn,
-                                             const CUtensorMap* to, const AtArgs& g, int n_rows, int row_tiles,
-                                             int total, volatile int* abort_flag) {
-  using C = AtCfg<DH>;
-  constexpr uint32_t kPart = IS_V ? C::kVBytes : C::kKBytes;
-  int stage = 0;
-  uint32_t phase = 0;
-  int issued[kAtStages];
-  for (int s2 = 0; s2 < kAtStages; ++s2) issued[s2] = -1;
-  for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
-    const int h = item / row_tiles, rt = item % row_tiles;
-    const int nt = at_tiles(g, h, rt, n_rows);
-    for (int t = 0; t < nt && !*abort_flag; ++t) {
-      if (!mbar_wait_sleep(&empty[stage], phase ^ 1)) {
-        set_error(g.err, kDevErrTimeout);
-        *abort_flag = 1;
-        break;
-      }
-      uint8_t* st = ring + stage * 2 * kPart;
-      mbar_arrive_expect_tx(&full[stage], 2 * kPart);
-      if (IS_V) {
-        tma_load_3d(st, tn, t * kAtCols, 0, h, &full[stage]);
-        tma_load_3d(st + kPart, to, t * kAtCols, 0, h, &full[stage]);
-      } else {
-#pragma unroll
-        for (int c = 0; c < DH / 64; ++c) tma_load_3d(st + c * (kAtCols * 128), tn, c * 64, t * kAtCols, h, &full[stage]);
-#pragma unroll
-        for (int c = 0; c < DH / 64; ++c)
-          tma_load_3d(st + kPart + c * (kAtCols * 128), to, c * 64, t * kAtCols, h, &full[stage]);
-      }
-      issued[stage] = phase;
-      if (++stage == kAtStages) {
-        stage = 0;
-        phase ^= 1;
-      }
-    }
-  }
-  // never leave with a copy in flight: wait (bounded) for the last load of every slot
-  for (int s2 = 0; s2 < kAtStages; ++s2)
-    if (issued[s2] >= 0) (void)mbar_wait(&full[s2], (uint32_t)issued[s2]);
-}
-
-// Score-MMA role (one thread): S(t) = [Q_new K_new^T | Q_old K_old^T] into the
-// score buffer once the rows have copied S(t-1) out, the K slot released when
-// the MMAs complete.
-// s_empty: [0] the S_new half of the buffer, [1] the S_old half (one
-// completion per tile, waited here in order).  s_full: [half * 2 + (t & 1)],
-// one barrier per half and tile parity, so that each row group waits only on
-// barriers that complete on its own tiles (a phase it waits for is never two
-// completions behind).
-template <int DH>
-__device__ __forceinline__ void pp_s_role(const uint8_t* kring, uint64_t* k_full, uint64_t* k_empty, uint64_t* s_full,
-                                          uint64_t* s_empty, uint64_t* q_ready, volatile int* abort_flag,
-                                          uint32_t tmem, const AtArgs& g, int n_rows, int row_tiles, int total) {
+// Score-MMA role of one half (one thread each): S_new(t) = Q_new K_new^T
+// (HALF 0) or S_old(t) = Q_old K_old^T (HALF 1) into its half of the score
+// buffer once the K tiles are in and the rows copied the half of S(t-1) out.
+// A thread that issues tcgen05.mma waits while the tensor pipe takes its
+// MMAs, so the two halves and P.V each have their own thread: none waits
+// behind another's MMAs or hand-offs.  The K slot is released when both
+// halves' MMAs complete (k_empty counts two commits).
+// s_empty: [HALF] (one completion per tile, waited here in order).
+// s_full: [HALF * 2 + (t & 1)], one barrier per half and tile parity, so that
+// each row group waits only on barriers that complete on its own tiles (a
+// phase it waits for is never two completions behind).
+template <int DH, int HALF>
+__device__ __forceinline__ void pp_s_half_role(const uint8_t* kring, uint64_t* k_full, uint64_t* k_empty,
+                                               uint64_t* s_full, uint64_t* s_empty, uint64_t* q_ready,
+                                               volatile int* abort_flag, uint32_t tmem, const AtArgs& g, int n_rows,
+                                               int row_tiles, int total) {
   using C = AtCfg<DH>;
   using P = PpCfg<DH>;
   int ks = 0;
-  uint32_t kph = 0, u = 0, item_no = 0;
+  uint32_t kph = 0, u = 0, item_no = 0;  // item_no counts the items that have tiles
   bool ok = true;
-  for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x, ++item_no) {
+  for (int item = blockIdx.x; item < total && ok && !*abort_flag; item += gridDim.x) {
     const int h = item / row_tiles, rt = item % row_tiles;
     const int nt = at_tiles(g, h, rt, n_rows);
+    if (nt == 0) continue;  // the rows signal q_ready only for items with tiles
     if (!mbar_wait_sleep(q_ready, item_no & 1)) {
       ok = false;
       break;
     }
+    ++item_no;
     for (int t = 0; t < nt; ++t, ++u) {
-      const uint32_t k_addr = smem_u32(kring + ks * 2 * C::kKBytes);
-      // S_new(t) once the K tiles are in and the rows copied S_new(t-1) out
-      if (!mbar_wait_sleep(&k_full[ks], kph) || (u > 0 && !mbar_wait_sleep(&s_empty[0], (u - 1) & 1))) {
+      const uint32_t k_addr = smem_u32(kring + ks * 2 * C::kKBytes) + HALF * C::kKBytes;
+      if (!mbar_wait_sleep(&k_full[ks], kph) || (u > 0 && !mbar_wait_sleep(&s_empty[HALF], (u - 1) & 1))) {
         ok = false;
         break;
       }
@@ -740,21 +701,10 @@ __device__ __forceinline__ void pp_s_role(const uint8_t* kring, uint64_t* k_full
 #pragma unroll
       for (int kk = 0; kk < DH / 16; ++kk) {
         const uint32_t kd = k_addr + (kk >> 2) * (kAtCols * 128) + (kk & 3) * 32;
-        umma_f16_ts(tmem + P::kColS, tmem + P::kColQn + kk * 8, sw128_kmajor_desc(kd), C::kIdescS, kk > 0);
+        umma_f16_ts(tmem + P::kColS + 64 * HALF, tmem + (HALF ? P::kColQo : P::kColQn) + kk * 8,
+                    sw128_kmajor_desc(kd), C::kIdescS, kk > 0);
       }
-      umma_commit(&s_full[u & 1]);
-      // S_old(t) once the rows copied S_old(t-1) out
-      if (u > 0 && !mbar_wait_sleep(&s_empty[1], (u - 1) & 1)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < DH / 16; ++kk) {
-        const uint32_t kd = k_addr + C::kKBytes + (kk >> 2) * (kAtCols * 128) + (kk & 3) * 32;
-        umma_f16_ts(tmem + P::kColS + 64, tmem + P::kColQo + kk * 8, sw128_kmajor_desc(kd), C::kIdescS, kk > 0);
-      }
-      umma_commit(&s_full[2 + (u & 1)]);
+      umma_commit(&s_full[2 * HALF + (u & 1)]);
       umma_commit(&k_empty[ks]);
       if (++ks == kAtStages) {
         ks = 0;
@@ -765,6 +715,63 @@ __device__ __forceinline__ void pp_s_role(const uint8_t* kring, uint64_t* k_full
   if (!ok) {
     set_error(g.err, kDevErrTimeout);
     *abort_flag = 1;
+  }
+}
+
+// Load role (one thread): for every tile the K slot ([K_new | K_old]) and
+// the V slot ([V_new^T | V_old^T]) by TMA, each into its ring once free.
+template <int DH>
+__device__ __forceinline__ void pp_load_role(uint8_t* kring, uint8_t* vring, uint64_t* k_full, uint64_t* k_empty,
+                                             uint64_t* v_full, uint64_t* v_empty, const CUtensorMap* tkn,
+                                             const CUtensorMap* tko, const CUtensorMap* tvn, const CUtensorMap* tvo,
+                                             const AtArgs& g, int n_rows, int row_tiles, int total,
+                                             volatile int* abort_flag) {
+  using C = AtCfg<DH>;
+  int ks = 0, vs = 0;
+  uint32_t kph = 0, vph = 0;
+  int kiss[kAtStages], viss[kAtStages];
+  for (int s2 = 0; s2 < kAtStages; ++s2) kiss[s2] = viss[s2] = -1;
+  for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
+    const int h = item / row_tiles, rt = item % row_tiles;
+    const int nt = at_tiles(g, h, rt, n_rows);
+    for (int t = 0; t < nt && !*abort_flag; ++t) {
+      if (!mbar_wait_sleep(&k_empty[ks], kph ^ 1)) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      uint8_t* st = kring + ks * 2 * C::kKBytes;
+      mbar_arrive_expect_tx(&k_full[ks], 2 * C::kKBytes);
+#pragma unroll
+      for (int c = 0; c < DH / 64; ++c) tma_load_3d(st + c * (kAtCols * 128), tkn, c * 64, t * kAtCols, h, &k_full[ks]);
+#pragma unroll
+      for (int c = 0; c < DH / 64; ++c)
+        tma_load_3d(st + C::kKBytes + c * (kAtCols * 128), tko, c * 64, t * kAtCols, h, &k_full[ks]);
+      kiss[ks] = kph;
+      if (++ks == kAtStages) {
+        ks = 0;
+        kph ^= 1;
+      }
+      if (!mbar_wait_sleep(&v_empty[vs], vph ^ 1)) {
+        set_error(g.err, kDevErrTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      uint8_t* sv = vring + vs * 2 * C::kVBytes;
+      mbar_arrive_expect_tx(&v_full[vs], 2 * C::kVBytes);
+      tma_load_3d(sv, tvn, t * kAtCols, 0, h, &v_full[vs]);
+      tma_load_3d(sv + C::kVBytes, tvo, t * kAtCols, 0, h, &v_full[vs]);
+      viss[vs] = vph;
+      if (++vs == kAtStages) {
+        vs = 0;
+        vph ^= 1;
+      }
+    }
+  }
+  // never leave with a copy in flight: wait (bounded) for the last load of every slot
+  for (int s2 = 0; s2 < kAtStages; ++s2) {
+    if (kiss[s2] >= 0) (void)mbar_wait(&k_full[s2], (uint32_t)kiss[s2]);
+    if (viss[s2] >= 0) (void)mbar_wait(&v_full[s2], (uint32_t)viss[s2]);
   }
 }
 
@@ -851,7 +858,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
   if (threadIdx.x == 0) {
     for (int s = 0; s < kAtStages; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&k_empty[s], 1);
+      mbar_init(&k_empty[s], 2);  // both score halves
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
@@ -879,13 +886,16 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 
   if (warp == 8) {
     if (lane == 0)
-      pp_load_role<DH, false>(kring, k_full, k_empty, &tm_kn, &tm_ko, g, n_rows, row_tiles, total, abort_flag);
+      pp_load_role<DH>(kring, vring, k_full, k_empty, v_full, v_empty, &tm_kn, &tm_ko, &tm_vn, &tm_vo, g, n_rows,
+                       row_tiles, total, abort_flag);
   } else if (warp == 9) {
     if (lane == 0)
-      pp_s_role<DH>(kring, k_full, k_empty, s_full, s_empty, q_ready, abort_flag, tmem, g, n_rows, row_tiles, total);
+      pp_s_half_role<DH, 0>(kring, k_full, k_empty, s_full, s_empty, q_ready, abort_flag, tmem, g, n_rows, row_tiles,
+                            total);
   } else if (warp == 10) {
     if (lane == 0)
-      pp_load_role<DH, true>(vring, v_full, v_empty, &tm_vn, &tm_vo, g, n_rows, row_tiles, total, abort_flag);
+      pp_s_half_role<DH, 1>(kring, k_full, k_empty, s_full, s_empty, q_ready, abort_flag, tmem, g, n_rows, row_tiles,
+                            total);
   } else if (warp == 11) {
     if (lane == 0)
       pp_pv_role<DH>(vring, v_full, v_empty, p_full, pv_done, pv_done4, abort_flag, tmem, g, n_rows, row_tiles, total);
@@ -989,7 +999,9 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(q_ready);
+        // only items with tiles: the score issuers wait on q_ready for those
+        // alone, so the rows can never run two phases ahead of them
+        if (nt > 0) mbar_arrive(q_ready);
         // bring the next item's rows (this thread's q and half of N) into L2
         const int item_next = item + gridDim.x;
         if (item_next < total) {
