@@ -104,7 +104,7 @@ inline Workspace workspace_layout(const flashloop_params* p) {
 // the split of the dense loop-1 pass (nsplit column ranges of `range`
 // columns per sequence) and of the sparse loops (nblk ranges per head).
 struct DecodeLayout {
-  size_t k_new, v_new, scores, part_m, part_mu, part_Z, part_N, total;
+  size_t k_new, v_new, scores, part_m, part_mu, part_Z, part_N, kv_part, total;
   int nsplit, range, nblk;
 };
 

@@ -71,6 +71,8 @@ struct DecodeArgs {
   int nsplit;           // dense: column ranges per sequence
   int range;            // dense: columns per range (multiple of kChunkCols)
   int32_t* err;
+  uint16_t* kv_part;    // [B*H, k, 2, dh] fp16: Khat, Vhat of the selected columns after the last sparse loop
+  int write_part;       // the loop writes Khat^(loop), Vhat^(loop) to kv_part (a later loop reads them)
 };
 
 __device__ __forceinline__ float half_bits_f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
@@ -562,6 +564,10 @@ __global__ void __launch_bounds__(kThreads) decode_dense_merge_kernel(DecodeArgs
 // Khat^(r-1), Khat^(r), Vhat^(r-1), Vhat^(r) and fold
 // e_new Vhat^(r) - e_old Vhat^(r-1) into an online sum with a running
 // reference max per column group.
+// The selection is fixed after loop 1, so loop r keeps the selected columns'
+// Khat^(r), Vhat^(r) (fp16) for loop r+1: loop 2 rebuilds Khat^(1) from the
+// INT8 base, and loop r >= 3 starts from the kept Khat^(r-1) and adds only
+// its own residual stream (two streams instead of r).
 // ---------------------------------------------------------------------------
 // acc[e] += code(e) * s for E8 consecutive BITS-bit two's-complement codes
 // held in little-endian words w.
@@ -593,29 +599,65 @@ __device__ __forceinline__ void cp_async4(void* smem, const void* gmem) {
 // Shared-memory layout of one gather stage of kSparseStageCols columns:
 // K and V codes of every stream (base, then loop 2..LOOP residuals), then the
 // K and V scales of every stream.  Offsets depend on the loops' code widths.
+// Streams of a loop: LOOP 2 the INT8 base and the loop-2 residual; LOOP >= 3
+// the kept fp16 Khat^(LOOP-1) / Vhat^(LOOP-1) (stream 0, no scale) and the
+// loop's residual (stream 1).
 template <int DH, int LOOP>
 struct SparseStage {
+  static constexpr bool PART = LOOP >= 3;
+  static constexpr int NS = PART ? 2 : LOOP;
   static constexpr int G = DH / 32;
-  int rb[LOOP];               // code bytes of one column in stream l (0 = base)
-  int off_k[LOOP], off_v[LOOP];
+  int rb[NS];               // bytes of one column in stream l
+  int off_k[NS], off_v[NS];
   int off_ks, off_vs, bytes;
   __host__ __device__ SparseStage(const int* bits) {
     int off = 0;
 #pragma unroll
-    for (int l = 0; l < LOOP; ++l) {
-      rb[l] = l == 0 ? DH : DH * bits[l] / 8;
+    for (int l = 0; l < NS; ++l) {
+      rb[l] = l == 0 ? (PART ? 2 * DH : DH) : DH * bits[PART ? LOOP - 1 : l] / 8;
       off_k[l] = off;
       off += kSparseStageCols * rb[l];
       off_v[l] = off;
       off += kSparseStageCols * rb[l];
     }
     off_ks = off;
-    off += LOOP * kSparseStageCols * G * 2;
+    off += NS * kSparseStageCols * G * 2;
     off_vs = off;
-    off += LOOP * kSparseStageCols * G * 2;
+    off += NS * kSparseStageCols * G * 2;
     bytes = off;
   }
 };
+
+// E8 fp16 values (this lane's slice) of a kept column row in a stage, as float.
+template <int E8>
+__device__ __forceinline__ void stage_part(const uint8_t* row, int e0, float (&x)[E8]) {
+#pragma unroll
+  for (int v = 0; v < E8 / 8; ++v) {
+    const uint4 w = *reinterpret_cast<const uint4*>(row + e0 * 2 + v * 16);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
+      x[8 * v + 2 * q] = f.x;
+      x[8 * v + 2 * q + 1] = f.y;
+    }
+  }
+}
+
+// Store E8 values as fp16 (this lane's slice of a kept column row).
+template <int E8>
+__device__ __forceinline__ void store_part(uint16_t* dst, const float (&x)[E8]) {
+#pragma unroll
+  for (int v = 0; v < E8 / 8; ++v) {
+    uint32_t ww[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const __half2 hh = __floats2half2_rn(x[8 * v + 2 * q], x[8 * v + 2 * q + 1]);
+      ww[q] = *reinterpret_cast<const uint32_t*>(&hh);
+    }
+    *reinterpret_cast<uint4*>(dst + v * 8) = make_uint4(ww[0], ww[1], ww[2], ww[3]);
+  }
+}
 
 // E8 codes (this lane's slice, element e0 on) of one column of stream l in
 // a stage, added times s to acc (l = 0: the INT8 base, assigned).
@@ -659,7 +701,10 @@ __device__ __forceinline__ void stage_codes(const uint8_t* row, int bits, int e0
 template <int DH, int LOOP>
 __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArgs a) {
   constexpr int E8 = DH / 8, G = DH / 32;
-  const SparseStage<DH, LOOP> L(a.bits);
+  using LS = SparseStage<DH, LOOP>;
+  constexpr bool PART = LS::PART;
+  constexpr int NS = LS::NS;
+  const LS L(a.bits);
   extern __shared__ __align__(16) uint8_t sm[];
   int* srow = reinterpret_cast<int*>(sm + (size_t)kSparseStages * L.bytes);  // [LOOP][kSparseCols]
   uint8_t* stok = reinterpret_cast<uint8_t*>(srow + LOOP * kSparseCols);   // [kSparseCols]
@@ -684,9 +729,14 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
     const bool tok = j == a.S;
     const size_t t = (size_t)b * a.S + j;
     stok[i] = tok;
-    srow[i] = tok ? b : (int)t;
+    if (PART) {  // the kept row (selection index) and the loop's residual row
+      srow[i] = c_begin + i;
+      srow[kSparseCols + i] = tok ? b : a.cslot[LOOP - 1][t];
+    } else {
+      srow[i] = tok ? b : (int)t;
 #pragma unroll
-    for (int l = 2; l <= LOOP; ++l) srow[(l - 1) * kSparseCols + i] = tok ? b : a.cslot[l - 1][t];
+      for (int l = 2; l <= LOOP; ++l) srow[(l - 1) * kSparseCols + i] = tok ? b : a.cslot[l - 1][t];
+    }
   }
   __syncthreads();
 
@@ -704,21 +754,24 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
         const KVStreams& S = kv == 0 ? (tok ? a.tk : a.ck) : (tok ? a.tv : a.cv);
         const int* off = kv == 0 ? L.off_k : L.off_v;
 #pragma unroll
-        for (int l = 0; l < LOOP; ++l) {
+        for (int l = 0; l < NS; ++l) {
           const int row = srow[l * kSparseCols + c];
           const int nch = L.rb[l] / 16;
-          if (row >= 0 && cu < nch) {
-            const uint8_t* src = (l == 0 ? reinterpret_cast<const uint8_t*>(S.base_codes)
-                                         : S.res_codes[l]) +
-                                 ((size_t)row * a.H + h) * L.rb[l] + cu * 16;
-            cp_async16(buf + off[l] + cl * L.rb[l] + cu * 16, src, 16);
-          }
+          if (row < 0) continue;
+          const uint8_t* src;
+          if (PART && l == 0)  // the kept Khat / Vhat row of this selected column
+            src = reinterpret_cast<const uint8_t*>(a.kv_part) + (((size_t)bh * a.k + row) * 2 + kv) * DH * 2;
+          else
+            src = (l == 0 ? reinterpret_cast<const uint8_t*>(S.base_codes) : S.res_codes[PART ? LOOP - 1 : l]) +
+                  ((size_t)row * a.H + h) * L.rb[l];
+          for (int ch = cu; ch < nch; ch += 8) cp_async16(buf + off[l] + cl * L.rb[l] + ch * 16, src + ch * 16, 16);
         }
       }
-      // scales: 2*LOOP copies of G fp16 per column, two per thread
+      // scales: 2*NS copies of G fp16 per column (the kept rows have none)
 #pragma unroll
-      for (int i = cu; i < 2 * LOOP; i += 8) {
-        const int kv = i / LOOP, l = i - kv * LOOP;
+      for (int i = cu; i < 2 * NS; i += 8) {
+        const int kv = i / NS, l = i - kv * NS;
+        if (PART && l == 0) continue;
         const KVStreams& S = kv == 0 ? (tok ? a.tk : a.ck) : (tok ? a.tv : a.cv);
         const int row = srow[l * kSparseCols + c];
         uint8_t* dst = buf + (kv == 0 ? L.off_ks : L.off_vs) + ((size_t)l * kSparseStageCols + cl) * G * 2;
@@ -726,7 +779,8 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
           if constexpr (G == 4) *reinterpret_cast<uint2*>(dst) = make_uint2(0u, 0u);
           else *reinterpret_cast<uint32_t*>(dst) = 0u;
         } else {
-          const uint16_t* src = (l == 0 ? S.base_scales : S.res_scales[l]) + ((size_t)row * a.H + h) * G;
+          const uint16_t* src =
+              (l == 0 ? S.base_scales : S.res_scales[PART ? LOOP - 1 : l]) + ((size_t)row * a.H + h) * G;
           if constexpr (G == 4) cp_async8(dst, src);
           else cp_async4(dst, src);
         }
@@ -768,17 +822,23 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
     const bool valid = jl < n;
     // K: Khat^(LOOP-1) and Khat^(LOOP) of this lane's slice
     float xo[E8], xn[E8];
+    uint16_t* part_row = a.kv_part + ((size_t)bh * a.k + c_begin + jl) * 2 * DH + e0;
     {
       const uint16_t* ks = reinterpret_cast<const uint16_t*>(buf + L.off_ks);
-      stage_codes<E8>(buf + L.off_k[0] + grp * L.rb[0], 8, e0, half_bits_f(ks[grp * G + g]), xo, true);
+      if (PART) {
+        stage_part<E8>(buf + L.off_k[0] + grp * L.rb[0], e0, xo);
+      } else {
+        stage_codes<E8>(buf + L.off_k[0] + grp * L.rb[0], 8, e0, half_bits_f(ks[grp * G + g]), xo, true);
 #pragma unroll
-      for (int l = 1; l < LOOP - 1; ++l)
-        stage_codes<E8>(buf + L.off_k[l] + grp * L.rb[l], a.bits[l], e0,
-                        half_bits_f(ks[(l * kSparseStageCols + grp) * G + g]), xo, false);
+        for (int l = 1; l < LOOP - 1; ++l)
+          stage_codes<E8>(buf + L.off_k[l] + grp * L.rb[l], a.bits[l], e0,
+                          half_bits_f(ks[(l * kSparseStageCols + grp) * G + g]), xo, false);
+      }
 #pragma unroll
       for (int e = 0; e < E8; ++e) xn[e] = xo[e];
-      stage_codes<E8>(buf + L.off_k[LOOP - 1] + grp * L.rb[LOOP - 1], a.bits[LOOP - 1], e0,
-                      half_bits_f(ks[((LOOP - 1) * kSparseStageCols + grp) * G + g]), xn, false);
+      stage_codes<E8>(buf + L.off_k[NS - 1] + grp * L.rb[NS - 1], a.bits[LOOP - 1], e0,
+                      half_bits_f(ks[((NS - 1) * kSparseStageCols + grp) * G + g]), xn, false);
+      if (a.write_part && valid) store_part<E8>(part_row, xn);
     }
     float dol = 0.f, dnw = 0.f;
 #pragma unroll
@@ -804,15 +864,20 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
       }
       const float en = ex2(sn - mu), eo = ex2(so - mu);
       const uint16_t* vs = reinterpret_cast<const uint16_t*>(buf + L.off_vs);
-      stage_codes<E8>(buf + L.off_v[0] + grp * L.rb[0], 8, e0, half_bits_f(vs[grp * G + g]), xo, true);
+      if (PART) {
+        stage_part<E8>(buf + L.off_v[0] + grp * L.rb[0], e0, xo);
+      } else {
+        stage_codes<E8>(buf + L.off_v[0] + grp * L.rb[0], 8, e0, half_bits_f(vs[grp * G + g]), xo, true);
 #pragma unroll
-      for (int l = 1; l < LOOP - 1; ++l)
-        stage_codes<E8>(buf + L.off_v[l] + grp * L.rb[l], a.bits[l], e0,
-                        half_bits_f(vs[(l * kSparseStageCols + grp) * G + g]), xo, false);
+        for (int l = 1; l < LOOP - 1; ++l)
+          stage_codes<E8>(buf + L.off_v[l] + grp * L.rb[l], a.bits[l], e0,
+                          half_bits_f(vs[(l * kSparseStageCols + grp) * G + g]), xo, false);
+      }
 #pragma unroll
       for (int e = 0; e < E8; ++e) xn[e] = xo[e];
-      stage_codes<E8>(buf + L.off_v[LOOP - 1] + grp * L.rb[LOOP - 1], a.bits[LOOP - 1], e0,
-                      half_bits_f(vs[((LOOP - 1) * kSparseStageCols + grp) * G + g]), xn, false);
+      stage_codes<E8>(buf + L.off_v[NS - 1] + grp * L.rb[NS - 1], a.bits[LOOP - 1], e0,
+                      half_bits_f(vs[((NS - 1) * kSparseStageCols + grp) * G + g]), xn, false);
+      if (a.write_part) store_part<E8>(part_row + DH, xn);
 #pragma unroll
       for (int e = 0; e < E8; ++e) acc[e] = fmaf(en, xn[e], fmaf(-eo, xo[e], acc[e]));
       zn += en;
@@ -878,7 +943,7 @@ __global__ void __launch_bounds__(kSparseThreads) decode_sparse_kernel(DecodeArg
 template <int DH, int LOOP>
 static int launch_sparse_t(const DecodeArgs& a, dim3 grid, cudaStream_t stream) {
   const SparseStage<DH, LOOP> L(a.bits);
-  const size_t smem = (size_t)kSparseStages * L.bytes + (size_t)LOOP * kSparseCols * 4 + kSparseCols;
+  const size_t smem = (size_t)kSparseStages * L.bytes + (size_t)LOOP * kSparseCols * 4 + kSparseCols;  // rows [LOOP][cols] (>= NS), tokens
   static size_t attr = 0;
   if (smem > attr) {
     FL_TRY(cudaFuncSetAttribute(decode_sparse_kernel<DH, LOOP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -951,6 +1016,7 @@ DecodeLayout decode_layout(const flashloop_params* p) {
   L.part_Z = off; off = align256(off + np * sizeof(float));
   const size_t nn = std::max(B * (size_t)L.nsplit * H * dh, B * H * (size_t)L.nblk * dh);
   L.part_N = off; off = align256(off + nn * sizeof(float));
+  L.kv_part = off; off = align256(off + B * H * (size_t)k * 2 * dh * sizeof(uint16_t));
   L.total = off;
   return L;
 }
@@ -989,6 +1055,8 @@ static DecodeArgs make_args(const flashloop_params* p, int loop, const flashloop
   a.nsplit = L.nsplit;
   a.range = L.range;
   a.err = ds->err_word;
+  a.kv_part = ws_ptr<uint16_t>(ds->workspace, L.kv_part);
+  a.write_part = loop >= 2 && loop < p->n_loops;
   return a;
 }
 

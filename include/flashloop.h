@@ -380,7 +380,8 @@ typedef struct flashloop_decode_state {
   uint16_t* O;               /* bf16 [B, d_model] */
   uint16_t* Y;               /* bf16 [B, d_model] */
   int32_t* err_word;         /* device error word, 0 = no error */
-  void* workspace;           /* scratch (need not be cleared) */
+  void* workspace;           /* scratch (need not be cleared); carries the selected columns' rebuilt
+                                K/V from one loop to the next (see flashloop_decode_attn) */
   size_t workspace_bytes;    /* >= flashloop_decode_workspace_bytes(params) */
 } flashloop_decode_state;
 
@@ -404,8 +405,12 @@ size_t flashloop_decode_workspace_bytes(const flashloop_params* p);
  * loop r >= 2: for the selected columns j,
  *   s_old = q^(r-1).Khat_j^(r-1)/sqrt(dh), s_new = q^(r).Khat_j^(r)/sqrt(dh),
  *   m' = max(m, max s_new), Z' = e^(m-m') Z - sum e^(s_old-m') + sum e^(s_new-m'),
- *   N' likewise with Vhat^(r-1), Vhat^(r); O = N'/Z' (bf16).  Khat/Vhat are
- *   rebuilt from the packed streams in the loads (float32 sums in loop order).
+ *   N' likewise with Vhat^(r-1), Vhat^(r); O = N'/Z' (bf16).  The selection
+ *   is fixed after loop 1, so the rebuilt columns carry over: loop 2 rebuilds
+ *   Khat^(1), Vhat^(1) from the INT8 base (float32) and adds the loop-2
+ *   residual; loop r >= 3 starts from the Khat^(r-1), Vhat^(r-1) that loop r-1
+ *   left in ds->workspace (fp16) and adds the loop-r residual (float32).  The
+ *   loops of a step therefore run in order 1..R on one workspace.
  * Argument errors are returned before any launch; a column index outside
  * [0, S] sets FLASHLOOP_DEVERR_INDEX. */
 int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
