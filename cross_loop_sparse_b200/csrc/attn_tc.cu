@@ -1215,10 +1215,13 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 // same type as the keys, as kind::f16 requires), the frame m_i + log2(Z_i)
 // in log2 units (so a contribution is one exp2: 2^(s - m) / Z = 2^(s - frame))
 // and the row token.
-// Roles: warps 0-7 reduce (two per TMEM lane quarter, each 32 of a tile's 64
-// rows) and load the item's keys into TMEM (A operand); warp 8 allocates TMEM
-// and streams the row tiles (TMA for q, bulk copies for frames and tokens);
-// warp 9 issues the MMAs.  All waits are bounded.
+// Roles: warps 0-7 reduce and load the item's keys into TMEM (A operand):
+// group 0 (warps 0-3) takes the tiles with an even block-wide tile counter,
+// group 1 (warps 4-7) the odd ones, one thread per column over all 64 rows of
+// the tile, so that one group's exponentials overlap the other group's waits
+// and loads; warp 8 allocates TMEM and streams the row tiles (TMA for q, bulk
+// copies for frames and tokens); warp 9 issues the MMAs.  All waits are
+// bounded.
 // ---------------------------------------------------------------------------
 constexpr int kCmtCols = 128, kCmtRows = 64, kCmtStages = 4, kCmtThreads = 320;
 constexpr int kCmtRowThreads = 256;
@@ -1291,11 +1294,11 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
   if (threadIdx.x == 0) {
     for (int s = 0; s < kCmtStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1 + kCmtRowThreads);
+      mbar_init(&empty[s], 1 + kCmtRowThreads / 2);  // MMA commit + the tile's row group
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&s_full[b], 1);
-      mbar_init(&s_empty[b], kCmtRowThreads);
+      mbar_init(&s_empty[b], kCmtRowThreads / 2);
     }
     mbar_init(a_ready, kCmtRowThreads);
     *abort_flag = 0;
@@ -1399,8 +1402,8 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
     }
   } else {
     // ------------------------------------------------------------ reducers
-    // Thread (quarter, half): TMEM lane = column quarter*32 + lane of the
-    // item; half 0 takes rows 0..31 of each tile, half 1 rows 32..63.  A
+    // Thread (quarter, group): TMEM lane = column quarter*32 + lane of the
+    // item; group g handles the tiles with (u & 1) == g, all 64 rows.  A
     // named barrier cannot time out, so after a failed wait a warp goes on
     // through the same barriers without touching TMEM ("dead").
     const int quarter = warp & 3, half = warp >> 2;
@@ -1427,7 +1430,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
       const int nt = item_rows(item, a_begin);
       const int c = ct * kCmtCols + col;
       const int ctok = c < g.kc ? (g.cols ? __ldg(g.cols + (size_t)h * g.kc + c) : c) : 0x7fffffff;
-      // this column's keys into TMEM (the MMA's A operand): half h loads
+      // this column's keys into TMEM (the MMA's A operand): group h loads
       // elements [h*DH/2, (h+1)*DH/2)
       if (!dead) {
 #pragma unroll 1
@@ -1448,50 +1451,53 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
       }
       float acc = 0.f;
       for (int t = 0; t < nt; ++t, ++u) {
-        wait_or_die(&full[stage], phase);
-        wait_or_die(&s_full[u & 1], (u >> 1) & 1);
-        if (!dead) {
-          uint32_t r[32];
-          __syncwarp();
-          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + half * 32, r);
-          tmem_wait_ld();
-          // p = 2^(s - m_i) / Z_i * g_i = 2^(s - frame_i); rows past the last
-          // have frame +inf (p = 0).  Row tokens ascend, so only a tile whose
-          // first row lies before this column's token needs the causal mask.
-          const uint8_t* side = smem + stage * C::kStageBytes + C::kQBytes;
-          const float4* sm4 = reinterpret_cast<const float4*>(side) + half * 8;
-          const int* stok = reinterpret_cast<const int*>(side + 256) + half * 32;
-          float pa[4] = {0.f, 0.f, 0.f, 0.f};
-          if (stok[0] >= ctok) {
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 f = sm4[e4];
-              pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
-              pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
-              pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
-              pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
-            }
-          } else {
-#pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-              const float4 f = sm4[e4];
-              const float fr[4] = {f.x, f.y, f.z, f.w};
-#pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                const float v = ex2(__uint_as_float(r[4 * e4 + k]) - fr[k]);
-                pa[k] += stok[4 * e4 + k] >= ctok ? v : 0.f;
-              }
-            }
-          }
-          acc += (pa[0] + pa[1]) + (pa[2] + pa[3]);
-          tc_fence_before();
-          mbar_arrive(&s_empty[u & 1]);
-          mbar_arrive(&empty[stage]);
-        }
+        const int st_now = stage;
+        const uint32_t ph_now = phase;
         if (++stage == kCmtStages) {
           stage = 0;
           phase ^= 1;
         }
+        if ((int)(u & 1) != half) continue;  // the other group's tile
+        wait_or_die(&full[st_now], ph_now);
+        wait_or_die(&s_full[u & 1], (u >> 1) & 1);
+        if (dead) continue;
+        uint32_t r[64];
+        __syncwarp();
+        tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows, *reinterpret_cast<uint32_t(*)[32]>(r));
+        tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+        tmem_wait_ld();
+        tc_fence_before();
+        mbar_arrive(&s_empty[u & 1]);
+        // p = 2^(s - m_i) / Z_i * g_i = 2^(s - frame_i); rows past the last
+        // have frame +inf (p = 0).  Row tokens ascend, so only a tile whose
+        // first row lies before this column's token needs the causal mask.
+        const uint8_t* side = smem + st_now * C::kStageBytes + C::kQBytes;
+        const float4* sm4 = reinterpret_cast<const float4*>(side);
+        const int* stok = reinterpret_cast<const int*>(side + 256);
+        float pa[4] = {0.f, 0.f, 0.f, 0.f};
+        if (stok[0] >= ctok) {
+#pragma unroll
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const float4 f = sm4[e4];
+            pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
+            pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
+            pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
+            pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
+          }
+        } else {
+#pragma unroll
+          for (int e4 = 0; e4 < 16; ++e4) {
+            const float4 f = sm4[e4];
+            const float fr[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const float v = ex2(__uint_as_float(r[4 * e4 + k]) - fr[k]);
+              pa[k] += stok[4 * e4 + k] >= ctok ? v : 0.f;
+            }
+          }
+        }
+        acc += (pa[0] + pa[1]) + (pa[2] + pa[3]);
+        mbar_arrive(&empty[st_now]);
       }
       // the two halves' sums of each column
       xsum[half * 128 + col] = acc;
