@@ -1210,31 +1210,31 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 // rows' final state.  Transposed score tiles S^T = Khat_tile . q_tile^T put
 // one column in each TMEM lane, so a column's mass is a sum inside one
 // thread (no cross-lane reduction).  A work item = 128 selected columns of
-// one head; it walks 64-row tiles from the first row whose token reaches the
-// item's smallest column token.  Rows come prepared per head: fp16 q (the
+// one head; it walks 128-row tiles (M128 N128 score MMAs) from the first row
+// whose token reaches the item's smallest column token.  Rows come prepared per head: fp16 q (the
 // same type as the keys, as kind::f16 requires), the frame m_i + log2(Z_i)
 // in log2 units (so a contribution is one exp2: 2^(s - m) / Z = 2^(s - frame))
 // and the row token.
 // Roles: warps 0-7 reduce and load the item's keys into TMEM (A operand):
 // group 0 (warps 0-3) takes the tiles with an even block-wide tile counter,
-// group 1 (warps 4-7) the odd ones, one thread per column over all 64 rows of
+// group 1 (warps 4-7) the odd ones, one thread per column over all 128 rows of
 // the tile, so that one group's exponentials overlap the other group's waits
 // and loads; warp 8 allocates TMEM and streams the row tiles (TMA for q, bulk
 // copies for frames and tokens); warp 9 issues the MMAs.  All waits are
 // bounded.
 // ---------------------------------------------------------------------------
-constexpr int kCmtCols = 128, kCmtRows = 64, kCmtStages = 4, kCmtThreads = 320;
+constexpr int kCmtCols = 128, kCmtRows = 128, kCmtStages = 4, kCmtThreads = 320;
 constexpr int kCmtRowThreads = 256;
 
 template <int DH>
 struct CmtCfg {
-  static constexpr int kQBytes = kCmtRows * DH * 2;  // q tile: 64 rows x DH (DH/64 swizzle chunks)
-  static constexpr int kSideBytes = 1024;            // frames and tokens of the tile (2 x 256 B); keeps
+  static constexpr int kQBytes = kCmtRows * DH * 2;  // q tile: 128 rows x DH (DH/64 swizzle chunks)
+  static constexpr int kSideBytes = 1024;            // frames and tokens of the tile (2 x 512 B); keeps
                                                      // every stage's q tile on a 1024-byte swizzle atom
   static constexpr int kStageBytes = kQBytes + kSideBytes;
   static constexpr int kSmem = 1024 + kCmtStages * kStageBytes + 256 + 2 * 128 * 4;
   static constexpr uint32_t kColA = 0;       // keys, fp16 pairs: DH/2 columns
-  static constexpr uint32_t kColS = 64;      // two S^T buffers of 64 columns
+  static constexpr uint32_t kColS = 64;      // two S^T buffers of 128 columns
   static constexpr uint32_t kIdesc = f16_idesc(128, kCmtRows, 0);
 };
 
@@ -1305,7 +1305,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
     fence_mbar_init();
   }
   if (warp == 8) {
-    tmem_alloc(tmem_slot, 256);
+    tmem_alloc(tmem_slot, 512);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -1349,7 +1349,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
             tma_load_3d(st + c * (kCmtRows * 128), &tm_q, c * 64, a0, h, &full[stage]);
           uint8_t* side = st + C::kQBytes;
           bulk_g2s(side, g.m2 + (size_t)h * g.n_cap + a0, kCmtRows * 4, &full[stage]);
-          bulk_g2s(side + 256, g.rtok + a0, kCmtRows * 4, &full[stage]);
+          bulk_g2s(side + 512, g.rtok + a0, kCmtRows * 4, &full[stage]);
           issued[stage] = phase;
           if (++stage == kCmtStages) {
             stage = 0;
@@ -1403,7 +1403,8 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
   } else {
     // ------------------------------------------------------------ reducers
     // Thread (quarter, group): TMEM lane = column quarter*32 + lane of the
-    // item; group g handles the tiles with (u & 1) == g, all 64 rows.  A
+    // item; group g handles the tiles with (u & 1) == g, all 128 rows (in two
+    // halves of 64 loaded from TMEM one after the other).  A
     // named barrier cannot time out, so after a failed wait a warp goes on
     // through the same barriers without touching TMEM ("dead").
     const int quarter = warp & 3, half = warp >> 2;
@@ -1461,38 +1462,43 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
         wait_or_die(&full[st_now], ph_now);
         wait_or_die(&s_full[u & 1], (u >> 1) & 1);
         if (dead) continue;
-        uint32_t r[64];
-        __syncwarp();
-        tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows, *reinterpret_cast<uint32_t(*)[32]>(r));
-        tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-        tmem_wait_ld();
-        tc_fence_before();
-        mbar_arrive(&s_empty[u & 1]);
-        // p = 2^(s - m_i) / Z_i * g_i = 2^(s - frame_i); rows past the last
-        // have frame +inf (p = 0).  Row tokens ascend, so only a tile whose
-        // first row lies before this column's token needs the causal mask.
         const uint8_t* side = smem + st_now * C::kStageBytes + C::kQBytes;
-        const float4* sm4 = reinterpret_cast<const float4*>(side);
-        const int* stok = reinterpret_cast<const int*>(side + 256);
+        const int* stok = reinterpret_cast<const int*>(side + 512);
+        const bool diag = stok[0] < ctok;
         float pa[4] = {0.f, 0.f, 0.f, 0.f};
-        if (stok[0] >= ctok) {
-#pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
-            const float4 f = sm4[e4];
-            pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
-            pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
-            pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
-            pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
+#pragma unroll 1
+        for (int hh = 0; hh < 2; ++hh) {
+          uint32_t r[64];
+          __syncwarp();
+          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + hh * 64 + 32,
+                    *reinterpret_cast<uint32_t(*)[32]>(r + 32));
+          tmem_wait_ld();
+          if (hh == 1) {
+            tc_fence_before();
+            mbar_arrive(&s_empty[u & 1]);
           }
-        } else {
+          const float4* sm4 = reinterpret_cast<const float4*>(side) + hh * 16;
+          const int* st2 = stok + hh * 64;
+          if (!diag) {
 #pragma unroll
-          for (int e4 = 0; e4 < 16; ++e4) {
-            const float4 f = sm4[e4];
-            const float fr[4] = {f.x, f.y, f.z, f.w};
+            for (int e4 = 0; e4 < 16; ++e4) {
+              const float4 f = sm4[e4];
+              pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
+              pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
+              pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
+              pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
+            }
+          } else {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              const float v = ex2(__uint_as_float(r[4 * e4 + k]) - fr[k]);
-              pa[k] += stok[4 * e4 + k] >= ctok ? v : 0.f;
+            for (int e4 = 0; e4 < 16; ++e4) {
+              const float4 f = sm4[e4];
+              const float fr[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                const float v = ex2(__uint_as_float(r[4 * e4 + k]) - fr[k]);
+                pa[k] += st2[4 * e4 + k] >= ctok ? v : 0.f;
+              }
             }
           }
         }
@@ -1511,7 +1517,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
   __syncthreads();
   if (warp == 8) {
     tc_fence_after();
-    tmem_dealloc(tmem, 256);
+    tmem_dealloc(tmem, 512);
   }
 }
 

@@ -86,9 +86,9 @@ inline Workspace workspace_layout(const flashloop_params* p) {
   w.ticket = off; off = align256(off + 16);
   w.flags = off; off = align256(off + S);
   w.keys = off; off = align256(off + S * sizeof(float));
-  const size_t S64 = (S + 63) / 64 * 64;  // the column mass pads its rows to whole 64-row tiles
-  const size_t cmq = S * H * dh * sizeof(float) > S64 * H * dh * 2 ? S * H * dh * sizeof(float) : S64 * H * dh * 2;
-  const size_t cmr = S * H * dh * sizeof(float) > S64 * (8 * H + 4) ? S * H * dh * sizeof(float) : S64 * (8 * H + 4);
+  const size_t S128 = (S + 127) / 128 * 128;  // the column mass pads its rows to whole 128-row tiles
+  const size_t cmq = S * H * dh * sizeof(float) > S128 * H * dh * 2 ? S * H * dh * sizeof(float) : S128 * H * dh * 2;
+  const size_t cmr = S * H * dh * sizeof(float) > S128 * (8 * H + 4) ? S * H * dh * sizeof(float) : S128 * (8 * H + 4);
   w.cm_q = off; off = align256(off + cmq);
   w.cm_rows = off; off = align256(off + cmr);
   size_t sel = 4 * H * (size_t)pad8(max_topk(p)) * dh;
