@@ -231,10 +231,37 @@ paper_tail_kernel(const float* __restrict__ k, const float* __restrict__ v, cons
   }
 }
 
+// E consecutive elements c0.. of stream row `row` (loop l) dequantised: the
+// same arithmetic as paper_deq, with the codes, scales and minima of the
+// lane's slice loaded together.
+template <int DH, bool KEY, int E>
+__device__ __forceinline__ void paper_deq_vec(const PaperStreams& ps, int l, int row, int h, int H, int c0,
+                                              float (&out)[E]) {
+  const uint8_t* cp = ps.codes[l - 1] + ((size_t)row * H + h) * (DH / 2) + (c0 >> 1);
+  uint32_t cw;
+  if (E == 4) cw = *reinterpret_cast<const uint16_t*>(cp);
+  else cw = *cp;
+  if (KEY) {
+    const size_t gi = ((size_t)(row / kPaperGroup) * H + h) * DH + c0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float code = static_cast<float>((cw >> (4 * e)) & 15u);
+      out[e] = fmaf(code, half_bits_f(ps.scale[l - 1][gi + e]), half_bits_f(ps.minv[l - 1][gi + e]));
+    }
+  } else {
+    const size_t gi = ((size_t)row * H + h) * (DH / kPaperGroup) + c0 / kPaperGroup;
+    const float sc = half_bits_f(ps.scale[l - 1][gi]), mn = half_bits_f(ps.minv[l - 1][gi]);
+#pragma unroll
+    for (int e = 0; e < E; ++e) out[e] = fmaf(static_cast<float>((cw >> (4 * e)) & 15u), sc, mn);
+  }
+}
+
 // (a5) in the pages' setting: the selected columns' reconstructions of loops
 // r-1 and r (loop 1: of every token), as fp16 K [H, kcp, dh] scaled by kscale
-// and transposed V [H, dh, kcp].  One block = 64 columns of one head; V rows
-// are staged in shared memory and written transposed.
+// and transposed V [H, dh, kcp].  One block = 64 columns of one head; a warp
+// takes one column at a time, each lane DH/32 consecutive elements; the sum
+// over loops runs once, keeping loop r-1's value on the way; V rows are
+// staged in shared memory and written transposed.
 template <int DH>
 __global__ void __launch_bounds__(256)
 paper_selcol_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, int H, int body, int loop,
@@ -245,6 +272,7 @@ paper_selcol_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, in
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int h = blockIdx.y, j0 = blockIdx.x * 64;
   const bool has_old = loop > 1;
+  const int c0 = lane * E;
   for (int cl = warp; cl < 64; cl += 8) {
     const int col = j0 + cl;
     int j = -1;
@@ -257,15 +285,53 @@ paper_selcol_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, in
     }
     float kn[E], ko[E], vn[E], vo[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int c = lane * E + e;
-      kn[e] = ko[e] = vn[e] = vo[e] = 0.f;
-      if (j >= 0) {
-        kn[e] = paper_recon<DH, true>(kps, lt, body, j, h, H, c, loop);
-        vn[e] = paper_recon<DH, false>(vps, lt, body, j, h, H, c, loop);
+    for (int e = 0; e < E; ++e) kn[e] = ko[e] = vn[e] = vo[e] = 0.f;
+    if (j >= body) {
+      // a tail token: the bf16 value of the latest loop <= r (and <= r-1) that stored it
+      int ln = loop;
+      while (ln > 1 && lt.slot[ln - 1][j] < 0) --ln;
+      int lo = has_old ? loop - 1 : 1;
+      while (lo > 1 && lt.slot[lo - 1][j] < 0) --lo;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        const size_t ti = ((size_t)(j - body) * H + h) * DH + c0 + e;
+        kn[e] = bf16_bits_to_float(kps.tail[ln - 1][ti]);
+        vn[e] = bf16_bits_to_float(vps.tail[ln - 1][ti]);
         if (has_old) {
-          ko[e] = paper_recon<DH, true>(kps, lt, body, j, h, H, c, loop - 1);
-          vo[e] = paper_recon<DH, false>(vps, lt, body, j, h, H, c, loop - 1);
+          ko[e] = bf16_bits_to_float(kps.tail[lo - 1][ti]);
+          vo[e] = bf16_bits_to_float(vps.tail[lo - 1][ti]);
+        }
+      }
+    } else if (j >= 0) {
+      // body: the loop-1 codes, then in loop order the residual of every loop
+      // where the token was active (float32 additions, as paper_recon)
+      paper_deq_vec<DH, true, E>(kps, 1, j, h, H, c0, kn);
+      paper_deq_vec<DH, false, E>(vps, 1, j, h, H, c0, vn);
+      if (loop == 2) {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          ko[e] = kn[e];
+          vo[e] = vn[e];
+        }
+      }
+      for (int l = 2; l <= loop; ++l) {
+        const int sl = lt.slot[l - 1][j];
+        if (sl >= 0) {
+          float dk[E], dv[E];
+          paper_deq_vec<DH, true, E>(kps, l, sl, h, H, c0, dk);
+          paper_deq_vec<DH, false, E>(vps, l, sl, h, H, c0, dv);
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            kn[e] = kn[e] + dk[e];
+            vn[e] = vn[e] + dv[e];
+          }
+        }
+        if (l == loop - 1) {
+#pragma unroll
+          for (int e = 0; e < E; ++e) {
+            ko[e] = kn[e];
+            vo[e] = vn[e];
+          }
         }
       }
     }
@@ -276,7 +342,7 @@ paper_selcol_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, in
            half_range_ok(vo[e]);
     if (!ok) set_error(err, FLASHLOOP_DEVERR_RANGE);
     if (col < kcp) {
-      const size_t off = ((size_t)h * kcp + col) * DH + lane * E;
+      const size_t off = ((size_t)h * kcp + col) * DH + c0;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
         k_new[off + e] = __float2half_rn(kn[e] * kscale);
@@ -285,8 +351,8 @@ paper_selcol_kernel(const int32_t* __restrict__ cols, int kc, int kcp, int S, in
     }
 #pragma unroll
     for (int e = 0; e < E; ++e) {
-      sv[1][cl][lane * E + e] = __float2half_rn(vn[e]);
-      sv[0][cl][lane * E + e] = __float2half_rn(vo[e]);
+      sv[1][cl][c0 + e] = __float2half_rn(vn[e]);
+      sv[0][cl][c0 + e] = __float2half_rn(vo[e]);
     }
   }
   __syncthreads();
