@@ -8,10 +8,11 @@
 // r-1 (row = the token's position in the loop's active list).
 //
 // Kernels:
-//   paper_key_quant_kernel   one block per (64-row group, head), one thread per
-//                            channel: the residuals of its 64 rows in registers,
-//                            their minimum and maximum, scale, minimum, codes
-//                            (two channels share a byte: lanes pair up);
+//   paper_key_quant_kernel   one block per (64-row group, head), four threads per
+//                            channel, 16 rows each: the residuals in registers,
+//                            the group's minimum and maximum through shared
+//                            memory, scale, minimum, codes (two channels share a
+//                            byte: lanes pair up);
 //   paper_value_quant_kernel one warp per (row, head, 64-channel group), two
 //                            channels per lane, warp reductions;
 //   paper_tail_kernel        bf16 copies of the tail tokens active at the loop;
@@ -29,6 +30,7 @@ namespace fl {
 
 constexpr int kPaperGroup = FLASHLOOP_PAPER_GROUP;
 constexpr float kPaperLevels = 15.f;
+constexpr int kPaperKeyQ = 4;  // threads per channel in the key quantiser (16 of a group's 64 rows each)
 
 struct PaperStreams {
   const uint8_t* codes[FLASHLOOP_MAX_LOOPS];
@@ -116,12 +118,15 @@ __device__ __forceinline__ uint32_t paper_code(float x, float s, float lo) {
 }
 
 template <int DH>
-__global__ void __launch_bounds__(DH)
+__global__ void __launch_bounds__(kPaperKeyQ * DH)
 paper_key_quant_kernel(const float* __restrict__ x, const int32_t* __restrict__ active,
                        const int32_t* __restrict__ n_active, int n_cap, int S, int H, int body, int loop,
                        PaperStreams ps, LoopTables lt, PaperOut out, int32_t* err) {
+  constexpr int kR = kPaperGroup / kPaperKeyQ;  // rows per thread
   __shared__ int s_rows;
-  const int c = threadIdx.x, h = blockIdx.y, g = blockIdx.x;
+  __shared__ float s_mn[kPaperKeyQ][DH], s_mx[kPaperKeyQ][DH];
+  const int c = threadIdx.x % DH, q = threadIdx.x / DH;
+  const int h = blockIdx.y, g = blockIdx.x;
   if (threadIdx.x == 0) {
     int n = active ? *n_active : S;
     if (n > n_cap) n = n_cap;
@@ -129,12 +134,12 @@ paper_key_quant_kernel(const float* __restrict__ x, const int32_t* __restrict__ 
   }
   __syncthreads();
   const int rows = s_rows;
-  const int r0 = g * kPaperGroup;
-  if (r0 >= rows) return;
-  float rho[kPaperGroup];
+  const int r0 = g * kPaperGroup + q * kR;
+  if (g * kPaperGroup >= rows) return;  // the whole block: no row of this group
+  float rho[kR];
   float mn = INFINITY, mx = -INFINITY;
 #pragma unroll
-  for (int i = 0; i < kPaperGroup; ++i) {
+  for (int i = 0; i < kR; ++i) {
     const int row = r0 + i;
     rho[i] = 0.f;
     if (row < rows) {
@@ -150,14 +155,25 @@ paper_key_quant_kernel(const float* __restrict__ x, const int32_t* __restrict__ 
       mx = fmaxf(mx, v);
     }
   }
+  // the group's minimum and maximum over its 64 rows (kPaperKeyQ threads per channel)
+  s_mn[q][c] = mn;
+  s_mx[q][c] = mx;
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kPaperKeyQ; ++k) {
+    mn = fminf(mn, s_mn[k][c]);
+    mx = fmaxf(mx, s_mx[k][c]);
+  }
   uint16_t s16, lo16;
   float s, lo;
   paper_group_params(mn, mx, s16, lo16, s, lo);
-  const size_t gi = ((size_t)g * H + h) * DH + c;
-  out.scale[gi] = s16;
-  out.minv[gi] = lo16;
+  if (q == 0) {
+    const size_t gi = ((size_t)g * H + h) * DH + c;
+    out.scale[gi] = s16;
+    out.minv[gi] = lo16;
+  }
 #pragma unroll
-  for (int i = 0; i < kPaperGroup; ++i) {
+  for (int i = 0; i < kR; ++i) {
     const int row = r0 + i;
     const uint32_t code = paper_code(rho[i], s, lo);
     const uint32_t other = __shfl_down_sync(0xffffffffu, code, 1);  // channel c + 1
@@ -395,13 +411,13 @@ int launch_paper_quant(const flashloop_params* p, int loop, const float* k, cons
   int tgrid = (int)((titems + 255) / 256);
   if (tgrid < 1) tgrid = 1;
   if (dh == 128) {
-    paper_key_quant_kernel<128><<<kgrid, 128, 0, stream>>>(k, active, n_active, n_cap, S, H, body, loop, kps, lt, ko,
+    paper_key_quant_kernel<128><<<kgrid, kPaperKeyQ * 128, 0, stream>>>(k, active, n_active, n_cap, S, H, body, loop, kps, lt, ko,
                                                            st->err_word);
     paper_value_quant_kernel<128><<<vgrid, 256, 0, stream>>>(v, active, n_active, n_cap, S, H, body, loop, vps, lt,
                                                              vo, st->err_word);
     paper_tail_kernel<128><<<tgrid, 256, 0, stream>>>(k, v, active, n_active, n_cap, S, H, body, ko.tail, vo.tail);
   } else {
-    paper_key_quant_kernel<64><<<kgrid, 64, 0, stream>>>(k, active, n_active, n_cap, S, H, body, loop, kps, lt, ko,
+    paper_key_quant_kernel<64><<<kgrid, kPaperKeyQ * 64, 0, stream>>>(k, active, n_active, n_cap, S, H, body, loop, kps, lt, ko,
                                                          st->err_word);
     paper_value_quant_kernel<64><<<vgrid, 256, 0, stream>>>(v, active, n_active, n_cap, S, H, body, loop, vps, lt,
                                                             vo, st->err_word);
