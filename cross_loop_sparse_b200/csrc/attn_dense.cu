@@ -12,23 +12,31 @@
 // x DH) and a ring of five K / V slots of 128 columns, a slot holding a K tile
 // (128 x DH) or a V^T tile (DH x 128), filled by TMA.
 // TMEM (512 columns): N_A, N_B (float32, DH columns each), then per tile a
-// 128-column score buffer; P (fp16 pairs, 64 columns) is written over its
-// first half and feeds the P.V MMA from TMEM.
+// 128-column score region of two 64-column halves; the P of a half (fp16
+// pairs, 32 columns) is written over the first columns of its scores and
+// feeds that half's P.V MMA from TMEM.
 //
-// Roles (14 warps):
-//   warps 0-3 / 4-7  rows of tile A / B, one thread per row (its TMEM lane):
-//                    a tile is taken as two halves of 64 columns, each with the
-//                    causal mask, the running maximum (a per-row reference
-//                    raised only when a half's maximum exceeds it by 8 in log2
-//                    units; raising it in the second half also rescales the
-//                    first half's P), exponentials, sums and P; at the end of
-//                    the item the write-back O = N / Z, N, m, Z;
+// Each K / V tile is taken as two halves of 64 columns, each with its own
+// score MMA (M128 N64), its own P and its own P.V (K = 64), so the scores of
+// the next tile's first half are computed while the rows work on the second
+// half of this one: the rows never wait for a whole P.V + score round trip.
+//
+// Roles (15 warps):
+//   warps 0-3 / 4-7  rows of tile A / B, one thread per row (its TMEM lane),
+//                    per half: the causal mask, the running maximum (a per-row
+//                    reference raised only when a half's maximum exceeds it by
+//                    8 in log2 units; raising it rescales the numerator once
+//                    the P.V of the previous half has completed), exponentials,
+//                    sums and P; at the end of the item the write-back
+//                    O = N / Z, N, m, Z;
 //   warps 8-11       the next item's queries: bf16 rows converted to fp16 and
 //                    stored swizzled (fp16 range checked);
 //   warp 12          TMEM allocation and the K / V TMA loads;
-//   warp 13          MMA issue (M128 N128 score MMAs, both operands in shared
-//                    memory; P.V with P from TMEM), alternating the tiles:
-//                    S_A(0) S_B(0) | PV_A(t) S_A(t+1) | PV_B(t) S_B(t+1) | ...
+//   warps 13 / 14    MMA issue for tile A / B (one thread each: a thread that
+//                    issues tcgen05.mma waits while the tensor pipe takes its
+//                    MMAs, so each tile has its own issuer), in the order
+//                    PV(t, 0) S(t+1, 0) PV(t, 1) S(t+1, 1); a K / V slot is
+//                    released when both issuers are done with it.
 // Every wait is bounded; a wait that gives up sets FLASHLOOP_DEVERR_TIMEOUT and
 // the CTA unwinds.
 #include <cuda.h>
@@ -43,10 +51,10 @@ namespace fl {
 
 constexpr int kDnRows = 128;     // rows per tile (TMEM lanes)
 constexpr int kDnCols = 128;     // columns per K / V tile
-constexpr int kDnThreads = 448;  // 14 warps
+constexpr int kDnThreads = 480;  // 15 warps
 constexpr int kDnWarpQ = 8;      // warps 8-11
 constexpr int kDnWarpTma = 12;
-constexpr int kDnWarpMma = 13;
+constexpr int kDnWarpMma = 13;   // warps 13 (tile A) and 14 (tile B)
 constexpr float kDnLog2e = 1.4426950408889634f;
 constexpr float kDnRescale = 8.f;
 
@@ -61,10 +69,11 @@ struct DnCfg {
   static constexpr int kRingOff = 2 * kQBytes;
   static constexpr int kBarOff = kRingOff + kStages * kSlotBytes;
   static constexpr int kSmem = 1024 + kBarOff + 512;
-  static constexpr uint32_t kColS = 256;  // tile X: scores at 256 + 128 X; numerator at X * DH
-  static constexpr uint32_t kIdescS = f16_idesc(128, kDnCols, 0);
+  static constexpr uint32_t kColS = 256;  // tile X: scores at 256 + 128 X (half h at +64 h); numerator at X * DH
+  static constexpr uint32_t kIdescS = f16_idesc(128, 64, 0);
   static constexpr uint32_t kIdescPV = f16_idesc(128, DH, 0);
   static_assert(kSmem <= 232448, "shared memory per block");
+  static_assert((2 * kStages + 21) * 8 + 8 <= 512, "barriers");
 };
 
 struct DnArgs {
@@ -99,15 +108,15 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kBarOff);
   uint64_t* kv_full = bars;                 // [stages] TMA bytes landed
-  uint64_t* kv_empty = bars + C::kStages;   // [stages] MMAs done with the slot
-  uint64_t* s_full = bars + 2 * C::kStages; // [2] scores of a tile in TMEM
-  uint64_t* p_full = s_full + 2;            // [2] P of a tile written (128 row threads)
-  uint64_t* pv_done = p_full + 2;           // [2] a tile's P.V completed
-  uint64_t* acc_full = pv_done + 2;         // [2] the item's last P.V of a tile completed
-  uint64_t* n_free = acc_full + 2;          // [2] the write-back has read the numerator (128 threads)
-  uint64_t* q_full = n_free + 2;            // [2] a tile's queries stored (128 threads)
-  uint64_t* q_empty = q_full + 2;           // [2] the item's S MMAs of a tile completed
-  uint64_t* fin = q_empty + 2;              // [1] every MMA completed
+  uint64_t* kv_empty = bars + C::kStages;   // [stages] both issuers done with the slot (2 arrivals)
+  uint64_t* s_full = bars + 2 * C::kStages; // [X * 2 + h] scores of a half in TMEM
+  uint64_t* p_full = s_full + 4;            // [X * 2 + h] P of a half written (128 row threads)
+  uint64_t* pv_done = p_full + 4;           // [X] a half's P.V completed (two completions per tile)
+  uint64_t* acc_full = pv_done + 2;         // [X] the item's last P.V of a tile completed
+  uint64_t* n_free = acc_full + 2;          // [X] the write-back has read the numerator (128 threads)
+  uint64_t* q_full = n_free + 2;            // [X] a tile's queries stored (128 threads)
+  uint64_t* q_empty = q_full + 2;           // [X] the item's S MMAs of a tile completed
+  uint64_t* fin = q_empty + 2;              // [1] every MMA of both issuers completed (2 commits)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(fin + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   uint8_t* ring = smem + C::kRingOff;
@@ -124,18 +133,20 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&kv_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&kv_empty[s], 2);
+    }
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&p_full[i], kDnRows);
     }
     for (int x = 0; x < 2; ++x) {
-      mbar_init(&s_full[x], 1);
-      mbar_init(&p_full[x], kDnRows);
       mbar_init(&pv_done[x], 1);
       mbar_init(&acc_full[x], 1);
       mbar_init(&n_free[x], kDnRows);
       mbar_init(&q_full[x], kDnRows);
       mbar_init(&q_empty[x], 1);
     }
-    mbar_init(fin, 1);
+    mbar_init(fin, 2);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -191,11 +202,11 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       for (int s = 0; s < C::kStages; ++s)
         if (issued[s] >= 0) (void)mbar_wait(&kv_full[s], (uint32_t)issued[s]);
     }
-  } else if (warp == kDnWarpMma) {
-    // ------------------------------------------------------------ MMA issue
+  } else if (warp == kDnWarpMma || warp == kDnWarpMma + 1) {
+    // ------------------------------------------------------------ MMA issue, one thread per tile
     if (lane == 0) {
-      uint32_t seq = 0, item_no = 0;
-      uint32_t pc[2] = {0u, 0u};
+      const int x = warp - kDnWarpMma;
+      uint32_t seq = 0, item_no = 0, u = 0;
       bool ok = true;
       auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
         if (*abort_flag || !mbar_wait_sleep(bar, parity)) {
@@ -208,71 +219,84 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       };
       auto slot_of = [&](uint32_t s) { return (int)(s % C::kStages); };
       auto par_of = [&](uint32_t s) { return (s / C::kStages) & 1u; };
-      auto issue_s = [&](int x, int slot) {
-        const uint32_t q = smem_u32(smem + x * C::kQBytes);
-        const uint32_t k = smem_u32(ring + slot * C::kSlotBytes);
-        const uint32_t d = tmem + C::kColS + 128u * x;
+      const uint32_t q = smem_u32(smem + x * C::kQBytes);
+      const uint32_t scol = tmem + C::kColS + 128u * x;
+      // S(., hf) = Q K[64 hf, 64 hf + 64)^T into the half's 64 columns
+      auto issue_s = [&](int slot, int hf) {
+        const uint32_t k = smem_u32(ring + slot * C::kSlotBytes) + hf * 64 * 128;
 #pragma unroll
         for (int ks = 0; ks < DH / 16; ++ks)
-          umma_f16(d, sw128_kmajor_desc(q + (ks >> 2) * C::kQChunk + (ks & 3) * 32),
+          umma_f16(scol + 64u * hf, sw128_kmajor_desc(q + (ks >> 2) * C::kQChunk + (ks & 3) * 32),
                    sw128_kmajor_desc(k + (ks >> 2) * C::kKChunk + (ks & 3) * 32), C::kIdescS, ks > 0);
       };
-      auto issue_pv = [&](int x, int slot, bool acc) {
-        const uint32_t v = smem_u32(ring + slot * C::kSlotBytes);
-        const uint32_t pcol = tmem + C::kColS + 128u * x;
+      // N += P(., hf) V[64 hf, 64 hf + 64)
+      auto issue_pv = [&](int slot, int hf, bool acc) {
+        const uint32_t v = smem_u32(ring + slot * C::kSlotBytes) + hf * C::kVChunk;
+        const uint32_t pcol = scol + 64u * hf;
         const uint32_t d = tmem + (uint32_t)(x * DH);
 #pragma unroll
-        for (int ks = 0; ks < kDnCols / 16; ++ks)
-          umma_f16_ts(d, pcol + ks * 8, sw128_kmajor_desc(v + (ks >> 2) * C::kVChunk + (ks & 3) * 32),
-                      C::kIdescPV, (acc || ks > 0) ? 1u : 0u);
+        for (int ks = 0; ks < 4; ++ks)
+          umma_f16_ts(d, pcol + ks * 8, sw128_kmajor_desc(v + ks * 32), C::kIdescPV, (acc || ks > 0) ? 1u : 0u);
+      };
+      // a slot this tile does not read: released once its load has landed
+      auto skip = [&](uint32_t s) -> bool {
+        if (!wait(&kv_full[slot_of(s)], par_of(s))) return false;
+        mbar_arrive(&kv_empty[slot_of(s)]);
+        return true;
       };
       for (int item = blockIdx.x; item < total && ok; item += gridDim.x, ++item_no) {
         const int p = item_p(item);
-        const int ntx[2] = {dn_tiles(g.S, p, 0), dn_tiles(g.S, p, 1)};
-        const int nt = max(ntx[0], ntx[1]);
-        if (!wait(&q_full[0], item_no & 1) || !wait(&q_full[1], item_no & 1)) break;
-        for (int x = 0; x < 2; ++x)
-          if (ntx[x] == 0) umma_commit(&q_empty[x]);
+        const int my = dn_tiles(g.S, p, x);
+        const int nt = max(dn_tiles(g.S, p, 0), dn_tiles(g.S, p, 1));
+        if (!wait(&q_full[x], item_no & 1)) break;
+        if (my == 0) umma_commit(&q_empty[x]);
         const uint32_t base = seq;
         if (nt > 0) {
-          if (!wait(&kv_full[slot_of(base)], par_of(base))) break;
-          for (int x = 0; x < 2; ++x) {
-            if (ntx[x] == 0) continue;
-            issue_s(x, slot_of(base));
-            umma_commit(&s_full[x]);
-            if (ntx[x] == 1) umma_commit(&q_empty[x]);
+          if (my > 0) {
+            if (!wait(&kv_full[slot_of(base)], par_of(base))) break;
+            for (int hf = 0; hf < 2; ++hf) {
+              issue_s(slot_of(base), hf);
+              umma_commit(&s_full[2 * x + hf]);
+            }
+            if (my == 1) umma_commit(&q_empty[x]);
+            umma_commit(&kv_empty[slot_of(base)]);
+          } else if (!skip(base)) {
+            break;
           }
-          umma_commit(&kv_empty[slot_of(base)]);
         }
         for (int t = 0; t < nt && ok; ++t) {
           const uint32_t vs = base + 2 * t + 1, ks_next = base + 2 * t + 2;
+          if (t >= my) {
+            if (!skip(vs)) break;
+            if (t + 1 < nt && !skip(ks_next)) break;
+            continue;
+          }
           if (!wait(&kv_full[slot_of(vs)], par_of(vs))) break;
-          bool k_next = false;
-          for (int x = 0; x < 2 && ok; ++x) {
-            if (t >= ntx[x]) continue;
-            if (t == 0 && item_no > 0 && !wait(&n_free[x], (item_no - 1) & 1)) break;
-            if (!wait(&p_full[x], pc[x] & 1)) break;
-            ++pc[x];
-            issue_pv(x, slot_of(vs), t > 0);
+          for (int hf = 0; hf < 2 && ok; ++hf, ++u) {
+            if (t == 0 && hf == 0 && item_no > 0 && !wait(&n_free[x], (item_no - 1) & 1)) break;
+            if (!wait(&p_full[2 * x + hf], (u >> 1) & 1)) break;
+            issue_pv(slot_of(vs), hf, t > 0 || hf > 0);
             umma_commit(&pv_done[x]);
-            if (t == ntx[x] - 1) umma_commit(&acc_full[x]);
-            if (t + 1 < ntx[x]) {
-              if (!k_next) {
-                if (!wait(&kv_full[slot_of(ks_next)], par_of(ks_next))) break;
-                k_next = true;
-              }
-              issue_s(x, slot_of(ks_next));
-              umma_commit(&s_full[x]);
-              if (t + 1 == ntx[x] - 1) umma_commit(&q_empty[x]);
+            if (t == my - 1 && hf == 1) umma_commit(&acc_full[x]);
+            if (t + 1 < my) {
+              if (hf == 0 && !wait(&kv_full[slot_of(ks_next)], par_of(ks_next))) break;
+              issue_s(slot_of(ks_next), hf);
+              umma_commit(&s_full[2 * x + hf]);
+              if (t + 1 == my - 1 && hf == 1) umma_commit(&q_empty[x]);
             }
           }
           if (!ok) break;
           umma_commit(&kv_empty[slot_of(vs)]);
-          if (t + 1 < nt) umma_commit(&kv_empty[slot_of(ks_next)]);
+          if (t + 1 < nt) {
+            if (t + 1 < my) {
+              umma_commit(&kv_empty[slot_of(ks_next)]);
+            } else if (!skip(ks_next)) {
+              break;
+            }
+          }
         }
         if (!ok) break;
-        for (int x = 0; x < 2 && ok; ++x) {
-          if (ntx[x] != 0) continue;
+        if (my == 0) {
           if (item_no > 0 && !wait(&n_free[x], (item_no - 1) & 1)) break;
           umma_commit(&acc_full[x]);
         }
@@ -348,7 +372,7 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
     const uint32_t lane_base = (uint32_t)(quarter * 32) << 16;
     const uint32_t sbase = tmem + lane_base + C::kColS + 128u * x;
     const uint32_t nbase = tmem + lane_base + (uint32_t)(x * DH);
-    uint32_t u = 0, item_no = 0;
+    uint32_t u = 0, item_no = 0;  // u: halves of this tile so far (two per column tile)
     bool ok = true;
     auto wait = [&](uint64_t* bar, uint32_t parity) -> bool {
       if (*abort_flag || !__all_sync(0xffffffffu, mbar_wait_sleep(bar, parity))) {
@@ -365,18 +389,19 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
       const int tok0 = p * 2 * kDnRows + x * kDnRows + row;
       const int tok = tok0 < g.S ? tok0 : -1;
       float m_ref = -INFINITY, z = 0.f;
-      for (int t = 0; t < nt; ++t, ++u) {
-        if (!wait(&s_full[x], u & 1)) break;
+      for (int t = 0; t < nt && ok; ++t) {
 #pragma unroll 1
-        for (int h2 = 0; h2 < 2; ++h2) {
-          // columns [128t + 64h2, +64): the valid ones (j <= tok) form a prefix
-          const int nvalid = tok < 0 ? 0 : min(max(tok + 1 - (t * kDnCols + 64 * h2), 0), 64);
+        for (int hf = 0; hf < 2; ++hf, ++u) {
+          if (!wait(&s_full[2 * x + hf], (u >> 1) & 1)) break;
+          // columns [128t + 64hf, +64): the valid ones (j <= tok) form a prefix
+          const int nvalid = tok < 0 ? 0 : min(max(tok + 1 - (t * kDnCols + 64 * hf), 0), 64);
+          const uint32_t shalf = sbase + 64u * hf;
           uint32_t s[64];
           {
             uint32_t (&s0)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[0]);
             uint32_t (&s1)[32] = *reinterpret_cast<uint32_t(*)[32]>(&s[32]);
-            tmem_ld32(sbase + 64 * h2, s0);
-            tmem_ld32(sbase + 64 * h2 + 32, s1);
+            tmem_ld32(shalf, s0);
+            tmem_ld32(shalf + 32, s1);
             tmem_wait_ld();
           }
           if (nvalid < 64) {
@@ -384,21 +409,15 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
             for (int e = 0; e < 64; ++e)
               if (e >= nvalid) s[e] = 0xff800000u;  // -inf
           }
-          float t32[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) t32[e] = fmaxf(__uint_as_float(s[e]), __uint_as_float(s[e + 32]));
-#pragma unroll
-          for (int w = 16; w > 0; w >>= 1)
-#pragma unroll
-            for (int e = 0; e < w; ++e) t32[e] = fmaxf(t32[e], t32[e + w]);
-          const float mx = t32[0];
+          const float mx = max64(s);
           const bool need = mx > m_ref + kDnRescale;
           if (__any_sync(0xffffffffu, need)) {
-            // raise the reference: the numerator accumulated so far, Z and this
-            // tile's first half of P scale by 2^(m_ref - mx)
+            // raise the reference: the numerator accumulated so far and Z
+            // scale by 2^(m_ref - mx); the numerator once the previous half's
+            // P.V (the last one issued for this tile) has completed
             const float new_ref = need ? mx : m_ref;
             const float f = need ? ex2(m_ref - new_ref) : 1.f;
-            if (t > 0) {
+            if (t > 0 || hf > 0) {
               if (!wait(&pv_done[x], (u - 1) & 1)) break;
 #pragma unroll 1
               for (int cc = 0; cc < DH; cc += 16) {
@@ -409,20 +428,6 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
                 for (int e = 0; e < 16; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * f);
                 tmem_st16(nbase + cc, r);
               }
-              tmem_wait_st();
-            }
-            if (h2 == 1) {
-              uint32_t r[32];
-              tmem_wait_st();
-              tmem_ld32(sbase, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) {
-                const __half2 v = *reinterpret_cast<const __half2*>(&r[e]);
-                const float2 fv = __half22float2(v);
-                r[e] = pack_half2(fv.x * f, fv.y * f);
-              }
-              tmem_st32(sbase, r);
             }
             z *= f;
             m_ref = new_ref;
@@ -432,18 +437,19 @@ attn_dense_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constan
           uint32_t pk[32];
 #pragma unroll
           for (int e2 = 0; e2 < 32; ++e2) {
-            const float p0 = ex2(__uint_as_float(s[2 * e2]) - mr);
-            const float p1 = ex2(__uint_as_float(s[2 * e2 + 1]) - mr);
-            za[e2 & 3] += p0 + p1;
+            float x0 = __uint_as_float(s[2 * e2]), x1 = __uint_as_float(s[2 * e2 + 1]);
+            sub2_rn(x0, x1, mr);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (e2 & 1) add2_rn(za[2], za[3], p0, p1);
+            else add2_rn(za[0], za[1], p0, p1);
             pk[e2] = pack_half2(p0, p1);
           }
-          tmem_st32(sbase + 32 * h2, pk);
+          tmem_st32(shalf, pk);
           z += (za[0] + za[1]) + (za[2] + za[3]);
+          tmem_wait_st();
+          tc_fence_before();
+          mbar_arrive(&p_full[2 * x + hf]);
         }
-        if (!ok) break;
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(&p_full[x]);
       }
       if (!ok) break;
       // write-back: O = N / Z, N, m, Z

@@ -1041,14 +1041,7 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
             for (int e = 0; e < 64; ++e)
               if (e >= nvalid) sc[e] = 0xff800000u;  // -inf
           }
-          // eight running maxima (short chains, few live registers next to the
-          // 128 scores)
-          float m8[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) m8[e] = __uint_as_float(sc[e]);
-#pragma unroll
-          for (int e = 8; e < 64; ++e) m8[e & 7] = fmaxf(m8[e & 7], __uint_as_float(sc[e]));
-          mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
+          mx = max64(sc);
         }
         // the reference after tile t-1 (this item's), from the other group
         float m_prev = m_init;
@@ -1104,9 +1097,11 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           uint32_t pk[16];
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
-            const float p0 = ex2(__uint_as_float(sc[32 * hf + 2 * e2]) - m_ref);
-            const float p1 = ex2(__uint_as_float(sc[32 * hf + 2 * e2 + 1]) - m_ref);
-            za[e2 & 3] += p0 + p1;
+            float x0 = __uint_as_float(sc[32 * hf + 2 * e2]), x1 = __uint_as_float(sc[32 * hf + 2 * e2 + 1]);
+            sub2_rn(x0, x1, m_ref);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (e2 & 1) add2_rn(za[2], za[3], p0, p1);
+            else add2_rn(za[0], za[1], p0, p1);
             pk[e2] = pack_half2(p0, p1);
           }
           __syncwarp();
@@ -1132,9 +1127,11 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
           uint32_t pk[16];
 #pragma unroll
           for (int e2 = 0; e2 < 16; ++e2) {
-            const float p0 = ex2(__uint_as_float(sc[32 * hf + 2 * e2]) - m_ref);
-            const float p1 = ex2(__uint_as_float(sc[32 * hf + 2 * e2 + 1]) - m_ref);
-            zb[e2 & 3] += p0 + p1;
+            float x0 = __uint_as_float(sc[32 * hf + 2 * e2]), x1 = __uint_as_float(sc[32 * hf + 2 * e2 + 1]);
+            sub2_rn(x0, x1, m_ref);
+            const float p0 = ex2(x0), p1 = ex2(x1);
+            if (e2 & 1) add2_rn(zb[2], zb[3], p0, p1);
+            else add2_rn(zb[0], zb[1], p0, p1);
             pk[e2] = pack_half2(-p0, -p1);
           }
           __syncwarp();
@@ -1484,10 +1481,12 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
 #pragma unroll
             for (int e4 = 0; e4 < 16; ++e4) {
               const float4 f = sm4[e4];
-              pa[0] += ex2(__uint_as_float(r[4 * e4]) - f.x);
-              pa[1] += ex2(__uint_as_float(r[4 * e4 + 1]) - f.y);
-              pa[2] += ex2(__uint_as_float(r[4 * e4 + 2]) - f.z);
-              pa[3] += ex2(__uint_as_float(r[4 * e4 + 3]) - f.w);
+              float x0 = __uint_as_float(r[4 * e4]), x1 = __uint_as_float(r[4 * e4 + 1]);
+              float x2 = __uint_as_float(r[4 * e4 + 2]), x3 = __uint_as_float(r[4 * e4 + 3]);
+              sub2v_rn(x0, x1, f.x, f.y);
+              sub2v_rn(x2, x3, f.z, f.w);
+              add2_rn(pa[0], pa[1], ex2(x0), ex2(x1));
+              add2_rn(pa[2], pa[3], ex2(x2), ex2(x3));
             }
           } else {
 #pragma unroll

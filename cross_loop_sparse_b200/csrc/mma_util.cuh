@@ -62,4 +62,50 @@ __device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// max(a, b, c) in one instruction (exact, as two fmaxf).
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;\n" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// (a, b) -= (m, m) as one packed float32 pair operation, rounded like two
+// scalar subtractions.
+__device__ __forceinline__ void sub2_rn(float& a, float& b, float m) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %2};\n\t"
+      "sub.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}\n"
+      : "+f"(a), "+f"(b)
+      : "f"(m));
+}
+
+// (a, b) -= (c, d) as one packed float32 pair operation.
+__device__ __forceinline__ void sub2v_rn(float& a, float& b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "sub.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}\n"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+
+// (a, b) += (c, d) as one packed float32 pair operation.
+__device__ __forceinline__ void add2_rn(float& a, float& b, float c, float d) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "add.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}\n"
+      : "+f"(a), "+f"(b)
+      : "f"(c), "f"(d));
+}
+
+// Largest of 64 values (a tree of three-input maxima: 32 instructions).
+__device__ __forceinline__ float max64(const uint32_t (&s)[64]) {
+  float a[22];
+#pragma unroll
+  for (int i = 0; i < 21; ++i)
+    a[i] = max3f(__uint_as_float(s[3 * i]), __uint_as_float(s[3 * i + 1]), __uint_as_float(s[3 * i + 2]));
+  a[21] = __uint_as_float(s[63]);
+  float b[8];
+#pragma unroll
+  for (int i = 0; i < 7; ++i) b[i] = max3f(a[3 * i], a[3 * i + 1], a[3 * i + 2]);
+  b[7] = a[21];
+  return max3f(max3f(b[0], b[1], b[2]), max3f(b[3], b[4], b[5]), fmaxf(b[6], b[7]));
+}
+
 }  // namespace fl
