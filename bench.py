@@ -34,7 +34,7 @@ DECODE_METRIC = "decode tokens/s (B sequences x 1 token x R loops) at S_ctx=32K,
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # DRAM bytes (read + write) of one launch of the dominant kernel, from the ncu captures summarised
 # under profiles/; None once the kernel changes until it is re-captured.
-ATTN_LOOP2_TRAFFIC = {"attn_pp_kernel<128>": 479127296 + 271289600}
+ATTN_LOOP2_TRAFFIC = {"attn_pp_kernel<128>": 479589376 + 271851776}
 ATTN_KERNEL = "attn_pp_kernel<128>"
 # captured on 2 sequences and scaled by 4 (traffic in proportion to the columns read)
 DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": 1169.5e6}
