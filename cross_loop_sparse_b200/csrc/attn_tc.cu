@@ -1218,7 +1218,8 @@ attn_pp_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
 // the tile, so that one group's exponentials overlap the other group's waits
 // and loads; warp 8 allocates TMEM and streams the row tiles (TMA for q, bulk
 // copies for frames and tokens); warp 9 issues the MMAs.  All waits are
-// bounded.
+// bounded.  Three score buffers in TMEM (tile u in buffer u % 3) let the MMA
+// run up to three tiles ahead of the reducers.
 // ---------------------------------------------------------------------------
 constexpr int kCmtCols = 128, kCmtRows = 128, kCmtStages = 4, kCmtThreads = 320;
 constexpr int kCmtRowThreads = 256;
@@ -1231,7 +1232,7 @@ struct CmtCfg {
   static constexpr int kStageBytes = kQBytes + kSideBytes;
   static constexpr int kSmem = 1024 + kCmtStages * kStageBytes + 256 + 2 * 128 * 4;
   static constexpr uint32_t kColA = 0;       // keys, fp16 pairs: DH/2 columns
-  static constexpr uint32_t kColS = 64;      // two S^T buffers of 128 columns
+  static constexpr uint32_t kColS = 64;      // three S^T buffers of 128 columns (tile u in buffer u % 3)
   static constexpr uint32_t kIdesc = f16_idesc(128, kCmtRows, 0);
 };
 
@@ -1274,9 +1275,9 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kCmtStages * C::kStageBytes);
   uint64_t* full = bars;                       // [stages]
   uint64_t* empty = bars + kCmtStages;         // [stages]: MMA commit + 256 reducer arrivals
-  uint64_t* s_full = bars + 2 * kCmtStages;    // [2]
-  uint64_t* s_empty = s_full + 2;              // [2]
-  uint64_t* a_ready = s_empty + 2;             // [1]
+  uint64_t* s_full = bars + 2 * kCmtStages;    // [3]
+  uint64_t* s_empty = s_full + 3;              // [3]
+  uint64_t* a_ready = s_empty + 3;             // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(a_ready + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   float* xsum = reinterpret_cast<float*>(smem + kCmtStages * C::kStageBytes + 256);  // [2][128]
@@ -1293,7 +1294,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1 + kCmtRowThreads / 2);  // MMA commit + the tile's row group
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < 3; ++b) {
       mbar_init(&s_full[b], 1);
       mbar_init(&s_empty[b], kCmtRowThreads / 2);
     }
@@ -1373,21 +1374,22 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
         tc_fence_after();
         bool ok = true;
         for (int t = 0; t < nt; ++t, ++u) {
-          if (!mbar_wait_sleep(&full[stage], phase) || (u >= 2 && !mbar_wait_sleep(&s_empty[u & 1], ((u >> 1) - 1) & 1))) {
+          // buffer u % 3 was last read by tile u - 3 (released by its group)
+          if (!mbar_wait_sleep(&full[stage], phase) || (u >= 3 && !mbar_wait_sleep(&s_empty[u % 3], ((u / 3) - 1) & 1))) {
             set_error(g.err, kDevErrTimeout);
             *abort_flag = 1;
             ok = false;
             break;
           }
           tc_fence_after();
-          const uint32_t sb = tmem + C::kColS + (u & 1) * kCmtRows;
+          const uint32_t sb = tmem + C::kColS + (u % 3) * kCmtRows;
           const uint32_t q_addr = smem_u32(smem + stage * C::kStageBytes);
 #pragma unroll
           for (int ks = 0; ks < DH / 16; ++ks) {
             const uint32_t qd = q_addr + (ks >> 2) * (kCmtRows * 128) + (ks & 3) * 32;
             umma_f16_ts(sb, tmem + C::kColA + ks * 8, sw128_kmajor_desc(qd), C::kIdesc, ks > 0);
           }
-          umma_commit(&s_full[u & 1]);
+          umma_commit(&s_full[u % 3]);
           umma_commit(&empty[stage]);
           if (++stage == kCmtStages) {
             stage = 0;
@@ -1457,7 +1459,7 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
         }
         if ((int)(u & 1) != half) continue;  // the other group's tile
         wait_or_die(&full[st_now], ph_now);
-        wait_or_die(&s_full[u & 1], (u >> 1) & 1);
+        wait_or_die(&s_full[u % 3], (u / 3) & 1);
         if (dead) continue;
         const uint8_t* side = smem + st_now * C::kStageBytes + C::kQBytes;
         const int* stok = reinterpret_cast<const int*>(side + 512);
@@ -1467,13 +1469,13 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
         for (int hh = 0; hh < 2; ++hh) {
           uint32_t r[64];
           __syncwarp();
-          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
-          tmem_ld32(tmem + lane_base + C::kColS + (u & 1) * kCmtRows + hh * 64 + 32,
+          tmem_ld32(tmem + lane_base + C::kColS + (u % 3) * kCmtRows + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(tmem + lane_base + C::kColS + (u % 3) * kCmtRows + hh * 64 + 32,
                     *reinterpret_cast<uint32_t(*)[32]>(r + 32));
           tmem_wait_ld();
           if (hh == 1) {
             tc_fence_before();
-            mbar_arrive(&s_empty[u & 1]);
+            mbar_arrive(&s_empty[u % 3]);
           }
           const float4* sm4 = reinterpret_cast<const float4*>(side) + hh * 16;
           const int* st2 = stok + hh * 64;
