@@ -1362,15 +1362,20 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
     // ------------------------------------------------------------ MMA issue
     if (lane == 0) {
       int stage = 0;
-      uint32_t phase = 0, u = 0, item_no = 0;
-      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x, ++item_no) {
+      uint32_t phase = 0, u = 0, ready_no = 0;  // ready_no: items with row tiles so far
+      for (int item = blockIdx.x; item < total && !*abort_flag; item += gridDim.x) {
         int a_begin;
         const int nt = item_rows(item, a_begin);
-        if (!mbar_wait_sleep(a_ready, item_no & 1)) {
+        if (nt == 0) continue;  // no row reaches the item's columns: no keys, no MMAs
+        // a_ready completes once per item with row tiles, so that the reducers
+        // (who fill the keys of an item only after every tile of the previous
+        // such item) are never two completions ahead of this wait
+        if (!mbar_wait_sleep(a_ready, ready_no & 1)) {
           set_error(g.err, kDevErrTimeout);
           *abort_flag = 1;
           break;
         }
+        ++ready_no;
         tc_fence_after();
         bool ok = true;
         for (int t = 0; t < nt; ++t, ++u) {
@@ -1431,8 +1436,8 @@ colmass_tc_kernel(const __grid_constant__ CUtensorMap tm_q, CmtArgs g) {
       const int c = ct * kCmtCols + col;
       const int ctok = c < g.kc ? (g.cols ? __ldg(g.cols + (size_t)h * g.kc + c) : c) : 0x7fffffff;
       // this column's keys into TMEM (the MMA's A operand): group h loads
-      // elements [h*DH/2, (h+1)*DH/2)
-      if (!dead) {
+      // elements [h*DH/2, (h+1)*DH/2); an item without row tiles needs none
+      if (!dead && nt > 0) {
 #pragma unroll 1
         for (int e0 = half * (DH / 2); e0 < (half + 1) * (DH / 2); e0 += 32) {
           uint32_t r[16];
