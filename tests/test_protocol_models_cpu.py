@@ -1,0 +1,324 @@
+"""Models of two kernels' mbarrier protocols, run as random schedules on the CPU.
+
+An mbarrier wait names only the parity of the phase it wants, so a waiter
+that is two or more completions behind (or ahead) reads the wrong phase.  Each
+model below re-states one kernel's roles as Python generators with the same
+barriers, counts and phase arithmetic, runs them under random interleavings
+(TMA loads land in any order; tcgen05 MMAs and commits complete in issue
+order), and asserts at every poll that the barrier is within one phase of the
+one the waiter wants, and that the schedule always makes progress.
+
+- attn_dense_kernel (csrc/attn_dense.cu): two 128-row tiles per work item, a
+  K/V slot ring released by both tiles' MMA issuers, per-half score, P and
+  P.V barriers, the rescale wait on the previous half's P.V.
+- colmass_tc_kernel (csrc/attn_tc.cu): a q-tile ring, three TMEM score
+  buffers (tile u in buffer u % 3), two reducer groups taking alternate tiles,
+  and the keys barrier used only by work items that have row tiles.
+
+Each model also runs with a planted protocol mistake and must then fail:
+that shows the checks can see the class of error they are there for.
+"""
+import random
+
+import pytest
+
+
+class Bar:
+    def __init__(self, count):
+        self.count, self.pending, self.done = count, 0, 0
+
+    def arrive(self):
+        self.pending += 1
+        if self.pending == self.count:
+            self.pending = 0
+            self.done += 1
+
+
+class Stuck(Exception):
+    pass
+
+
+def wait(bars, name, k):
+    """Wait for the completion of phase k (k < 0: a fresh barrier's 'previous
+    phase', always complete).  A poll checks k <= completed <= k + 1."""
+    while True:
+        b = bars[name]
+        if k >= 0:
+            assert k <= b.done <= k + 1, (name, k, b.done)
+        if b.done > k:
+            return
+        yield None
+
+
+def run_schedule(bars, threads, loads, pipe, rnd, idle_limit=20000):
+    """Interleave the roles at random with the two asynchronous engines: TMA
+    loads (complete in any order) and the MMA pipe (in issue order)."""
+    alive, idle = list(threads), 0
+    while alive:
+        moved = False
+        if loads and rnd.random() < 0.5:
+            bars[loads.pop(rnd.randrange(len(loads)))].arrive()
+            moved = True
+        if pipe and rnd.random() < 0.5:
+            kind, name = pipe.pop(0)
+            if kind == "commit":
+                bars[name].arrive()
+            moved = True
+        th = rnd.choice(alive)
+        try:
+            step = next(th)
+            idle = 0 if (step is not None or moved) else idle + 1
+        except StopIteration:
+            alive.remove(th)
+            idle = 0
+        if idle > idle_limit and not loads and not pipe:
+            raise Stuck()
+
+
+# --------------------------------------------------------------- attn_dense_kernel
+ROWS, COLS = 128, 128
+
+
+def dn_tiles(S, p, x):
+    first = p * 2 * ROWS + x * ROWS
+    if first >= S:
+        return 0
+    return (min(S, first + ROWS) - 1 + COLS) // COLS
+
+
+def dense_cta(S, H, grid, blk, stages, rnd, plant=None):
+    pairs = (S + 2 * ROWS - 1) // (2 * ROWS)
+    total = pairs * H
+    items = list(range(blk, total, grid))
+    item_p = lambda it: pairs - 1 - it % pairs
+    B = {}
+    for s in range(stages):
+        B[("kv_full", s)] = Bar(1)
+        B[("kv_empty", s)] = Bar(1 if plant == "kv_empty_count" else 2)
+    for i in range(4):
+        B[("s_full", i)] = Bar(1)
+        B[("p_full", i)] = Bar(1)  # the 128 row threads move together in the model
+    for x in range(2):
+        for n in ("pv_done", "acc_full", "n_free", "q_full", "q_empty"):
+            B[(n, x)] = Bar(1)
+    B["fin"] = Bar(2)
+    loads, pipe = [], []
+
+    def tma():
+        seq = 0
+        for item in items:
+            p = item_p(item)
+            for _t in range(max(dn_tiles(S, p, 0), dn_tiles(S, p, 1))):
+                for _kv in range(2):
+                    yield from wait(B, ("kv_empty", seq % stages), seq // stages - 1)
+                    loads.append(("kv_full", seq % stages))
+                    seq += 1
+
+    def issuer(x):
+        seq = u = 0
+        slot, phase = (lambda s: s % stages), (lambda s: s // stages)
+
+        def skip(s):
+            yield from wait(B, ("kv_full", slot(s)), phase(s))
+            B[("kv_empty", slot(s))].arrive()
+
+        for item_no, item in enumerate(items):
+            p = item_p(item)
+            my = dn_tiles(S, p, x)
+            nt = max(dn_tiles(S, p, 0), dn_tiles(S, p, 1))
+            yield from wait(B, ("q_full", x), item_no)
+            if my == 0:
+                pipe.append(("commit", ("q_empty", x)))
+            base = seq
+            if nt > 0:
+                if my > 0:
+                    yield from wait(B, ("kv_full", slot(base)), phase(base))
+                    for hf in range(2):
+                        pipe.extend([("mma", None), ("commit", ("s_full", 2 * x + hf))])
+                    if my == 1:
+                        pipe.append(("commit", ("q_empty", x)))
+                    pipe.append(("commit", ("kv_empty", slot(base))))
+                else:
+                    yield from skip(base)
+            for t in range(nt):
+                vs, ks = base + 2 * t + 1, base + 2 * t + 2
+                if t >= my:
+                    yield from skip(vs)
+                    if t + 1 < nt:
+                        yield from skip(ks)
+                    continue
+                yield from wait(B, ("kv_full", slot(vs)), phase(vs))
+                for hf in range(2):
+                    if t == 0 and hf == 0 and item_no > 0:
+                        yield from wait(B, ("n_free", x), item_no - 1)
+                    yield from wait(B, ("p_full", 2 * x + hf), u >> 1)
+                    pipe.extend([("mma", None), ("commit", ("pv_done", x))])
+                    if t == my - 1 and hf == 1:
+                        pipe.append(("commit", ("acc_full", x)))
+                    if t + 1 < my:
+                        if hf == 0:
+                            yield from wait(B, ("kv_full", slot(ks)), phase(ks))
+                        pipe.extend([("mma", None), ("commit", ("s_full", 2 * x + hf))])
+                        if t + 1 == my - 1 and hf == 1:
+                            pipe.append(("commit", ("q_empty", x)))
+                    u += 1
+                pipe.append(("commit", ("kv_empty", slot(vs))))
+                if t + 1 < nt:
+                    if t + 1 < my:
+                        pipe.append(("commit", ("kv_empty", slot(ks))))
+                    else:
+                        yield from skip(ks)
+            if my == 0:
+                if item_no > 0:
+                    yield from wait(B, ("n_free", x), item_no - 1)
+                pipe.append(("commit", ("acc_full", x)))
+            seq = base + 2 * nt
+        pipe.append(("commit", "fin"))
+        yield from wait(B, "fin", 0)
+
+    def queries():
+        if items:
+            for x in range(2):
+                B[("q_full", x)].arrive()
+        for item_no in range(len(items) - 1):
+            for x in range(2):
+                yield from wait(B, ("q_empty", x), item_no)
+                B[("q_full", x)].arrive()
+
+    def rows(x):
+        u = 0
+        for item_no, item in enumerate(items):
+            for t in range(dn_tiles(S, item_p(item), x)):
+                for hf in range(2):
+                    yield from wait(B, ("s_full", 2 * x + hf), u >> 1)
+                    if (t > 0 or hf > 0) and rnd.random() < 0.3:  # the running maximum rose
+                        k = u if plant == "pv_phase" else u - 1
+                        yield from wait(B, ("pv_done", x), k)
+                    for _ in range(rnd.randint(0, 3)):
+                        yield None
+                    B[("p_full", 2 * x + hf)].arrive()
+                    u += 1
+            yield from wait(B, ("acc_full", x), item_no)
+            B[("n_free", x)].arrive()
+
+    threads = [tma(), issuer(0), issuer(1), queries(), rows(0), rows(1)]
+    run_schedule(B, threads, loads, pipe, rnd)
+
+
+DENSE_SHAPES = [(256, 2, 4), (300, 2, 3), (40, 1, 1), (1000, 3, 5), (4096, 2, 7), (129, 2, 1), (513, 2, 148)]
+
+
+@pytest.mark.parametrize("S,H,grid", DENSE_SHAPES)
+def test_dense_protocol_phases_and_progress(S, H, grid):
+    pairs = (S + 2 * ROWS - 1) // (2 * ROWS)
+    for stages in (5, 10):
+        for seed in range(3):
+            rnd = random.Random(seed * 1000 + S)
+            for blk in range(min(grid, pairs * H)):
+                dense_cta(S, H, grid, blk, stages, rnd)
+
+
+@pytest.mark.parametrize("plant", ["pv_phase", "kv_empty_count"])
+def test_dense_protocol_model_catches_planted_mistakes(plant):
+    caught = 0
+    for seed in range(5):
+        try:
+            dense_cta(1000, 1, 1, 0, 5, random.Random(seed), plant=plant)
+        except (AssertionError, Stuck):
+            caught += 1
+    assert caught > 0
+
+
+# --------------------------------------------------------------- colmass_tc_kernel
+def colmass_cta(nts, stages, nbuf, rnd, keys_every_item=False):
+    """nts: row tiles of each of the CTA's work items (0: no row reaches the
+    item's columns).  keys_every_item models a keys barrier completed by every
+    item, with or without row tiles."""
+    B = {}
+    for s in range(stages):
+        B[("full", s)] = Bar(1)
+        B[("empty", s)] = Bar(2)  # the MMA commit + the tile's reducer group
+    for b in range(nbuf):
+        B[("s_full", b)] = Bar(1)
+        B[("s_empty", b)] = Bar(1)
+    B["a_ready"] = Bar(2)  # both reducer groups
+    B["pair"] = Bar(2)  # the named barrier between the groups at an item's end
+    loads, pipe = [], []
+
+    def loader():
+        fills = [0] * stages
+        u = 0
+        for nt in nts:
+            for _t in range(nt):
+                st = u % stages
+                yield from wait(B, ("empty", st), fills[st] - 1)
+                loads.append(("full", st))
+                fills[st] += 1
+                u += 1
+
+    def mma():
+        uses = [0] * stages
+        u = ready_no = 0
+        for item_no, nt in enumerate(nts):
+            if keys_every_item:
+                yield from wait(B, "a_ready", item_no)
+            elif nt > 0:
+                yield from wait(B, "a_ready", ready_no)
+                ready_no += 1
+            for _ in range(rnd.randint(0, 30)):  # a late MMA thread
+                yield None
+            for _t in range(nt):
+                st = u % stages
+                yield from wait(B, ("full", st), uses[st])
+                uses[st] += 1
+                if u >= nbuf:
+                    yield from wait(B, ("s_empty", u % nbuf), u // nbuf - 1)
+                pipe.extend([("mma", None), ("commit", ("s_full", u % nbuf)), ("commit", ("empty", st))])
+                u += 1
+
+    def reducers(grp):
+        uses = [0] * stages
+        u = gen = 0
+        for nt in nts:
+            if keys_every_item or nt > 0:
+                B["a_ready"].arrive()
+            for _t in range(nt):
+                st = u % stages
+                k = uses[st]
+                uses[st] += 1
+                if u % 2 == grp:
+                    yield from wait(B, ("full", st), k)
+                    yield from wait(B, ("s_full", u % nbuf), u // nbuf)
+                    for _ in range(rnd.randint(0, 3)):
+                        yield None
+                    B[("s_empty", u % nbuf)].arrive()
+                    for _ in range(rnd.randint(0, 3)):
+                        yield None
+                    B[("empty", st)].arrive()
+                u += 1
+            B["pair"].arrive()
+            gen += 1
+            yield from wait(B, "pair", gen - 1)
+
+    run_schedule(B, [loader(), mma(), reducers(0), reducers(1)], loads, pipe, rnd, idle_limit=5000)
+
+
+def _random_items(rnd):
+    return [rnd.choice([0, 0, 1, 2, 3, 5]) for _ in range(rnd.randint(1, 8))]
+
+
+def test_colmass_protocol_phases_and_progress():
+    for seed in range(200):
+        rnd = random.Random(seed)
+        colmass_cta(_random_items(rnd), 4, 3, rnd)
+
+
+def test_colmass_protocol_model_catches_a_keys_barrier_on_empty_items():
+    caught = 0
+    for seed in range(200):
+        rnd = random.Random(seed)
+        try:
+            colmass_cta(_random_items(rnd), 4, 3, rnd, keys_every_item=True)
+        except (AssertionError, Stuck):
+            caught += 1
+    assert caught > 0
