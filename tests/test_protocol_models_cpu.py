@@ -14,6 +14,11 @@ one the waiter wants, and that the schedule always makes progress.
 - colmass_tc_kernel (csrc/attn_tc.cu): a q-tile ring, three TMEM score
   buffers (tile u in buffer u % 3), two reducer groups taking alternate tiles,
   and the keys barrier used only by work items that have row tiles.
+- attn_pp_kernel (csrc/attn_tc.cu): K and V rings, two score issuers and a
+  P.V issuer, per-half and per-parity score barriers, the P buffers' reuse
+  wait, the rescale wait on the other group's P.V (four barriers by t mod 4),
+  the named-barrier hand-off of the running reference between the two row
+  groups, and the q barrier used only by work items that have column tiles.
 
 Each model also runs with a planted protocol mistake and must then fail:
 that shows the checks can see the class of error they are there for.
@@ -319,6 +324,151 @@ def test_colmass_protocol_model_catches_a_keys_barrier_on_empty_items():
         rnd = random.Random(seed)
         try:
             colmass_cta(_random_items(rnd), 4, 3, rnd, keys_every_item=True)
+        except (AssertionError, Stuck):
+            caught += 1
+    assert caught > 0
+
+
+# --------------------------------------------------------------- attn_pp_kernel
+class NamedHandoff:
+    """bar.arrive by the giving warp, bar.sync by the taking warp, one barrier
+    id reused for every hand-off: a second give before the take would count
+    towards the same barrier instance, so at most one may be outstanding."""
+
+    def __init__(self):
+        self.given = 0
+        self.taken = 0
+
+    def give(self):
+        assert self.given == self.taken, "a second give before the take"
+        self.given += 1
+
+    def take(self):
+        while self.given == self.taken:
+            yield None
+        self.taken += 1
+
+
+def pp_cta(nts, stages, rnd, plant=None):
+    """nts: column tiles of each of the CTA's work items (0: no selected column
+    at or before the item's rows).  Row groups take alternate tiles by a
+    block-wide counter u; both groups load the item's q and N halves, hand
+    the running reference to each other per tile, and meet at the item's end."""
+    B = {}
+    for s in range(stages):
+        B[("k_full", s)] = Bar(1)
+        B[("k_empty", s)] = Bar(2)  # both score halves
+        B[("v_full", s)] = Bar(1)
+        B[("v_empty", s)] = Bar(1)
+    for i in range(4):
+        B[("s_full", i)] = Bar(1)
+        B[("pv_done4", i)] = Bar(1)
+    for i in range(2):
+        B[("s_empty", i)] = Bar(1)  # the tile's group
+        B[("p_full", i)] = Bar(1)
+        B[("pv_done", i)] = Bar(1)
+    B["q_ready"] = Bar(2)  # both groups
+    B["end"] = Bar(2)
+    hand = [NamedHandoff(), NamedHandoff()]  # hand[g]: group g gives to the other
+    loads, pipe = [], []
+
+    def loader():
+        ks = vs = 0
+        kfill = [0] * stages
+        vfill = [0] * stages
+        for nt in nts:
+            for _t in range(nt):
+                yield from wait(B, ("k_empty", ks), kfill[ks] - 1)
+                loads.append(("k_full", ks))
+                kfill[ks] += 1
+                ks = (ks + 1) % stages
+                yield from wait(B, ("v_empty", vs), vfill[vs] - 1)
+                loads.append(("v_full", vs))
+                vfill[vs] += 1
+                vs = (vs + 1) % stages
+
+    def s_half(half):
+        u = item_no = 0
+        for nt in nts:
+            if nt == 0:
+                continue
+            yield from wait(B, "q_ready", item_no)
+            item_no += 1
+            for _t in range(nt):
+                ks = u % stages
+                yield from wait(B, ("k_full", ks), u // stages)
+                if u > 0:
+                    yield from wait(B, ("s_empty", half), u - 1)
+                pipe.extend([("mma", None), ("commit", ("s_full", 2 * half + (u & 1))), ("commit", ("k_empty", ks))])
+                u += 1
+
+    def pv():
+        u = 0
+        for nt in nts:
+            for _t in range(nt):
+                yield from wait(B, ("p_full", u & 1), u >> 1)
+                yield from wait(B, ("v_full", u % stages), u // stages)
+                pipe.extend([("mma", None), ("commit", ("v_empty", u % stages)), ("commit", ("pv_done", u & 1)),
+                             ("commit", ("pv_done4", u & 3))])
+                u += 1
+
+    def rows(grp):
+        u = 0
+        end_gen = 0
+        for nt in nts:
+            if nt > 0:
+                B["q_ready"].arrive()
+            for t in range(nt):
+                b = u & 1
+                if b != grp:
+                    u += 1
+                    continue
+                yield from wait(B, ("s_full", b), u >> 1)
+                B[("s_empty", 0)].arrive()
+                if t > 0:
+                    yield from hand[grp ^ 1].take()
+                if t + 1 < nt:
+                    hand[grp].give()
+                if u >= 2:
+                    yield from wait(B, ("pv_done", b), (u - 2) >> 1)
+                if t > 0 and rnd.random() < 0.3:  # the reference rose: N waits for P(t-1).V
+                    k = (u - 1) >> 2
+                    if plant == "pv_done4_phase":
+                        k += 1
+                    yield from wait(B, ("pv_done4", (u - 1) & 3), k)
+                for _ in range(rnd.randint(0, 3)):
+                    yield None
+                yield from wait(B, ("s_full", 2 + b), u >> 1)
+                B[("s_empty", 1)].arrive()
+                B[("p_full", b)].arrive()
+                u += 1
+            if nt > 0:
+                yield from wait(B, ("pv_done4", (u - 1) & 3), (u - 1) >> 2)
+            for _sync in range(2):
+                B["end"].arrive()
+                end_gen += 1
+                yield from wait(B, "end", end_gen - 1)
+
+    threads = [loader(), s_half(0), s_half(1), pv(), rows(0), rows(1)]
+    run_schedule(B, threads, loads, pipe, rnd, idle_limit=5000)
+
+
+def _pp_items(rnd):
+    return [rnd.choice([0, 1, 1, 2, 3, 4, 5, 7]) for _ in range(rnd.randint(1, 7))]
+
+
+def test_pp_protocol_phases_and_progress():
+    for seed in range(300):
+        rnd = random.Random(seed)
+        pp_cta(_pp_items(rnd), 3, rnd)
+
+
+def test_pp_protocol_model_catches_a_planted_phase():
+    caught = 0
+    for seed in range(100):
+        rnd = random.Random(seed)
+        try:
+            pp_cta(_pp_items(rnd), 3, rnd, plant="pv_done4_phase")
         except (AssertionError, Stuck):
             caught += 1
     assert caught > 0
