@@ -158,7 +158,7 @@ def run_cuda(args, cfg, rank, world, local_rank):
     xs = [to_dev(x) for x in X]
     wqkv, wo = to_dev(W["wqkv"]), to_dev(W["wo"])
     paper = args.kv_scheme == "paper"
-    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass, attn_pairs=args.sm_pairs, kv_scheme=args.kv_scheme)
+    p = F.Params.from_config(cfg, fixed_mass=args.fixed_mass, kv_scheme=args.kv_scheme)
     st = F.FlashLoopState(p, device=dev)
     S, d, R = cfg.seq, cfg.d_model, cfg.n_loops
     F.flashloop_loop_step(p, 1, xs[0], None, wqkv, wo, st)
@@ -281,11 +281,9 @@ def run_cuda(args, cfg, rank, world, local_rank):
     achieved = flop2 / (ms2 * 1e-3) / 1e12
     roofline = {"bound": "tensor", "achieved": round(achieved, 2), "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": round(achieved / peaks["bf16_tflops"], 4),
-                "traffic": None if (args.fixed_mass or args.sm_pairs) else ATTN_LOOP2_TRAFFIC.get(ATTN_KERNEL),
+                "traffic": None if args.fixed_mass else ATTN_LOOP2_TRAFFIC.get(ATTN_KERNEL),
                 "kernel": ("attn_tc_kernel<128> statistics + update passes, loop 2 (fixed-mass form, tcgen05)"
                            if args.fixed_mass else
-                           "attn_pair_kernel<128>, loop-2 launch (sparse attention update, tcgen05 on SM pairs)"
-                           if args.sm_pairs else
                            f"{ATTN_KERNEL}, loop-2 launch (sparse attention update, tcgen05)"),
                 "algorithmic": f"8*dh FLOP x {pairs[2]} causal-valid (row, column, head) pairs = {flop2:.4g} FLOP",
                 "peak_source": f"{peak_kind} bf16 dense burst (fp16 operands run at the bf16 rate)",
@@ -384,8 +382,6 @@ def run_cuda(args, cfg, rank, world, local_rank):
     # a variant of the path: the config says so (the reference arm has no such line)
     if args.fixed_mass:
         variants.append("fixed-mass form of the update")
-    if args.sm_pairs:
-        variants.append("attention on SM pairs")
     if paper:
         variants.append("the pages' cache setting (INT4 asymmetric groups of 64, 64-token bf16 tail)")
     variant = ", ".join(variants) or None
@@ -760,8 +756,6 @@ def main():
     ap.add_argument("--fixed-mass", action="store_true",
                     help="prefill workloads: the fixed-mass form of the sparse update (no CPU baseline: its "
                          "oracle keeps explicit S x S distributions)")
-    ap.add_argument("--sm-pairs", action="store_true",
-                    help="prefill workloads: the running update on SM pairs (cta_group::2)")
     ap.add_argument("--kv-scheme", choices=["spec", "paper"], default="spec",
                     help="prefill workloads: K/V streams as INT8 + INT4/INT2 symmetric residuals (spec) or the "
                          "pages' own setting, INT4 asymmetric groups of 64 with a 64-token bf16 tail (paper)")

@@ -77,6 +77,7 @@ static int check_params(const flashloop_params* p) {
   if (p->d_model % 128 != 0) return FLASHLOOP_ERR_UNSUPPORTED;
   if (!(p->tau >= 0.f) || !(p->rope_theta > 0.f)) return FLASHLOOP_ERR_INVALID_ARG;
   if (p->kv_scheme != 0 && p->kv_scheme != 1) return FLASHLOOP_ERR_UNSUPPORTED;
+  if (p->attn_pairs != 0) return FLASHLOOP_ERR_UNSUPPORTED;  // reserved
   if (p->kv_scheme == 0 && p->bits[0] != 8) return FLASHLOOP_ERR_UNSUPPORTED;
   for (int r = 2; r <= p->n_loops; ++r) {
     const int b = p->bits[r - 1];

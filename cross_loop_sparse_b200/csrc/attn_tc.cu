@@ -1697,17 +1697,10 @@ int launch_colmass_tc(const flashloop_params* p, const ColmassArgs& a, void* scr
 }
 
 // K buffers are [H, kcp, dh], V^T buffers [H, dh, kcp] (fp16), kcp = kc rounded up to 8.
-int launch_attn_pair(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream);
 int launch_attn_dense(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream);
 
 int launch_attn_tc(const flashloop_params* p, const AttnArgs& a, int kcp, cudaStream_t stream) {
   const int dh = p->head_dim, H = p->n_heads;
-  if (a.mode == kAtRunning && p->attn_pairs) {
-    // the running update on SM pairs (half of every K / V tile per SM), where
-    // the device can co-schedule them
-    const int rc = launch_attn_pair(p, a, kcp, stream);
-    if (rc != FLASHLOOP_ERR_UNSUPPORTED) return rc;
-  }
   // the dense loop: two row tiles per CTA sharing every K / V tile (attn_dense.cu)
   if (a.mode == kAtRunning && a.dense) return launch_attn_dense(p, a, kcp, stream);
   if (a.cols != nullptr && a.row_cnt == nullptr) return FLASHLOOP_ERR_INVALID_ARG;

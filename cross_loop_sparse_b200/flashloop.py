@@ -47,15 +47,15 @@ class Params(ctypes.Structure):
 
     @classmethod
     def from_config(cls, cfg, capacity=None, topk=None, tau=None, seq=None, token_budgets=None,
-                    fixed_mass=False, attn_pairs=False, kv_scheme="spec"):
+                    fixed_mass=False, kv_scheme="spec"):
         """Params of a workload.Config; capacities default to S (no overflow possible).
         token_budgets (per loop) selects top-k token retention with those budgets;
-        fixed_mass selects the fixed-mass form of the sparse update; attn_pairs runs
-        the running update on SM pairs."""
+        fixed_mass selects the fixed-mass form of the sparse update; attn_pairs
+        (reserved) stays 0."""
         p = cls()
         p.kv_scheme = {"spec": 0, "paper": 1}[kv_scheme]
         p.fixed_mass = 1 if fixed_mass else 0
-        p.attn_pairs = int(attn_pairs)
+        p.attn_pairs = 0
         p.seq = cfg.seq if seq is None else seq
         p.d_model, p.n_heads, p.head_dim = cfg.d_model, cfg.n_heads, cfg.head_dim
         p.n_loops, p.batch = cfg.n_loops, (cfg.batch if cfg.decode else 1)

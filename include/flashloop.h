@@ -79,8 +79,8 @@ typedef struct flashloop_params {
   int32_t capacity[FLASHLOOP_MAX_LOOPS]; /* rows allocated for loop r's active list and residual stream */
   int32_t gate_topk; /* 0: the tau threshold gate; else top-k token retention keeping capacity[r-1] tokens */
   int32_t fixed_mass; /* 0: running (m, N, Z) update; else the fixed-mass form (see flashloop_sparse_attn_update) */
-  int32_t attn_pairs; /* running update: 0 one SM per 128-row tile; 1 / 2 SM pairs sharing each K/V tile
-                         (cta_group::2) with two / four row threads per row */
+  int32_t attn_pairs; /* reserved, must be 0 (FLASHLOOP_ERR_UNSUPPORTED otherwise): the running update
+                         takes one SM per work item */
   int32_t kv_scheme;  /* 0: INT8 base + INT4/INT2 symmetric residuals (flashloop_kv streams);
                          1: the pages' own setting (flashloop_paper_kv streams, see below; prefill only) */
 } flashloop_params;

@@ -112,6 +112,8 @@ def test_host_checks_reject_bad_params():
     assert _status(p) == -1
     p = F.Params.from_config(cfg); p.n_loops = 17
     assert _status(p) == -1
+    p = F.Params.from_config(cfg); p.attn_pairs = 1  # reserved field
+    assert _status(p) == -2
     assert F.flashloop_status_string(-2).startswith("unsupported")
 
 

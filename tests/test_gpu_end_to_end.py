@@ -31,9 +31,8 @@ from gpu_helpers import bf16_rows, bf16_to_torch, row_rel_l2, torch_to_bf16_bits
 TOL = 1e-2
 
 
-def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None, fixed_mass=False, tau=None, attn_pairs=False):
-    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets, fixed_mass=fixed_mass, tau=tau,
-                             attn_pairs=attn_pairs)
+def run_gpu(cfg, W, X, stream=None, topk=None, token_budgets=None, fixed_mass=False, tau=None):
+    p = F.Params.from_config(cfg, topk=topk, token_budgets=token_budgets, fixed_mass=fixed_mass, tau=tau)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
@@ -192,12 +191,12 @@ def force_selection(p, orc, st, r, heads):
     st[f"cols{r}"][heads] = torch.from_numpy(np.stack(orc.T[r]).astype(np.int32)).cuda()
 
 
-def run_chained(cfg, W, X, orc, heads, check_y, topk=None, fixed_mass=False, tau=None, attn_pairs=0):
+def run_chained(cfg, W, X, orc, heads, check_y, topk=None, fixed_mass=False, tau=None):
     """Loops 1..R through the calls flashloop_loop_step makes, the oracle's
     codes and selections written into the GPU state after each is checked
     (oracle -> GPU); then O of the held heads (and Y, with every head held)
     within TOL on every active row.  Returns the per-loop worst errors."""
-    p = F.Params.from_config(cfg, topk=topk, fixed_mass=fixed_mass, tau=tau, attn_pairs=attn_pairs)
+    p = F.Params.from_config(cfg, topk=topk, fixed_mass=fixed_mass, tau=tau)
     st = F.FlashLoopState(p)
     xs = [bf16_to_torch(x) for x in X]
     wqkv, wo = bf16_to_torch(W["wqkv"]), bf16_to_torch(W["wo"])
@@ -483,20 +482,3 @@ def test_loop_step_fixed_mass_matches_oracle(case):
             assert abs(got - want) <= 2e-2 * want + 1e-6, (h, int(i), got, want)
     assert st.error_code() == 0
 
-
-@pytest.mark.parametrize("pairs", [1, 2])
-@pytest.mark.parametrize("name", ["tiny", "ouro14_4k"])
-def test_loop_step_on_sm_pairs_matches_oracle(name, pairs):
-    """The running update on SM pairs (two CTAs share every K / V tile, each
-    loading half; cta_group::2 MMAs over 256 rows), loop 1 included, with two
-    (pairs = 1) or four (pairs = 2) threads per row."""
-    cfg = CONFIGS[name]
-    W = make_weights(cfg)
-    X, _ = make_hidden_states(cfg)
-    orc = O.OracleSequence(cfg, W, X).run()
-    heads = list(range(cfg.n_heads))
-    chained = run_chained(cfg, W, X, orc, heads, True, attn_pairs=pairs)
-    p, st, snaps = run_gpu(cfg, W, X, attn_pairs=pairs)
-    assert p.attn_pairs == pairs
-    free = compare(cfg, orc, snaps, st, heads, True)
-    print(name, "pairs", "chained", chained, "free-running", free)
