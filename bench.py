@@ -38,6 +38,7 @@ ATTN_LOOP2_TRAFFIC = {"attn_pp_kernel<128>": 479589376 + 271851776}
 ATTN_KERNEL = "attn_pp_kernel<128>"
 # captured on 2 sequences and scaled by 4 (traffic in proportion to the columns read)
 DECODE_DENSE_TRAFFIC = {"decode_dense_kernel<128,8>": 1169.5e6}
+L2_BYTES = 126e6  # B200 L2 (126 MB)
 
 
 def max_over_ranks(value, device=None):
@@ -63,8 +64,12 @@ def load_peaks():
 def run_config(cfg, world, active_tokens, pairs):
     """The config object of both arms' lines (identical keys and values for
     the same workload, so the two lines compare)."""
+    x_mib = cfg.seq * cfg.d_model * 2 / 2**20            # one bf16 X_r
+    n_mib = cfg.n_heads * cfg.seq * cfg.head_dim * 4 / 2**20  # one float32 N slot
+    size = "larger" if cfg.seq * cfg.d_model * 2 > L2_BYTES else "smaller"
     return {"workload": workload_desc(cfg),
-            "l2": "inputs larger than L2: each X_r is 128 MiB and the N state 256 MiB per slot",
+            "l2": f"inputs {size} than L2 (126 MB): each X_r is {x_mib:g} MiB and the N state "
+                  f"{n_mib:g} MiB per slot",
             "parallelism": f"one sequence per rank, {world} rank(s), no exchange",
             "active_tokens": {f"loop{r}": int(n) for r, n in sorted(active_tokens.items())},
             "attention_pairs": {f"loop{r}": int(v) for r, v in sorted(pairs.items())}}
