@@ -19,6 +19,9 @@ one the waiter wants, and that the schedule always makes progress.
   wait, the rescale wait on the other group's P.V (four barriers by t mod 4),
   the named-barrier hand-off of the running reference between the two row
   groups, and the q barrier used only by work items that have column tiles.
+- tc_gemm_kernel (csrc/gemm_tc.cu): the A/B stage ring filled by the
+  gathering warps and TMA, the MMA thread, and the two TMEM accumulators the
+  epilogue drains while the next tile fills.
 
 Each model also runs with a planted protocol mistake and must then fail:
 that shows the checks can see the class of error they are there for.
@@ -469,6 +472,76 @@ def test_pp_protocol_model_catches_a_planted_phase():
         rnd = random.Random(seed)
         try:
             pp_cta(_pp_items(rnd), 3, rnd, plant="pv_done4_phase")
+        except (AssertionError, Stuck):
+            caught += 1
+    assert caught > 0
+
+
+# --------------------------------------------------------------- tc_gemm_kernel
+def gemm_cta(n_tiles, k_steps, stages, rnd, plant=None):
+    """The persistent projection: per tile, k_steps stages of A rows (gathered
+    by the producer warps, arriving when their copies land) and a B tile (TMA),
+    an MMA thread consuming them in order into one of two TMEM accumulators,
+    and the epilogue warps draining an accumulator while the next fills."""
+    B = {}
+    for s in range(stages):
+        B[("full", s)] = Bar(2)  # the producers' arrival (cp.async landed) + the TMA's bytes
+        B[("empty", s)] = Bar(1)
+    for b in range(2):
+        B[("acc_full", b)] = Bar(1)
+        B[("acc_empty", b)] = Bar(1)  # the epilogue threads
+    loads, pipe = [], []
+    total = n_tiles * k_steps
+
+    def producers():
+        for i in range(total):
+            st = i % stages
+            yield from wait(B, ("empty", st), i // stages - 1)
+            loads.append(("full", st))  # the gathered rows land
+
+    def tma():
+        for i in range(total):
+            st = i % stages
+            yield from wait(B, ("empty", st), i // stages - 1)
+            loads.append(("full", st))
+
+    def mma():
+        i = 0
+        for it in range(n_tiles):
+            buf = it & 1
+            k = it >> 1
+            if plant == "acc_phase":
+                k += 1
+            yield from wait(B, ("acc_empty", buf), k - 1)
+            for _k in range(k_steps):
+                yield from wait(B, ("full", i % stages), i // stages)
+                pipe.extend([("mma", None), ("commit", ("empty", i % stages))])
+                i += 1
+            pipe.append(("commit", ("acc_full", buf)))
+
+    def epilogue():
+        for it in range(n_tiles):
+            buf = it & 1
+            yield from wait(B, ("acc_full", buf), it >> 1)
+            for _ in range(rnd.randint(0, 5)):
+                yield None
+            B[("acc_empty", buf)].arrive()
+
+    run_schedule(B, [producers(), tma(), mma(), epilogue()], loads, pipe, rnd, idle_limit=5000)
+
+
+def test_gemm_protocol_phases_and_progress():
+    for seed in range(100):
+        rnd = random.Random(seed)
+        gemm_cta(rnd.randint(1, 7), rnd.randint(1, 9), 4, rnd)
+
+
+def test_gemm_protocol_model_catches_a_planted_phase():
+    caught = 0
+    for seed in range(30):
+        rnd = random.Random(seed)
+        try:
+            gemm_cta(5, 3, 4, rnd, plant="acc_phase")
         except (AssertionError, Stuck):
             caught += 1
     assert caught > 0
