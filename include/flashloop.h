@@ -159,7 +159,8 @@ typedef struct flashloop_state {
 
 /* ---------------------------------------------------------------- sizing */
 
-/* Scratch bytes the calls below need in state->workspace (host function). */
+/* Scratch bytes the calls below need in state->workspace (host function; a
+ * sizing helper, not an operation of the method). */
 size_t flashloop_workspace_bytes(const flashloop_params* p);
 
 /* Cache bytes of K and V for the given active counts n_r (n[0] = S):
@@ -169,7 +170,10 @@ size_t flashloop_cache_bytes(const flashloop_params* p, const int32_t* n_per_loo
 
 /* Fill the RoPE table: cs[2*(t*dh/2 + i)] = cos(t * theta^(-2i/dh)),
  * cs[2*(...)+1] = sin(...), for t < n_pos, computed in double precision and
- * rounded to float.  Rotate-half pairing (i, i + dh/2). */
+ * rounded to float.  Rotate-half pairing (i, i + dh/2).  [FlashLoop App. E
+ * quantises keys after RoPE; the pages fix no RoPE variant, and the
+ * rotate-half form with theta = p->rope_theta and position = token index is
+ * taken.]  cs: device, caller-owned, n_pos * dh floats. */
 int flashloop_rope_table(const flashloop_params* p, int32_t n_pos, float* cs, void* stream);
 
 /* ---------------------------------------------------------------- the path */
@@ -329,7 +333,10 @@ int flashloop_sparse_attn_update(const flashloop_params* p, int32_t loop, flashl
                                  int32_t want_colmass, void* stream);
 
 /* (a7) Gathered output projection: for a < *n_active, t = active[a]:
- * y[t] = bf16(o[t] W_o^T) (float32 accumulation); other rows untouched. */
+ * y[t] = bf16(o[t] W_o^T) (float32 accumulation); other rows untouched.
+ * [FlashLoop §4.1: active-token execution recomputes only the active rows;
+ * the sublayer's output weight W_o completes the attention block.]
+ * o, y: bf16 [S, d_model] (row = token); w_o: bf16 [d_model, d_model]. */
 int flashloop_out_proj(const flashloop_params* p, const uint16_t* o, const int32_t* active,
                        const int32_t* n_active, int32_t capacity, const uint16_t* w_o, uint16_t* y,
                        void* stream);
@@ -354,7 +361,8 @@ int flashloop_loop_step(const flashloop_params* p, int32_t loop, const uint16_t*
 int flashloop_kv_step(const flashloop_params* p, int32_t loop, const uint16_t* x_cur, const uint16_t* x_prev,
                       const uint16_t* w_qkv, flashloop_state* st, void* stream);
 
-/* Scratch bytes flashloop_kv_step needs in st->workspace (zero-filled once). */
+/* Scratch bytes flashloop_kv_step needs in st->workspace (zero-filled once;
+ * a sizing helper). */
 size_t flashloop_kv_workspace_bytes(const flashloop_params* p);
 
 /* ---------------------------------------------------------------- decode */
@@ -385,7 +393,8 @@ typedef struct flashloop_decode_state {
   size_t workspace_bytes;    /* >= flashloop_decode_workspace_bytes(params) */
 } flashloop_decode_state;
 
-/* Scratch bytes of flashloop_decode_step / flashloop_decode_attn (host function).
+/* Scratch bytes of flashloop_decode_step / flashloop_decode_attn (host function;
+ * a sizing helper).
  * p->batch = B in [1, 64]; additionally n_heads*head_dim must be a multiple of
  * 256 and n_heads*head_dim/32 a divisor of 256 that is a multiple of 8
  * (e.g. 16 x 128, 4 x 64); returns 0 for any other shape. */
@@ -416,7 +425,8 @@ size_t flashloop_decode_workspace_bytes(const flashloop_params* p);
 int flashloop_decode_attn(const flashloop_params* p, int32_t loop, const flashloop_state* ctx,
                           flashloop_decode_state* ds, void* stream);
 
-/* (a8) Projections of the decode token at loop `loop`: q, k, v = x_tok W_qkv^T
+/* (a8) [FlashLoop App. G: the decode path] Projections of the decode token
+ * at loop `loop`: q, k, v = x_tok W_qkv^T
  * (x_tok bf16 [B, d_model], float32 accumulation, RoPE at position S on q and
  * k; q -> ds->q slot of the loop); k and v quantised into the token streams
  * (INT8 base at loop 1, the residual against the reconstructed previous loop
@@ -432,12 +442,13 @@ int flashloop_decode_qkv(const flashloop_params* p, int32_t loop, const uint16_t
  * workspace by flashloop_decode_attn (call it first).  Needs S + 1 <= 49152. */
 int flashloop_decode_select(const flashloop_params* p, flashloop_decode_state* ds, void* stream);
 
-/* (a8) Output projection of the decode tokens: Y = bf16(O W_o^T), float32
- * accumulation. */
+/* (a8) [FlashLoop App. G: the decode path] Output projection of the decode
+ * tokens: Y = bf16(O W_o^T), float32 accumulation. */
 int flashloop_decode_out(const flashloop_params* p, const uint16_t* w_o, flashloop_decode_state* ds,
                          void* stream);
 
-/* (a8) One loop of the decode token, B sequences: flashloop_decode_qkv,
+/* (a8) [FlashLoop App. G: the decode path, its sparse selection fused with
+ * the dense loop-1 pass] One loop of the decode token, B sequences: flashloop_decode_qkv,
  * flashloop_decode_attn, flashloop_decode_select (loop 1, when R >= 2),
  * flashloop_decode_out. */
 int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_t* x_tok,
@@ -445,11 +456,13 @@ int flashloop_decode_step(const flashloop_params* p, int32_t loop, const uint16_
                           flashloop_decode_state* ds, void* stream);
 
 /* Host helper: the loop whose selection loop r uses (2 <= r): the latest
- * loop l <= r with l == 2 or topk[l-1] < topk[l-2]. */
+ * loop l <= r with l == 2 or topk[l-1] < topk[l-2].  [FlashLoop §4.2: the
+ * selection is re-ranked when the column budget shrinks, and kept otherwise.] */
 int32_t flashloop_selection_loop(const flashloop_params* p, int32_t loop);
 
 /* Copy *err_word to the host (synchronising the stream) and map it to a
- * status: FLASHLOOP_OK, or FLASHLOOP_ERR_DEVICE with the code in *code. */
+ * status: FLASHLOOP_OK, or FLASHLOOP_ERR_DEVICE with the code in *code
+ * (diagnostics; not an operation of the method). */
 int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* stream);
 
 /* Self-test of the bounded waits that every pipelined kernel of the library
@@ -462,7 +475,7 @@ int flashloop_check_error_word(const int32_t* err_word, int32_t* code, void* str
  * Returns FLASHLOOP_ERR_INVALID_ARG for another kind or a NULL err_word. */
 int flashloop_selftest_bounded_wait(int32_t kind, int32_t* err_word, void* stream);
 
-/* Static description of a status code. */
+/* Static description of a status code (diagnostics). */
 const char* flashloop_status_string(int status);
 
 #ifdef __cplusplus
