@@ -178,16 +178,18 @@ __device__ __forceinline__ void at_mma_role(uint8_t* smem, const AtBars& B, uint
     int stage = 0;
     uint32_t phase = 0;
     uint32_t u = 0;        // global tile counter (S buffer = u & 1)
-    uint32_t item_no = 0;
+    uint32_t item_no = 0;  // items with tiles so far
     bool ok = true;
-    for (int item = blockIdx.x; item < total && ok && !*B.abort_flag; item += gridDim.x, ++item_no) {
+    for (int item = blockIdx.x; item < total && ok && !*B.abort_flag; item += gridDim.x) {
       const int h = item / row_tiles, rt = item % row_tiles;
       const int nt = at_tiles(g, h, rt, n_rows);
+      if (nt == 0) continue;  // the rows signal q_ready only for items with tiles
       if (!mbar_wait_sleep(B.q_ready, item_no & 1)) {
         set_error(g.err, kDevErrTimeout);
         *B.abort_flag = 1;
         break;
       }
+      ++item_no;
       tc_fence_after();
       int prev_stage = -1;
       for (int t = 0; t <= nt; ++t) {
@@ -425,7 +427,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_kn, const __grid_constant_
         }
         tmem_wait_st();
         tc_fence_before();
-        mbar_arrive(q_ready);
+        // only items with tiles: the MMA thread waits on q_ready for those
+        // alone, so the rows can never run two phases ahead of it
+        if (nt > 0) mbar_arrive(q_ready);
         // bring the next item's rows (this thread's q and half of N) into L2
         // while this item runs: they are the item switch's loads
         const int item_next = item + gridDim.x;

@@ -19,6 +19,9 @@ one the waiter wants, and that the schedule always makes progress.
   wait, the rescale wait on the other group's P.V (four barriers by t mod 4),
   the named-barrier hand-off of the running reference between the two row
   groups, and the q barrier used only by work items that have column tiles.
+- attn_tc_kernel (csrc/attn_tc.cu, the fixed-mass passes): one MMA thread
+  alternating S(t) and P(t-1).V over two score buffers, and its q barrier
+  used only by work items that have column tiles.
 - tc_gemm_kernel (csrc/gemm_tc.cu): the A/B stage ring filled by the
   gathering warps and TMA, the MMA thread, and the two TMEM accumulators the
   epilogue drains while the next tile fills.
@@ -542,6 +545,94 @@ def test_gemm_protocol_model_catches_a_planted_phase():
         rnd = random.Random(seed)
         try:
             gemm_cta(5, 3, 4, rnd, plant="acc_phase")
+        except (AssertionError, Stuck):
+            caught += 1
+    assert caught > 0
+
+
+# --------------------------------------------------------------- attn_tc_kernel
+def tc_cta(nts, stages, rnd, q_every_item=False):
+    """The column-split update kernel of the fixed-mass passes: one MMA thread
+    issues S(t) into score buffer t & 1, then P(t-1).V; all row threads take
+    every tile.  q_every_item models a q barrier completed by every item,
+    with or without column tiles."""
+    B = {}
+    for s in range(stages):
+        B[("kv_full", s)] = Bar(1)
+        B[("kv_empty", s)] = Bar(1)
+    for i in range(2):
+        B[("s_full", i)] = Bar(1)
+        B[("p_full", i)] = Bar(1)  # the row threads move together in the model
+        B[("pv_done", i)] = Bar(1)
+    B["q_ready"] = Bar(1)
+    loads, pipe = [], []
+
+    def loader():
+        fills = [0] * stages
+        u = 0
+        for nt in nts:
+            for _t in range(nt):
+                st = u % stages
+                yield from wait(B, ("kv_empty", st), fills[st] - 1)
+                loads.append(("kv_full", st))
+                fills[st] += 1
+                u += 1
+
+    def mma():
+        u = item_no = 0
+        for nt in nts:
+            if not q_every_item and nt == 0:
+                continue
+            yield from wait(B, "q_ready", item_no)
+            item_no += 1
+            for _ in range(rnd.randint(0, 30)):  # a late MMA thread
+                yield None
+            prev_stage = -1
+            for t in range(nt + 1):
+                if t < nt:
+                    yield from wait(B, ("kv_full", u % stages), u // stages)
+                    pipe.extend([("mma", None), ("commit", ("s_full", u & 1))])
+                if t > 0:
+                    up = u - 1
+                    yield from wait(B, ("p_full", up & 1), up >> 1)
+                    pipe.extend([("mma", None), ("commit", ("kv_empty", prev_stage)),
+                                 ("commit", ("pv_done", up & 1))])
+                if t < nt:
+                    prev_stage = u % stages
+                    u += 1
+
+    def rows():
+        u = 0
+        for nt in nts:
+            if q_every_item or nt > 0:
+                B["q_ready"].arrive()
+            for t in range(nt):
+                yield from wait(B, ("s_full", u & 1), u >> 1)
+                if t > 0 and rnd.random() < 0.3:  # the reference rose: N waits for P(t-1).V
+                    yield from wait(B, ("pv_done", (u - 1) & 1), (u - 1) >> 1)
+                for _ in range(rnd.randint(0, 3)):
+                    yield None
+                B[("p_full", u & 1)].arrive()
+                u += 1
+            if nt > 0:
+                yield from wait(B, ("pv_done", (u - 1) & 1), (u - 1) >> 1)
+
+    run_schedule(B, [loader(), mma(), rows()], loads, pipe, rnd, idle_limit=5000)
+
+
+def test_tc_protocol_phases_and_progress():
+    for seed in range(300):
+        rnd = random.Random(seed)
+        tc_cta(_pp_items(rnd), 3, rnd)
+
+
+def test_tc_protocol_model_catches_a_q_barrier_on_empty_items():
+    caught = 0
+    for seed in range(300):
+        rnd = random.Random(seed)
+        items = [rnd.choice([0, 0, 1, 2, 3]) for _ in range(rnd.randint(2, 8))]
+        try:
+            tc_cta(items, 3, rnd, q_every_item=True)
         except (AssertionError, Stuck):
             caught += 1
     assert caught > 0
